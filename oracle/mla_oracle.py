@@ -1,0 +1,305 @@
+"""CPU oracle for decode-time Multi-head Latent Attention (MLA).
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import this module.  The CUDA library never
+calls it, and it shares no code with the CUDA library.
+
+Everything is plain NumPy in float64.  Each function follows the equations of
+the pages, written out directly:
+
+* "DeepSeek-V3 Technical Report" reading note (dogely.com), section on MLA:
+  c^KV_t = W^DKV h_t;  k^C_t = W^UK c^KV_t;  k^R_t = RoPE(W^KR h_t);
+  k_{t,i} = [k^C_{t,i}; k^R_t];  v^C_t = W^UV c^KV_t;
+  c^Q_t = W^DQ h_t;  q^C_t = W^UQ c^Q_t;  q^R_t = RoPE(W^QR c^Q_t);
+  q_{t,i} = [q^C_{t,i}; q^R_{t,i}];
+  o_{t,i} = sum_{j=1..t} Softmax_j(q_{t,i}^T k_{j,i} / sqrt(d_h + d_h^R)) v^C_{j,i};
+  u_t = W^O [o_{t,1}; ...; o_{t,n_h}].
+* "DeepSeek-V2: Strong, Economical, Efficient" (Chinese translation,
+  wiki.maxwellmou.com), §2.1.2 (only c^KV is cached), §2.1.3 (decoupled RoPE:
+  a shared k^R_t of width d_h^R is cached too, so a token costs
+  (d_c + d_h^R) elements per layer), Appendix B (V2-Lite computes the query
+  directly from h_t), Appendix C (W^UK can be absorbed into the query side and
+  W^UV into the output side by associativity).
+
+Readings of points the pages leave open (each is listed in the design doc):
+
+* RoPE follows the RoFormer form the pages cite (Su et al.): consecutive pairs
+  (x_{2k}, x_{2k+1}) rotated by angle p * theta_k, theta_k = base^(-2k/d_h^R),
+  base 10000, rotation [[cos, -sin], [sin, cos]].
+* The query of a decode step sits at position ctx-1 and its own key is in the
+  cache, so the softmax runs over positions 0 .. ctx-1 (the sum over j = 1..t).
+* ctx = 0 yields a zero output and log-sum-exp = -inf.
+* The log-sum-exp reported with an output is over the scaled scores
+  s_j = q^T k_j / sqrt(d_h + d_h^R), in natural-log units.
+
+Parity pins: every function below is pinned by tests/test_oracle_pins.py
+(closed forms, invariants, brute force, the pages' printed cache sizes).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+F64 = np.float64
+
+
+# ----------------------------------------------------------------------------
+# RoPE (decoupled part only)
+# ----------------------------------------------------------------------------
+
+def rope_theta(d_r: int, base: float) -> np.ndarray:
+    """theta_k = base^(-2k/d_r) for k = 0 .. d_r/2 - 1 (RoFormer frequencies)."""
+    k = np.arange(d_r // 2, dtype=F64)
+    return np.power(F64(base), -2.0 * k / F64(d_r))
+
+
+def rope(x: np.ndarray, pos, base: float) -> np.ndarray:
+    """Rotate consecutive pairs of the last axis of ``x`` by pos * theta_k.
+
+    ``pos`` is a scalar or an array broadcastable to x.shape[:-1].
+    """
+    x = np.asarray(x, dtype=F64)
+    d_r = x.shape[-1]
+    assert d_r % 2 == 0
+    theta = rope_theta(d_r, base)
+    ang = np.asarray(pos, dtype=F64)[..., None] * theta          # [..., d_r/2]
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty(np.broadcast_shapes(x.shape, ang.shape[:-1] + (d_r,)), dtype=F64)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
+
+
+# ----------------------------------------------------------------------------
+# cache (what a token leaves behind)
+# ----------------------------------------------------------------------------
+
+def cache_rows(h: np.ndarray, w_dkv: np.ndarray, w_kr: np.ndarray, positions,
+               base: float) -> np.ndarray:
+    """Cached row of each token: [c^KV_t ; k^R_t] with c^KV_t = W^DKV h_t and
+    k^R_t = RoPE(W^KR h_t) at the token's position.  h: [T, d] -> [T, d_c + d_r]."""
+    h = np.asarray(h, dtype=F64)
+    c = h @ np.asarray(w_dkv, dtype=F64).T
+    kr = rope(h @ np.asarray(w_kr, dtype=F64).T, np.asarray(positions), base)
+    return np.concatenate([c, kr], axis=-1)
+
+
+def kv_cache_elements_per_token(kind: str, *, n_h: int, d_h: int, layers: int = 1,
+                                n_g: int = 0, d_c: int = 0, d_r: int = 0) -> int:
+    """Per-token KV-cache size in elements for the mechanisms the pages compare
+    (V2 paper §2.1.4, Table 1): MHA 2 n_h d_h l, GQA 2 n_g d_h l, MQA 2 d_h l,
+    MLA (d_c + d_h^R) l."""
+    if kind == "MHA":
+        return 2 * n_h * d_h * layers
+    if kind == "GQA":
+        return 2 * n_g * d_h * layers
+    if kind == "MQA":
+        return 2 * d_h * layers
+    if kind == "MLA":
+        return (d_c + d_r) * layers
+    raise ValueError(kind)
+
+
+# ----------------------------------------------------------------------------
+# query (upstream of the decode boundary; used by oracle-only cross-checks)
+# ----------------------------------------------------------------------------
+
+def query_from_hidden(h_q: np.ndarray, qw: dict, n_h: int, d_h: int, d_r: int):
+    """q^C and q^R before rotation for one token, shapes [n_h, d_h], [n_h, d_r].
+
+    With query compression: c^Q = W^DQ h, q^C = W^UQ c^Q, q^R_raw = W^QR c^Q.
+    Without (V2-Lite, Appendix B): q^C = W^Q h, q^R_raw = W^QR h."""
+    h_q = np.asarray(h_q, dtype=F64)
+    if "w_dq" in qw:
+        cq = np.asarray(qw["w_dq"], F64) @ h_q
+        qc = np.asarray(qw["w_uq"], F64) @ cq
+        qr = np.asarray(qw["w_qr"], F64) @ cq
+    else:
+        qc = np.asarray(qw["w_q"], F64) @ h_q
+        qr = np.asarray(qw["w_qr"], F64) @ h_q
+    return qc.reshape(n_h, d_h), qr.reshape(n_h, d_r)
+
+
+# ----------------------------------------------------------------------------
+# explicit (textbook) attention: per-head keys and values are materialised
+# ----------------------------------------------------------------------------
+
+def explicit_keys_values(rows: np.ndarray, w_uk: np.ndarray, w_uv: np.ndarray,
+                         n_h: int, d_h: int, d_c: int, heads=None):
+    """k_{j,i} = [W^UK_i c_j ; k^R_j] and v_{j,i} = W^UV_i c_j, where W^UK_i is
+    rows i*d_h .. (i+1)*d_h of W^UK.  rows: [S, d_c + d_r].
+    Returns k [h, S, d_h + d_r], v [h, S, d_h] for the selected heads."""
+    rows = np.asarray(rows, dtype=F64)
+    c, kr = rows[:, :d_c], rows[:, d_c:]
+    heads = range(n_h) if heads is None else heads
+    ks, vs = [], []
+    for i in heads:
+        wk = np.asarray(w_uk[i * d_h:(i + 1) * d_h], dtype=F64)     # [d_h, d_c]
+        wv = np.asarray(w_uv[i * d_h:(i + 1) * d_h], dtype=F64)
+        ks.append(np.concatenate([c @ wk.T, kr], axis=1))
+        vs.append(c @ wv.T)
+    return np.stack(ks), np.stack(vs)
+
+
+def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Textbook attention for one query per head.  q [h, e], k [h, S, e],
+    v [h, S, f] -> (o [h, f], lse [h]); lse is log sum_j exp(scale q.k_j)."""
+    q, k, v = (np.asarray(a, dtype=F64) for a in (q, k, v))
+    S = k.shape[1]
+    if S == 0:
+        return np.zeros((q.shape[0], v.shape[2])), np.full(q.shape[0], -np.inf)
+    s = np.einsum("he,hse->hs", q, k) * F64(scale)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    o = np.einsum("hs,hsf->hf", p / l, v)
+    return o, (m + np.log(l))[:, 0]
+
+
+def softmax_scale(d_h: int, d_r: int) -> float:
+    """1 / sqrt(d_h + d_h^R): the scores divide by the root of the full
+    (content + rotary) query/key width."""
+    return 1.0 / math.sqrt(d_h + d_r)
+
+
+def mla_decode_explicit(q_nope, q_rope_raw, pos: int, rows, w_uk, w_uv, *, n_h, d_h, d_c,
+                        d_r, base, heads=None):
+    """One decode step for one sequence in the explicit form.
+    q_nope [n_h, d_h], q_rope_raw [n_h, d_r] (before RoPE), rows [S, d_c+d_r].
+    Returns (o [h, d_h], lse [h]) for the selected heads."""
+    heads = list(range(n_h)) if heads is None else list(heads)
+    qr = rope(np.asarray(q_rope_raw, F64)[heads], pos, base)
+    q = np.concatenate([np.asarray(q_nope, F64)[heads], qr], axis=1)
+    k, v = explicit_keys_values(rows, w_uk, w_uv, n_h, d_h, d_c, heads)
+    return softmax_attention(q, k, v, softmax_scale(d_h, d_r))
+
+
+# ----------------------------------------------------------------------------
+# absorbed form (Appendix C): attention runs on the cached rows directly
+# ----------------------------------------------------------------------------
+
+def absorb_query(q_nope, q_rope_raw, pos: int, w_uk, *, n_h, d_h, d_r, base) -> np.ndarray:
+    """q_abs_i = [W^UK_i^T q^C_i ; RoPE(q^R_i, pos)]  -> [n_h, d_c + d_r].
+    Then q_abs_i . [c_j ; k^R_j] = q^C_i . (W^UK_i c_j) + q^R_i . k^R_j."""
+    q_nope = np.asarray(q_nope, F64)
+    out = []
+    for i in range(n_h):
+        wk = np.asarray(w_uk[i * d_h:(i + 1) * d_h], F64)           # [d_h, d_c]
+        out.append(wk.T @ q_nope[i])
+    lat = np.stack(out)
+    return np.concatenate([lat, rope(np.asarray(q_rope_raw, F64), pos, base)], axis=1)
+
+
+def latent_attention(q_abs, rows, *, d_c: int, scale: float):
+    """Softmax over the latent rows: ctx_lat_i = sum_j p_ij c_j with
+    p_ij = softmax_j(scale q_abs_i . row_j).  Returns (ctx_lat [h, d_c], lse [h])."""
+    q_abs, rows = np.asarray(q_abs, F64), np.asarray(rows, F64)
+    if rows.shape[0] == 0:
+        return np.zeros((q_abs.shape[0], d_c)), np.full(q_abs.shape[0], -np.inf)
+    s = (q_abs @ rows.T) * F64(scale)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p / l) @ rows[:, :d_c], (m + np.log(l))[:, 0]
+
+
+def out_project(ctx_lat, w_uv, *, n_h, d_h, w_o=None):
+    """o_i = W^UV_i ctx_lat_i (W^UV absorbed to the output side), and optionally
+    u = W^O [o_1; ...; o_{n_h}]."""
+    ctx_lat = np.asarray(ctx_lat, F64)
+    o = np.stack([np.asarray(w_uv[i * d_h:(i + 1) * d_h], F64) @ ctx_lat[i]
+                  for i in range(n_h)])
+    if w_o is None:
+        return o, None
+    return o, np.asarray(w_o, F64) @ o.reshape(-1)
+
+
+def mla_decode_absorbed(q_nope, q_rope_raw, pos, rows, w_uk, w_uv, *, n_h, d_h, d_c, d_r,
+                        base, w_o=None):
+    """Full absorbed decode step for one sequence: returns dict with q_abs,
+    ctx_lat, lse, o (and u when W^O is given)."""
+    q_abs = absorb_query(q_nope, q_rope_raw, pos, w_uk, n_h=n_h, d_h=d_h, d_r=d_r, base=base)
+    ctx_lat, lse = latent_attention(q_abs, rows, d_c=d_c, scale=softmax_scale(d_h, d_r))
+    o, u = out_project(ctx_lat, w_uv, n_h=n_h, d_h=d_h, w_o=w_o)
+    return {"q_abs": q_abs, "ctx_lat": ctx_lat, "lse": lse, "o": o, "u": u}
+
+
+# ----------------------------------------------------------------------------
+# split-KV partials and their log-sum-exp merge
+# ----------------------------------------------------------------------------
+
+def split_partials(q_abs, rows, bounds, *, d_c: int, scale: float):
+    """Attention over each token range [a, b) of ``bounds`` separately:
+    list of (ctx_lat_part [h, d_c], lse_part [h])."""
+    return [latent_attention(q_abs, np.asarray(rows)[a:b], d_c=d_c, scale=scale)
+            for a, b in bounds]
+
+
+def combine_partials(parts):
+    """Merge per-range results: with m = max_s lse_s and w_s = exp(lse_s - m),
+    ctx = sum_s w_s ctx_s / sum_s w_s and lse = m + log sum_s w_s.  Ranges with
+    lse = -inf carry no weight; if all are -inf the result is 0 and -inf."""
+    lses = np.stack([p[1] for p in parts])                      # [S, h]
+    outs = np.stack([p[0] for p in parts])                      # [S, h, d]
+    m = lses.max(axis=0)
+    finite = np.isfinite(m)
+    msafe = np.where(finite, m, 0.0)
+    w = np.where(np.isfinite(lses), np.exp(lses - msafe), 0.0)
+    tot = w.sum(axis=0)
+    ctx = np.einsum("sh,shd->hd", w, outs) / np.where(tot > 0, tot, 1.0)[:, None]
+    lse = np.where(finite, msafe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return np.where(finite[:, None], ctx, 0.0), lse
+
+
+# ----------------------------------------------------------------------------
+# brute force (pure Python loops) for tiny inputs
+# ----------------------------------------------------------------------------
+
+def brute_force_decode(h_seq, q_nope, q_rope_raw, w: dict, *, n_h, d_h, d_c, d_r, base):
+    """Scalar-loop decode step for one sequence from its hidden states:
+    builds every cached row, every per-head key/value, and the softmax, one
+    multiply-add at a time.  Returns (o as nested lists [n_h][d_h], lse list [n_h])."""
+    S = len(h_seq)
+    d = len(h_seq[0])
+    rows = []
+    for t in range(S):
+        c = [sum(float(w["w_dkv"][r][k]) * float(h_seq[t][k]) for k in range(d))
+             for r in range(d_c)]
+        kr_raw = [sum(float(w["w_kr"][r][k]) * float(h_seq[t][k]) for k in range(d))
+                  for r in range(d_r)]
+        kr = [0.0] * d_r
+        for p in range(d_r // 2):
+            th = base ** (-2.0 * p / d_r)
+            a = t * th
+            kr[2 * p] = kr_raw[2 * p] * math.cos(a) - kr_raw[2 * p + 1] * math.sin(a)
+            kr[2 * p + 1] = kr_raw[2 * p] * math.sin(a) + kr_raw[2 * p + 1] * math.cos(a)
+        rows.append((c, kr))
+    pos = S - 1
+    out, lses = [], []
+    for i in range(n_h):
+        qr = [0.0] * d_r
+        for p in range(d_r // 2):
+            a = pos * base ** (-2.0 * p / d_r)
+            x0, x1 = float(q_rope_raw[i][2 * p]), float(q_rope_raw[i][2 * p + 1])
+            qr[2 * p] = x0 * math.cos(a) - x1 * math.sin(a)
+            qr[2 * p + 1] = x0 * math.sin(a) + x1 * math.cos(a)
+        scores, vals = [], []
+        for t in range(S):
+            c, kr = rows[t]
+            kc = [sum(float(w["w_uk"][i * d_h + r][k]) * c[k] for k in range(d_c))
+                  for r in range(d_h)]
+            vc = [sum(float(w["w_uv"][i * d_h + r][k]) * c[k] for k in range(d_c))
+                  for r in range(d_h)]
+            dot = sum(float(q_nope[i][r]) * kc[r] for r in range(d_h))
+            dot += sum(qr[r] * kr[r] for r in range(d_r))
+            scores.append(dot / math.sqrt(d_h + d_r))
+            vals.append(vc)
+        mx = max(scores)
+        e = [math.exp(s - mx) for s in scores]
+        z = sum(e)
+        out.append([sum(e[t] * vals[t][r] for t in range(S)) / z for r in range(d_h)])
+        lses.append(mx + math.log(z))
+    return out, lses

@@ -1,0 +1,311 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other
+than itself -- values the pages print, closed forms, invariants of the
+mathematics, brute force on tiny inputs -- so that a dropped term, a wrong sign
+or index, or a transposed operand fails at least one of them."""
+
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import mla_oracle as O
+from workloads import WORKLOADS, draw_query_weights, draw_weights, hidden_states, queries
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TINY = WORKLOADS["tiny_fp32"]
+
+
+def _golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                key, val = line.split()[:2]
+                out[key] = float(val)
+    return out
+
+
+def _rel(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# --------------------------------------------------------------------------
+# cache size: the pages print it
+# --------------------------------------------------------------------------
+
+def test_cache_size_matches_pages():
+    g = _golden("kv_cache_per_token.txt")
+    n_h, d_h, d_c, d_r = (int(g[k]) for k in ("v2_n_h", "v2_d_h", "v2_d_c", "v2_d_r"))
+    assert d_c == g["d_c_per_d_h"] * d_h
+    assert d_r == g["d_r_per_d_h"] * d_h
+    mla = O.kv_cache_elements_per_token("MLA", n_h=n_h, d_h=d_h, d_c=d_c, d_r=d_r)
+    assert mla == g["mla_per_d_h"] * d_h == 576
+    gqa = O.kv_cache_elements_per_token("GQA", n_h=n_h, d_h=d_h, n_g=1)
+    assert mla / gqa == g["mla_gqa_groups"]
+    mha = O.kv_cache_elements_per_token("MHA", n_h=n_h, d_h=d_h, layers=int(g["v2_layers"]))
+    assert O.kv_cache_elements_per_token("MLA", n_h=n_h, d_h=d_h, d_c=d_c, d_r=d_r,
+                                         layers=int(g["v2_layers"])) / mha == 576 / 32768
+    assert O.kv_cache_elements_per_token("MQA", n_h=n_h, d_h=d_h) == 2 * d_h
+    # the oracle's cached row has exactly d_c + d_h^R entries
+    rng = np.random.default_rng(0)
+    d = 64
+    rows = O.cache_rows(rng.standard_normal((3, d)), rng.standard_normal((d_c, d)),
+                        rng.standard_normal((d_r, d)), np.arange(3), 10000.0)
+    assert rows.shape == (3, mla)
+    # V2-Lite shares the per-token row width
+    assert int(g["lite_d_c"]) + int(g["lite_d_r"]) == mla
+
+
+# --------------------------------------------------------------------------
+# RoPE: hand values of the RoFormer rotation, and its invariants
+# --------------------------------------------------------------------------
+
+def test_rope_hand_values():
+    # d = 2: one pair, theta_0 = 1.  Position 1 rotates by one radian.
+    assert np.allclose(O.rope([1.0, 0.0], 1, 10000.0), [math.cos(1), math.sin(1)], atol=1e-15)
+    assert np.allclose(O.rope([0.0, 1.0], 1, 10000.0), [-math.sin(1), math.cos(1)], atol=1e-15)
+    # d = 4, base 10000: theta_1 = 10000^(-1/2) = 0.01, so position 100 turns pair 1 by 1 rad
+    # and pair 0 by 100 rad.
+    x = O.rope([1.0, 0.0, 1.0, 0.0], 100, 10000.0)
+    assert np.allclose(x, [math.cos(100), math.sin(100), math.cos(1), math.sin(1)], atol=1e-13)
+    # position 0 is the identity
+    v = np.arange(16.0)
+    assert np.array_equal(O.rope(v, 0, 10000.0), v)
+
+
+def test_rope_preserves_norm():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((50, 64))
+    pos = rng.integers(0, 131072, size=50)
+    y = O.rope(x, pos, 10000.0)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    rng = np.random.default_rng(2)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for m, n in [(0, 5), (17, 3), (131071, 130000)]:
+        ref = O.rope(q, m, 10000.0) @ O.rope(k, n, 10000.0)
+        for delta in (1, 977, 4096):
+            got = O.rope(q, m + delta, 10000.0) @ O.rope(k, n + delta, 10000.0)
+            assert abs(got - ref) <= 1e-9 * max(1.0, abs(ref))
+
+
+# --------------------------------------------------------------------------
+# absorbed form == explicit form (associativity), and why RoPE is decoupled
+# --------------------------------------------------------------------------
+
+def _tiny_inputs(seed=0, S=23):
+    wl = TINY
+    rng = np.random.default_rng(seed)
+    w = draw_weights(wl)
+    rows = rng.standard_normal((S, wl.D))
+    qn = rng.standard_normal((wl.n_h, wl.d_h))
+    qr = rng.standard_normal((wl.n_h, wl.d_r))
+    return wl, w, rows, qn, qr
+
+
+def test_absorbed_equals_explicit():
+    wl, w, rows, qn, qr = _tiny_inputs()
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base)
+    o_e, lse_e = O.mla_decode_explicit(qn, qr, 22, rows, w["w_uk"], w["w_uv"], **kw)
+    res = O.mla_decode_absorbed(qn, qr, 22, rows, w["w_uk"], w["w_uv"], **kw)
+    assert _rel(res["o"], o_e) <= 1e-12
+    assert np.allclose(res["lse"], lse_e, rtol=1e-13, atol=1e-13)
+
+
+def test_absorption_fails_if_rope_touches_content_keys():
+    """Rotating k^C (coupled RoPE) puts a position-dependent matrix between
+    W^Q and W^UK, so the absorbed form no longer matches: the oracle's
+    absorbed form must notice the difference."""
+    wl, w, rows, qn, qr = _tiny_inputs(seed=3)
+    d_h, d_c = wl.d_h, wl.d_c
+    S = rows.shape[0]
+    k_exp, v_exp = O.explicit_keys_values(rows, w["w_uk"], w["w_uv"], wl.n_h, d_h, d_c)
+    k_coupled = k_exp.copy()
+    k_coupled[:, :, :d_h] = O.rope(k_exp[:, :, :d_h], np.arange(S)[None, :], wl.rope_base)
+    q = np.concatenate([qn, O.rope(qr, S - 1, wl.rope_base)], axis=1)
+    o_coupled, _ = O.softmax_attention(q, k_coupled, v_exp, O.softmax_scale(d_h, wl.d_r))
+    res = O.mla_decode_absorbed(qn, qr, S - 1, rows, w["w_uk"], w["w_uv"], n_h=wl.n_h, d_h=d_h,
+                                d_c=d_c, d_r=wl.d_r, base=wl.rope_base)
+    assert _rel(res["o"], o_coupled) > 1e-3
+
+
+# --------------------------------------------------------------------------
+# closed forms of the softmax and its scale
+# --------------------------------------------------------------------------
+
+def _one_head_setup(d_h=32, d_c=128, d_r=16):
+    """W^UK_0 = W^UV_0 = [I_{d_h} 0] so that the per-head key/value of a row
+    are its first d_h latent entries."""
+    w_uk = np.zeros((d_h, d_c))
+    w_uk[:, :d_h] = np.eye(d_h)
+    return w_uk, w_uk.copy()
+
+
+def test_two_token_softmax_closed_form():
+    """Scores that differ by ln(3) give weights 3/4 and 1/4 -- the scale must be
+    1/sqrt(d_h + d_h^R)."""
+    d_h, d_c, d_r = 32, 128, 16
+    w_uk, w_uv = _one_head_setup(d_h, d_c, d_r)
+    gap = math.log(3.0) * math.sqrt(d_h + d_r)      # raw dot-product difference
+    rows = np.zeros((2, d_c + d_r))
+    rows[0, 0] = gap            # key 0 content: e_0 * gap
+    rows[0, 1] = 5.0            # value 0: 5 in coordinate 1
+    rows[1, 2] = -7.0           # value 1: -7 in coordinate 2, score 0
+    qn = np.zeros((1, d_h))
+    qn[0, 0] = 1.0
+    qr = np.zeros((1, d_r))
+    o, lse = O.mla_decode_explicit(qn, qr, 1, rows, w_uk, w_uv, n_h=1, d_h=d_h, d_c=d_c,
+                                   d_r=d_r, base=10000.0)
+    assert np.isclose(o[0, 0], 0.75 * gap, rtol=1e-14)
+    assert np.isclose(o[0, 1], 0.75 * 5.0, rtol=1e-14)
+    assert np.isclose(o[0, 2], 0.25 * -7.0, rtol=1e-14)
+    # lse = log(e^{ln 3} + e^0) = log 4
+    assert np.isclose(lse[0], math.log(4.0), rtol=1e-14)
+
+
+def test_rope_part_enters_scores():
+    """Only the decoupled parts differ: q^R = k^R_0 rotated to the same place
+    gives score |k^R|^2 / sqrt(d_h + d_r) for key 0 and 0 for key 1."""
+    d_h, d_c, d_r = 32, 128, 16
+    w_uk, w_uv = _one_head_setup(d_h, d_c, d_r)
+    rows = np.zeros((2, d_c + d_r))
+    kr = np.zeros(d_r)
+    kr[0] = math.sqrt(math.log(3.0) * math.sqrt(d_h + d_r))   # |k^R|^2 = ln3 sqrt(48)
+    rows[0, d_c:] = O.rope(kr, 0, 10000.0)
+    rows[0, 1], rows[1, 1] = 1.0, 0.0
+    # query at position 1 whose rotated q^R equals kr rotated by 0: pre-rotate by -1
+    qr = O.rope(kr, -1, 10000.0)[None, :]
+    qn = np.zeros((1, d_h))
+    o, _ = O.mla_decode_explicit(qn, qr, 1, rows, w_uk, w_uv, n_h=1, d_h=d_h, d_c=d_c, d_r=d_r,
+                                 base=10000.0)
+    assert np.isclose(o[0, 1], 0.75, rtol=1e-12)
+
+
+def test_ctx1_constant_and_zero_query():
+    wl, w, rows, qn, qr = _tiny_inputs(seed=5, S=9)
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base)
+    wuv = w["w_uv"].astype(np.float64)
+    per_head = lambda c: np.stack([wuv[i * wl.d_h:(i + 1) * wl.d_h] @ c for i in range(wl.n_h)])
+    # ctx = 1: the only value is returned
+    o, lse = O.mla_decode_explicit(qn, qr, 0, rows[:1], w["w_uk"], w["w_uv"], **kw)
+    assert _rel(o, per_head(rows[0, :wl.d_c])) <= 1e-13
+    # all rows equal: softmax weights are uniform, output is that value; lse = s + log S
+    same = np.repeat(rows[:1], 9, axis=0)
+    o, lse = O.mla_decode_explicit(qn, qr, 8, same, w["w_uk"], w["w_uv"], **kw)
+    assert _rel(o, per_head(rows[0, :wl.d_c])) <= 1e-13
+    # q = 0: uniform weights -> mean of the values, lse = log S
+    o, lse = O.mla_decode_explicit(np.zeros_like(qn), np.zeros_like(qr), 8, rows, w["w_uk"],
+                                   w["w_uv"], **kw)
+    assert _rel(o, per_head(rows[:, :wl.d_c].mean(axis=0))) <= 1e-13
+    assert np.allclose(lse, math.log(9), rtol=1e-14)
+
+
+def test_dominant_key_wins():
+    d_h, d_c, d_r = 32, 128, 16
+    w_uk, w_uv = _one_head_setup(d_h, d_c, d_r)
+    rng = np.random.default_rng(9)
+    rows = rng.standard_normal((40, d_c + d_r)) * 0.1
+    rows[13, 0] = 400.0
+    qn = np.zeros((1, d_h))
+    qn[0, 0] = 1.0
+    o, _ = O.mla_decode_explicit(qn, np.zeros((1, d_r)), 39, rows, w_uk, w_uv, n_h=1, d_h=d_h,
+                                 d_c=d_c, d_r=d_r, base=10000.0)
+    assert np.allclose(o[0], rows[13, :d_h], atol=1e-12)
+
+
+def test_empty_context():
+    wl, w, rows, qn, qr = _tiny_inputs()
+    q_abs = O.absorb_query(qn, qr, 0, w["w_uk"], n_h=wl.n_h, d_h=wl.d_h, d_r=wl.d_r,
+                           base=wl.rope_base)
+    ctx, lse = O.latent_attention(q_abs, rows[:0], d_c=wl.d_c, scale=0.1)
+    assert np.all(ctx == 0) and np.all(np.isneginf(lse))
+
+
+# --------------------------------------------------------------------------
+# split-KV: any partition merged by log-sum-exp equals one pass
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cuts", [(0, 64), (0, 1, 64), (0, 10, 11, 40, 64), (0, 0, 30, 30, 64)])
+def test_split_combine_is_exact(cuts):
+    rng = np.random.default_rng(11)
+    H, d_c, d_r = 4, 128, 16
+    rows = rng.standard_normal((64, d_c + d_r))
+    q_abs = rng.standard_normal((H, d_c + d_r))
+    scale = O.softmax_scale(32, d_r)
+    full_ctx, full_lse = O.latent_attention(q_abs, rows, d_c=d_c, scale=scale)
+    parts = O.split_partials(q_abs, rows, list(zip(cuts[:-1], cuts[1:])), d_c=d_c, scale=scale)
+    ctx, lse = O.combine_partials(parts)
+    assert _rel(ctx, full_ctx) <= 1e-13
+    assert np.allclose(lse, full_lse, rtol=1e-14)
+
+
+def test_combine_all_empty():
+    parts = [(np.zeros((2, 8)), np.full(2, -np.inf))] * 3
+    ctx, lse = O.combine_partials(parts)
+    assert np.all(ctx == 0) and np.all(np.isneginf(lse))
+
+
+# --------------------------------------------------------------------------
+# brute force on the tiny workload, from hidden states to outputs
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b", [0, 1])
+def test_brute_force_tiny_workload(b):
+    wl = TINY
+    w = draw_weights(wl)
+    ctx = wl.ctx[b]
+    h = hidden_states(wl, b, ctx)
+    qn, qr = queries(wl)
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base)
+    rows = O.cache_rows(h, w["w_dkv"], w["w_kr"], np.arange(ctx), wl.rope_base)
+    res = O.mla_decode_absorbed(qn[b], qr[b], ctx - 1, rows, w["w_uk"], w["w_uv"], **kw)
+    o_ex, lse_ex = O.mla_decode_explicit(qn[b], qr[b], ctx - 1, rows, w["w_uk"], w["w_uv"], **kw)
+    bf_o, bf_lse = O.brute_force_decode(h.tolist(), qn[b].tolist(), qr[b].tolist(),
+                                        {k: v.tolist() for k, v in w.items()}, **kw)
+    assert _rel(res["o"], bf_o) <= 1e-12
+    assert _rel(o_ex, bf_o) <= 1e-12
+    assert np.allclose(res["lse"], bf_lse, rtol=1e-12)
+
+
+def test_full_equations_with_query_compression():
+    """From h through c^Q, q^C, q^R (V3 note equations) to o: explicit and
+    absorbed agree, and u = W^O [o_1; ...; o_n] is the per-element sum."""
+    wl = TINY
+    w = draw_weights(wl, with_wo=True)
+    qw = draw_query_weights(wl)
+    ctx = wl.ctx[1]
+    h = hidden_states(wl, 1, ctx)
+    qc, qr = O.query_from_hidden(h[-1], qw, wl.n_h, wl.d_h, wl.d_r)
+    # c^Q path by hand for one element
+    cq = np.asarray(qw["w_dq"], np.float64) @ h[-1].astype(np.float64)
+    assert np.isclose(qc[2, 5], np.asarray(qw["w_uq"], np.float64)[2 * wl.d_h + 5] @ cq)
+    rows = O.cache_rows(h, w["w_dkv"], w["w_kr"], np.arange(ctx), wl.rope_base)
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base)
+    res = O.mla_decode_absorbed(qc, qr, ctx - 1, rows, w["w_uk"], w["w_uv"], w_o=w["w_o"], **kw)
+    o_ex, _ = O.mla_decode_explicit(qc, qr, ctx - 1, rows, w["w_uk"], w["w_uv"], **kw)
+    assert _rel(res["o"], o_ex) <= 1e-12
+    wo = np.asarray(w["w_o"], np.float64)
+    flat = res["o"].reshape(-1)
+    for j in (0, 77, wl.d_model - 1):
+        assert np.isclose(res["u"][j], sum(wo[j, k] * flat[k] for k in range(flat.size)),
+                          rtol=1e-12)
+
+
+def test_cache_rows_by_hand():
+    """One cached row element by element: c = W^DKV h, k^R = RoPE(W^KR h, p)."""
+    rng = np.random.default_rng(4)
+    d, d_c, d_r, p = 12, 6, 4, 7
+    h = rng.standard_normal((1, d))
+    wd, wk = rng.standard_normal((d_c, d)), rng.standard_normal((d_r, d))
+    row = O.cache_rows(h, wd, wk, [p], 10000.0)[0]
+    assert np.allclose(row[:d_c], [sum(wd[r, k] * h[0, k] for k in range(d)) for r in range(d_c)])
+    raw = [sum(wk[r, k] * h[0, k] for k in range(d)) for r in range(d_r)]
+    a0, a1 = p * 1.0, p * 10000.0 ** (-0.5)
+    want = [raw[0] * math.cos(a0) - raw[1] * math.sin(a0), raw[0] * math.sin(a0) + raw[1] * math.cos(a0),
+            raw[2] * math.cos(a1) - raw[3] * math.sin(a1), raw[2] * math.sin(a1) + raw[3] * math.cos(a1)]
+    assert np.allclose(row[d_c:], want, atol=1e-13)
