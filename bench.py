@@ -1,0 +1,397 @@
+#!/usr/bin/env python3
+"""Benchmark of one MLA decode step (append, absorb, split attention, combine,
+output projection) on DeepSeek-V2 attention shapes: B = 64 sequences,
+n_h = 128, ctx = 8192, bf16 latent cache [64, 8192, 576].
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is the whole step's algorithmic HBM
+traffic (latent cache read once plus the weights) per second, summed over all
+ranks (weak scaling: each rank runs its own batch); `ms_per_step` is the max
+over ranks.  `roofline` is the attention call timed on its own stream with
+CUDA events inside the timed region.  `e2e` repeats the step through the same
+C ABI from pinned host buffers, the per-step host->device and device->host
+copies inside the timed region.  `cpu_baseline` times the CPU oracle on a
+bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import signal
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "v2_b64_ctx8k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--num-parts", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1400.0, "fallback"
+
+
+def algorithmic_bytes(wl, ctx_sum, with_wo=False):
+    """Bytes one step must move at least: the latent cache once (sum ctx * D *
+    2) plus every weight once (W_DKV, W_KR, W_UK, W_UV [, W_O])."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    w = (wl.d_c + wl.d_r) * wl.d_model + 2 * wl.n_h * wl.d_h * wl.d_c
+    if with_wo:
+        w += wl.d_model * wl.n_h * wl.d_h
+    return ctx_sum * wl.D * esz + w * esz
+
+
+def algorithmic_flops(wl, ctx_sum):
+    attn = 2 * wl.n_h * ctx_sum * (wl.D + wl.d_c)
+    gemms = 2 * wl.B * (wl.n_h * wl.d_h * wl.d_c * 2 + wl.d_model * wl.D)
+    return attn, gemms
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the baseline; also the --impl reference arm)
+# ----------------------------------------------------------------------------
+
+def cpu_oracle_sample(wl, n_heads, budget_s=20.0):
+    """Time the oracle's explicit-form decode step (per-head keys and values,
+    textbook softmax) for one sequence of the workload, over `n_heads` heads,
+    repeating up to ~budget_s.  Returns (GB/s of latent cache scanned, sample
+    description, threads)."""
+    from oracle import mla_oracle as O
+    from workloads import draw_weights, queries, random_cache
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    ctx = int(wl.ctx[0]) if wl.ctx else 8192
+    w = draw_weights(wl)
+    rows = random_cache(wl.with_(B=1), ctx)[0].astype(np.float64)
+    qn, qr = queries(wl)
+    heads = list(range(n_heads))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.mla_decode_explicit(qn[0], qr[0], ctx - 1, rows, w["w_uk"], w["w_uv"], n_h=wl.n_h,
+                              d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base, heads=heads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or reps >= 50:
+            break
+    # algorithmic bytes of the sample: the sequence's latent rows once per
+    # pass, scaled to the fraction of heads processed (per-head work).
+    per_rep = ctx * wl.D * 2 * (n_heads / wl.n_h)
+    gbs = per_rep * reps / el / 1e9
+    desc = (f"explicit fp64 oracle, 1 sequence x ctx {ctx} x {n_heads}/{wl.n_h} heads, "
+            f"{reps} reps in {el:.1f}s, GB/s scaled by head fraction")
+    return gbs, desc, threads, el / reps
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from workloads import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    n_heads = 16
+    vals = []
+    for i in range(args.warmup + args.steps):
+        gbs, desc, threads, t = cpu_oracle_sample(wl, n_heads, budget_s=0.0)
+        if i >= args.warmup:
+            vals.append(t)
+    t = float(np.mean(vals))
+    per_step = wl.ctx[0] * wl.D * 2 * n_heads / wl.n_h
+    value = per_step / t / 1e9
+    line = {
+        "metric": "MLA decode: HBM GB/s (% of peak) and us/step at B=64, n_h=128, ctx 8K",
+        "impl": "reference", "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "n_h": wl.n_h, "ctx": wl.ctx[0],
+                   "sample_per_step": f"1 sequence x {n_heads} heads (explicit fp64 oracle)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"1 sequence x ctx {wl.ctx[0]} x {n_heads}/{wl.n_h} heads per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import head_latent_attention_09_b200 as M
+    from head_latent_attention_09_b200 import build as _build
+    from workloads import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    M.load()
+
+    wl = WORKLOADS[args.workload]
+    B, H, D, d = wl.B, wl.n_h, wl.D, wl.d_model
+    ctx = np.asarray(wl.ctx, dtype=np.int64)
+    cfg = M.mla_config(n_h=H, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, d_model=d,
+                       page_size=wl.page_size, rope_base=wl.rope_base, dtype=M.MLA_BF16)
+    handle = M.mla_create(cfg)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    bf = torch.bfloat16
+
+    def randn(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(bf)
+
+    w_dkv = randn(wl.d_c, d, std=d ** -0.5)
+    w_kr = randn(wl.d_r, d, std=d ** -0.5)
+    w_uk = randn(H * wl.d_h, wl.d_c, std=wl.d_c ** -0.5)
+    w_uv = randn(H * wl.d_h, wl.d_c, std=wl.d_c ** -0.5)
+    cap = int(ctx.max())
+    cache = torch.empty((B, cap, D), dtype=bf, device=dev)
+    # Fill positions 0 .. ctx-2 through the library's own append kernel.
+    chunk = 4096
+    for b in range(B):
+        for t0 in range(0, int(ctx[b]) - 1, chunk):
+            t1 = min(int(ctx[b]) - 1, t0 + chunk)
+            hb = randn(t1 - t0, d)
+            sp = torch.tensor([t0], dtype=torch.int32, device=dev)
+            M.mla_cache_append(handle, hb, 1, t1 - t0, sp, w_dkv, w_kr,
+                               cache.data_ptr() + 2 * b * cap * D, cap)
+    h_new = randn(B, 1, d)
+    q_nope = randn(B, H, wl.d_h)
+    q_rope = randn(B, H, wl.d_r)
+    pos = torch.from_numpy((ctx - 1).astype(np.int32)).to(dev)
+    ctx_d = torch.from_numpy(ctx.astype(np.int32)).to(dev)
+    q_abs = torch.empty((B, H, D), dtype=bf, device=dev)
+    ctx_lat = torch.empty((B, H, wl.d_c), dtype=bf, device=dev)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    o = torch.empty((B, H, wl.d_h), dtype=bf, device=dev)
+    P = args.num_parts or M.mla_default_num_parts(handle)
+    ws_bytes = M.mla_decode_workspace_size(handle, B, P)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step(ev_pair=None):
+        M.mla_cache_append(handle, h_new, B, 1, pos, w_dkv, w_kr, cache, cap, None, 0, sh)
+        M.mla_absorb_q(handle, q_nope, q_rope, pos, w_uk, q_abs, B, sh)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, ctx_d, B, P, ws, ws_bytes, sh)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+        M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
+        M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = M.mla_get_device_status(handle, sh)
+    if st != M.MLA_OK:
+        raise M.MlaError(st, "device status after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(attn_ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_ev]))
+    st = M.mla_get_device_status(handle, sh)
+    if st != M.MLA_OK:
+        raise M.MlaError(st, "device status after timing")
+
+    # ---- end to end: host buffers in pinned memory, copies inside the timed region
+    hp = {k: v.cpu().pin_memory() for k, v in
+          (("h_new", h_new), ("q_nope", q_nope), ("q_rope", q_rope), ("pos", pos), ("ctx", ctx_d))}
+    o_host = torch.empty(o.shape, dtype=bf).pin_memory()
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in hp.items()}
+    h2d = sum(v.numel() * v.element_size() for v in hp.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for k in hp:
+            dev_in[k].copy_(hp[k], non_blocking=True)
+        M.mla_cache_append(handle, dev_in["h_new"], B, 1, dev_in["pos"], w_dkv, w_kr, cache, cap,
+                           None, 0, sh)
+        M.mla_absorb_q(handle, dev_in["q_nope"], dev_in["q_rope"], dev_in["pos"], w_uk, q_abs, B, sh)
+        M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, dev_in["ctx"], B, P, ws, ws_bytes, sh)
+        M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
+        M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+
+    # ---- reduce over ranks: max time
+    times = torch.tensor([ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    ms, attn_ms, e2e_ms = times.tolist()
+    M.mla_destroy(handle)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ctx_sum = int(ctx.sum())
+    step_bytes = algorithmic_bytes(wl, ctx_sum)
+    attn_bytes = ctx_sum * D * 2
+    hbm_peak, tf_peak, peak_kind = peaks()
+    value = step_bytes * world / (ms * 1e-3) / 1e9
+    attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
+    attn_flops, gemm_flops = algorithmic_flops(wl, ctx_sum)
+    cpu = None
+    if not args.no_cpu_baseline:
+        gbs, desc, threads, _ = cpu_oracle_sample(wl, 16, budget_s=15.0)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": "MLA decode: HBM GB/s (% of peak) and us/step at B=64, n_h=128, ctx 8K",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "us_per_step": ms * 1e3,
+        "pct_of_peak": 100.0 * value / world / hbm_peak,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": B, "n_h": H, "d_h": wl.d_h, "d_c": wl.d_c,
+                   "d_r": wl.d_r, "d_model": d, "ctx": int(ctx[0]), "num_parts": P,
+                   "cache_bytes": attn_bytes,
+                   "l2": "inputs larger than L2 (latent cache %.0f MB per rank)" % (attn_bytes / 1e6),
+                   "parallelism": f"dp{world} (independent batches, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": attn_gbs / hbm_peak, "traffic": None,
+                     "peak_kind": peak_kind, "kernel": "mla_decode_attn (plan + attention)",
+                     "attn_us": attn_ms * 1e3,
+                     "frac_of_8TBps": attn_gbs / 8000.0,
+                     "tensor_tflops": attn_flops / (attn_ms * 1e-3) / 1e12},
+        "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

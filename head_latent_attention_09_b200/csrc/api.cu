@@ -1,0 +1,266 @@
+// C ABI entry points: argument checks, kernel selection, launches.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "internal.cuh"
+
+using namespace mla;
+
+namespace {
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+bool dtype_ok(int dt) { return dt == MLA_BF16 || dt == MLA_FP32; }
+
+size_t elt(const mla_config &c) { return c.dtype == MLA_FP32 ? 4 : 2; }
+
+// Attention kernel for a configuration.  The tensor-core kernels exist for the
+// DeepSeek-V2 attention shapes in bf16; everything else runs the generic
+// CUDA-core kernel.
+int choose_attn(const mla_config &c) {
+  if (c.dtype != MLA_BF16) return kAttnSimt;
+  if (c.d_c != 512 || c.d_r != 64) return kAttnSimt;
+  if (c.page_size != 0 && c.page_size != kTile) return kAttnSimt;
+  if (c.n_h == 128) return kAttnTcPair;
+  if (c.n_h <= 32 && c.n_h % 16 == 0) return kAttnTcSmallH;
+  return kAttnSimt;
+}
+
+int choose_gemm(const mla_config &c) {
+  if (c.dtype != MLA_BF16) return kGemmSimt;
+  // TMA needs 16-byte row pitches and the kernels tile d_c, d_h and d_model by 64.
+  if (c.d_c % 128 != 0 || c.d_h % 64 != 0 || c.d_h > 256 || c.d_model % 64 != 0) return kGemmSimt;
+  if (c.d_r % 16 != 0 || c.d_r > 128) return kGemmSimt;
+  return kGemmTc;
+}
+
+int default_parts(const mla_handle *h) {
+  switch (h->attn_kind) {
+    case kAttnTcPair: return h->num_sms / 2;       // one CTA pair per two SMs
+    case kAttnTcSmallH: return h->num_sms;         // one CTA per SM
+    default: return h->num_sms * 4;
+  }
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char *mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+    case MLA_ERR_DEVICE_BOUNDS: return "MLA_ERR_DEVICE_BOUNDS";
+    default: return "MLA_ERR_UNKNOWN";
+  }
+}
+
+int mla_config_validate(const mla_config *c) {
+  if (!c) return MLA_ERR_INVALID_ARG;
+  if (c->n_h <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_r <= 0 || c->d_model <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (c->d_r % 2 != 0 || c->page_size < 0 || !(c->rope_base > 0.0) || !dtype_ok(c->dtype))
+    return MLA_ERR_INVALID_ARG;
+  // Limits of the generic kernels (register tiles and shared-memory rows).
+  if (c->d_c > 512 || c->d_c + c->d_r > 576 || c->d_model > 12288 || c->d_h > 4096)
+    return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+int mla_create(const mla_config *cfg, mla_handle **out) {
+  if (!out) return MLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  int st = mla_config_validate(cfg);
+  if (st != MLA_OK) return st;
+  mla_handle *h = (mla_handle *)calloc(1, sizeof(mla_handle));
+  if (!h) return MLA_ERR_CUDA;
+  h->cfg = *cfg;
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    free(h);
+    return MLA_ERR_CUDA;
+  }
+  h->attn_kind = choose_attn(*cfg);
+  h->gemm_kind = choose_gemm(*cfg);
+  if ((h->attn_kind != kAttnSimt || h->gemm_kind != kGemmSimt) && !tma_available()) {
+    free(h);
+    return MLA_ERR_CUDA;
+  }
+  const int nth = cfg->d_r / 2;
+  double *theta = (double *)malloc(sizeof(double) * nth);
+  for (int k = 0; k < nth; ++k) theta[k] = pow(cfg->rope_base, -2.0 * k / (double)cfg->d_r);
+  cudaError_t e = cudaMalloc(&h->d_status, sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_theta, sizeof(double) * nth);
+  if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemcpy(h->d_theta, theta, sizeof(double) * nth, cudaMemcpyHostToDevice);
+  free(theta);
+  if (e != cudaSuccess) {
+    mla_destroy(h);
+    return MLA_ERR_CUDA;
+  }
+  *out = h;
+  return MLA_OK;
+}
+
+void mla_destroy(mla_handle *h) {
+  if (!h) return;
+  if (h->d_status) cudaFree(h->d_status);
+  if (h->d_theta) cudaFree(h->d_theta);
+  free(h);
+}
+
+int mla_cache_append(mla_handle *h, const void *x, int B, int T, const int *start_pos,
+                     const void *w_dkv, const void *w_kr, void *cache, long long cache_len,
+                     const int *block_table, int max_blocks_per_seq, mla_stream_t stream) {
+  if (!h || B < 0 || T < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MLA_OK;
+  if (!x || !start_pos || !w_dkv || !w_kr || !cache) return MLA_ERR_INVALID_ARG;
+  const mla_config &c = h->cfg;
+  if (c.page_size > 0 && (!block_table || max_blocks_per_seq <= 0)) return MLA_ERR_INVALID_ARG;
+  if (c.page_size == 0 && block_table) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaErrorNotSupported;
+  if (h->gemm_kind == kGemmTc)
+    e = launch_append_tc(c, x, B, T, start_pos, w_dkv, w_kr, cache, cache_len, block_table,
+                         max_blocks_per_seq, h->d_theta, h->d_status, s);
+  if (e == cudaErrorNotSupported)
+    e = launch_append_simt(c, x, B, T, start_pos, w_dkv, w_kr, cache, cache_len, block_table,
+                           max_blocks_per_seq, h->d_theta, h->d_status, s);
+  if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+int mla_absorb_q(mla_handle *h, const void *q_nope, const void *q_rope, const int *pos,
+                 const void *w_uk, void *q_abs, int B, mla_stream_t stream) {
+  if (!h || B < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!q_nope || !q_rope || !pos || !w_uk || !q_abs) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaErrorNotSupported;
+  if (h->gemm_kind == kGemmTc)
+    e = launch_absorb_tc(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, s);
+  if (e == cudaErrorNotSupported)
+    e = launch_absorb_simt(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, s);
+  if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+int mla_default_num_parts(const mla_handle *h) { return h ? default_parts(h) : 0; }
+
+size_t mla_decode_workspace_size(const mla_handle *h, int B, int num_parts) {
+  if (!h || B < 0 || num_parts < 0) return 0;
+  const int P = num_parts == 0 ? default_parts(h) : num_parts;
+  return ws_layout(h->cfg, B, P).total;
+}
+
+int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long long cache_len,
+                    const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
+                    int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
+  if (!h || B < 0 || num_parts < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!q_abs || !cache || !ctx_len) return MLA_ERR_INVALID_ARG;
+  const mla_config &c = h->cfg;
+  if (c.page_size > 0 && (!block_table || max_blocks_per_seq <= 0)) return MLA_ERR_INVALID_ARG;
+  if (c.page_size == 0 && block_table) return MLA_ERR_INVALID_ARG;
+  const int P = num_parts == 0 ? default_parts(h) : num_parts;
+  const WsLayout L = ws_layout(c, B, P);
+  if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_plan(ctx_len, B, P, (char *)workspace, L, h->d_status, s);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  AttnArgs a;
+  a.q_abs = q_abs;
+  a.cache = cache;
+  a.cache_len = cache_len;
+  a.block_table = block_table;
+  a.max_blocks = max_blocks_per_seq;
+  a.page_size = c.page_size;
+  a.ctx_len = ctx_len;
+  a.B = B;
+  a.n_h = c.n_h;
+  a.d_c = c.d_c;
+  a.d_r = c.d_r;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)(c.d_h + c.d_r)));
+  a.ws = (char *)workspace;
+  a.L = L;
+  a.status = h->d_status;
+  e = cudaErrorNotSupported;
+  if (h->attn_kind == kAttnTcPair && aligned16(q_abs) && aligned16(cache))
+    e = launch_attn_tc_pair(a, P, s);
+  else if (h->attn_kind == kAttnTcSmallH && aligned16(q_abs) && aligned16(cache))
+    e = launch_attn_tc_smallh(a, P, s);
+  if (e == cudaErrorNotSupported) e = launch_attn_simt(a, P, c.dtype == MLA_FP32, s);
+  if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+int mla_combine_splits(mla_handle *h, const void *workspace, size_t ws_bytes, int B, int num_parts,
+                       void *ctx_lat, float *lse, mla_stream_t stream) {
+  if (!h || B < 0 || num_parts < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!ctx_lat) return MLA_ERR_INVALID_ARG;
+  const int P = num_parts == 0 ? default_parts(h) : num_parts;
+  const WsLayout L = ws_layout(h->cfg, B, P);
+  if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  return from_cuda(launch_combine(h->cfg, (const char *)workspace, L, B, ctx_lat, lse,
+                                  (cudaStream_t)stream));
+}
+
+int mla_out_proj(mla_handle *h, const void *ctx_lat, const void *w_uv, const void *w_o, void *o,
+                 void *u, int B, mla_stream_t stream) {
+  if (!h || B < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!ctx_lat || !w_uv || !o || (w_o && !u)) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaErrorNotSupported;
+  if (h->gemm_kind == kGemmTc) e = launch_outproj_tc(h->cfg, ctx_lat, w_uv, o, B, s);
+  if (e == cudaErrorNotSupported) e = launch_outproj_simt(h->cfg, ctx_lat, w_uv, o, B, s);
+  if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
+  if (w_o) {
+    e = cudaErrorNotSupported;
+    if (h->gemm_kind == kGemmTc) e = launch_wo_tc(h->cfg, o, w_o, u, B, s);
+    if (e == cudaErrorNotSupported) e = launch_wo_simt(h->cfg, o, w_o, u, B, s);
+    if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+int mla_get_device_status(mla_handle *h, mla_stream_t stream) {
+  if (!h) return MLA_ERR_INVALID_ARG;
+  unsigned v = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpy(&v, h->d_status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v && cudaMemset(h->d_status, 0, sizeof(unsigned)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v & kStatusTimeout) return MLA_ERR_TIMEOUT;
+  if (v & kStatusBounds) return MLA_ERR_DEVICE_BOUNDS;
+  return MLA_OK;
+}
+
+long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *piece_base) {
+  if (!ctx_len || !piece_base || B < 0 || num_parts <= 0) return -1;
+  long long Ttot = 0;
+  for (int b = 0; b < B; ++b) {
+    if (ctx_len[b] < 0) return -1;
+    Ttot += ceil_div_ll(ctx_len[b], kTile);
+  }
+  const long long P = Ttot < num_parts ? Ttot : num_parts;
+  long long s = 0, n = 0;
+  for (int b = 0; b < B; ++b) {
+    piece_base[b] = n;
+    const long long t = ceil_div_ll(ctx_len[b], kTile);
+    if (t > 0) n += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
+    s += t;
+  }
+  piece_base[B] = n;
+  return n;
+}
+
+}  // extern "C"

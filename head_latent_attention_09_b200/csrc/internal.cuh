@@ -1,0 +1,155 @@
+// Internal declarations shared by the host runtime and the kernels of the MLA
+// decode library.  Nothing here is part of the public ABI (see include/mla.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// KV tokens per tile; the split plan and every attention kernel work in whole
+// tiles, and the paged fast paths require page_size == kTile.
+constexpr int kTile = 64;
+
+// Bits of the device status word.
+constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusBounds = 2u;
+
+// Attention kernel chosen for a configuration at mla_create time.
+enum AttnKind : int {
+  kAttnSimt = 0,      // generic CUDA-core kernel (any shape, fp32 or bf16)
+  kAttnTcPair = 1,    // bf16, n_h == 128, d_c == 512, d_r == 64: tcgen05, CTA pair
+  kAttnTcSmallH = 2,  // bf16, n_h <= 32 (multiple of 16), d_c == 512, d_r == 64
+};
+
+enum GemmKind : int { kGemmSimt = 0, kGemmTc = 1 };
+
+}  // namespace mla
+
+struct mla_handle {
+  mla_config cfg;
+  int device;
+  int num_sms;
+  unsigned *d_status;  // device status word (kStatus* bits)
+  double *d_theta;     // device [d_r/2] RoPE frequencies theta_k
+  int attn_kind;       // mla::AttnKind
+  int gemm_kind;       // mla::GemmKind
+};
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// Split plan.  Sequence b contributes T_b = ceil(ctx_b / kTile) tiles; the
+// batch's Ttot tiles, in sequence order, are cut into P equal shares
+// [begin(w), begin(w+1)).  A (share, sequence) intersection is a piece: it
+// yields one partial ctx_lat and log-sum-exp.  P is clamped to Ttot so that no
+// share is empty, which makes the pieces of one sequence a run of consecutive
+// shares.
+// ---------------------------------------------------------------------------
+__host__ __device__ inline long long plan_begin(long long w, long long P, long long Ttot) {
+  return w * Ttot / P;
+}
+// Largest share index whose range starts at or before tile t (0 <= t < Ttot).
+__host__ __device__ inline long long plan_share_of_tile(long long t, long long P, long long Ttot) {
+  return ((t + 1) * P - 1) / Ttot;
+}
+__host__ __device__ inline long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
+
+// Workspace header written by the plan kernel; the per-sequence arrays follow.
+struct WsHeader {
+  long long B;
+  long long P;           // effective number of shares (<= requested, <= Ttot)
+  long long Ttot;        // total tiles
+  long long n_pieces;    // total pieces
+};
+
+struct WsLayout {
+  size_t tile_prefix_off;  // int64 [B+1]
+  size_t piece_base_off;   // int64 [B+1]
+  size_t opart_off;        // float [max_pieces, n_h, d_c]
+  size_t lse_off;          // float [max_pieces, n_h]
+  size_t total;
+  long long max_pieces;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout ws_layout(const mla_config &cfg, int B, int P) {
+  WsLayout L;
+  L.max_pieces = (long long)P + B;
+  size_t off = align_up(sizeof(WsHeader), 256);
+  L.tile_prefix_off = off;
+  off = align_up(off + sizeof(long long) * (size_t)(B + 1), 256);
+  L.piece_base_off = off;
+  off = align_up(off + sizeof(long long) * (size_t)(B + 1), 256);
+  L.opart_off = off;
+  off = align_up(off + sizeof(float) * (size_t)L.max_pieces * cfg.n_h * cfg.d_c, 256);
+  L.lse_off = off;
+  off = align_up(off + sizeof(float) * (size_t)L.max_pieces * cfg.n_h, 256);
+  L.total = off;
+  return L;
+}
+
+// Arguments shared by the attention kernels.
+struct AttnArgs {
+  const void *q_abs;
+  const void *cache;
+  long long cache_len;
+  const int *block_table;
+  int max_blocks;
+  int page_size;
+  const int *ctx_len;
+  int B;
+  int n_h, d_c, d_r;
+  float scale_log2;  // log2(e) / sqrt(d_h + d_r)
+  char *ws;
+  WsLayout L;
+  unsigned *status;
+};
+
+// ---------------------------------------------------------------------------
+// Launchers (return cudaGetLastError() of the launch).
+// ---------------------------------------------------------------------------
+cudaError_t launch_plan(const int *ctx_len, int B, int P, char *ws, const WsLayout &L,
+                        unsigned *status, cudaStream_t s);
+
+cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s);
+cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
+                           void *ctx_lat, float *lse, cudaStream_t s);
+
+cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int T,
+                               const int *start_pos, const void *w_dkv, const void *w_kr,
+                               void *cache, long long cache_len, const int *block_table,
+                               int max_blocks, const double *theta, unsigned *status,
+                               cudaStream_t s);
+cudaError_t launch_absorb_simt(const mla_config &cfg, const void *q_nope, const void *q_rope,
+                               const int *pos, const void *w_uk, void *q_abs, int B,
+                               const double *theta, cudaStream_t s);
+cudaError_t launch_outproj_simt(const mla_config &cfg, const void *ctx_lat, const void *w_uv,
+                                void *o, int B, cudaStream_t s);
+cudaError_t launch_wo_simt(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
+                           cudaStream_t s);
+
+// tcgen05 paths (bf16 only); return cudaErrorNotSupported for shapes they lack.
+cudaError_t launch_append_tc(const mla_config &cfg, const void *h, int B, int T,
+                             const int *start_pos, const void *w_dkv, const void *w_kr,
+                             void *cache, long long cache_len, const int *block_table,
+                             int max_blocks, const double *theta, unsigned *status,
+                             cudaStream_t s);
+cudaError_t launch_absorb_tc(const mla_config &cfg, const void *q_nope, const void *q_rope,
+                             const int *pos, const void *w_uk, void *q_abs, int B,
+                             const double *theta, cudaStream_t s);
+cudaError_t launch_outproj_tc(const mla_config &cfg, const void *ctx_lat, const void *w_uv,
+                              void *o, int B, cudaStream_t s);
+cudaError_t launch_wo_tc(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
+                         cudaStream_t s);
+cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s);
+cudaError_t launch_attn_tc_smallh(const AttnArgs &a, int P, cudaStream_t s);
+
+// Resolve the driver entry point for tensor-map encoding (no libcuda link).
+bool tma_available();
+
+}  // namespace mla

@@ -1,0 +1,439 @@
+// CUDA-core kernels: the split plan, the log-sum-exp combine, and generic
+// (any shape, fp32 or bf16) versions of append / absorb / attention /
+// output projection.  The fp32 configuration runs entirely here; bf16 shapes
+// with a tensor-core kernel use those instead (see api.cu).
+#include <math_constants.h>
+
+#include "internal.cuh"
+
+namespace mla {
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Row index (in units of D-element rows) of token p of sequence b, or -1 when
+// the position is outside the cache / unmapped (the caller flags it).
+__device__ __forceinline__ long long cache_row(int b, long long p, long long cache_len,
+                                               const int *block_table, int max_blocks,
+                                               int page_size) {
+  if (p < 0) return -1;
+  if (page_size == 0) {
+    if (p >= cache_len) return -1;
+    return (long long)b * cache_len + p;
+  }
+  long long bi = p / page_size;
+  if (bi >= max_blocks) return -1;
+  int blk = block_table[(long long)b * max_blocks + bi];
+  if (blk < 0 || blk >= cache_len) return -1;
+  return (long long)blk * page_size + (p % page_size);
+}
+
+// ---------------------------------------------------------------------------
+// plan: one block of 1024 threads
+// ---------------------------------------------------------------------------
+__device__ long long block_exclusive_scan(long long v, long long *smem, long long *total) {
+  const int tid = threadIdx.x, n = blockDim.x;
+  smem[tid] = v;
+  __syncthreads();
+  for (int off = 1; off < n; off <<= 1) {
+    long long add = tid >= off ? smem[tid - off] : 0;
+    __syncthreads();
+    smem[tid] += add;
+    __syncthreads();
+  }
+  long long incl = smem[tid];
+  *total = smem[n - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, int P_req, char *ws,
+                                                    WsLayout L, unsigned *status) {
+  __shared__ long long scan[1024];
+  long long *tile_prefix = reinterpret_cast<long long *>(ws + L.tile_prefix_off);
+  long long *piece_base = reinterpret_cast<long long *>(ws + L.piece_base_off);
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (B + nt - 1) / nt;
+  const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
+
+  long long local = 0;
+  for (int b = b0; b < b1; ++b) {
+    int c = ctx_len[b];
+    if (c < 0) { atomicOr(status, kStatusBounds); c = 0; }
+    local += ceil_div_ll(c, kTile);
+  }
+  long long Ttot;
+  long long run = block_exclusive_scan(local, scan, &Ttot);
+  for (int b = b0; b < b1; ++b) {
+    tile_prefix[b] = run;
+    int c = max(ctx_len[b], 0);
+    run += ceil_div_ll(c, kTile);
+  }
+  if (tid == 0) tile_prefix[B] = Ttot;
+  const long long P = Ttot < (long long)P_req ? Ttot : (long long)P_req;
+
+  long long local_pieces = 0;
+  for (int b = b0; b < b1; ++b) {
+    long long s = tile_prefix[b];
+    long long t = ceil_div_ll(max(ctx_len[b], 0), kTile);
+    if (t > 0) local_pieces += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
+  }
+  long long n_pieces;
+  long long prun = block_exclusive_scan(local_pieces, scan, &n_pieces);
+  for (int b = b0; b < b1; ++b) {
+    piece_base[b] = prun;
+    long long s = tile_prefix[b];
+    long long t = ceil_div_ll(max(ctx_len[b], 0), kTile);
+    if (t > 0) prun += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
+  }
+  if (tid == 0) {
+    piece_base[B] = n_pieces;
+    WsHeader *hd = reinterpret_cast<WsHeader *>(ws);
+    hd->B = B;
+    hd->P = P;
+    hd->Ttot = Ttot;
+    hd->n_pieces = n_pieces;
+    if (n_pieces > L.max_pieces) atomicOr(status, kStatusBounds);  // cannot happen by construction
+  }
+}
+
+// ---------------------------------------------------------------------------
+// generic attention: one warp per head, lanes split the row's features
+// ---------------------------------------------------------------------------
+constexpr int kSimtMaxD = 576;      // d_c + d_r
+constexpr int kSimtMaxC = 512;      // d_c
+constexpr int kQPerLane = kSimtMaxD / 32;
+constexpr int kOPerLane = kSimtMaxC / 32;
+
+template <typename T>
+__global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
+  const WsHeader *hd = reinterpret_cast<const WsHeader *>(a.ws);
+  const long long P = hd->P, Ttot = hd->Ttot;
+  const int w = blockIdx.x;
+  if (w >= P) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * (blockDim.x >> 5) + warp;
+  if (h >= a.n_h) return;
+  const int D = a.d_c + a.d_r;
+  const long long *tp = reinterpret_cast<const long long *>(a.ws + a.L.tile_prefix_off);
+  const long long *pb = reinterpret_cast<const long long *>(a.ws + a.L.piece_base_off);
+  float *opart = reinterpret_cast<float *>(a.ws + a.L.opart_off);
+  float *lse = reinterpret_cast<float *>(a.ws + a.L.lse_off);
+  const T *cache = reinterpret_cast<const T *>(a.cache);
+  const T *qg = reinterpret_cast<const T *>(a.q_abs);
+
+  const long long t0 = plan_begin(w, P, Ttot), t1 = plan_begin(w + 1, P, Ttot);
+  // first sequence whose tiles reach past t0
+  int lo = 0, hi = a.B;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (tp[mid + 1] <= t0) lo = mid + 1; else hi = mid;
+  }
+  for (int b = lo; b < a.B && tp[b] < t1; ++b) {
+    const long long s0 = t0 > tp[b] ? t0 : tp[b];
+    const long long s1 = t1 < tp[b + 1] ? t1 : tp[b + 1];
+    if (s0 >= s1) continue;
+    const long long piece = pb[b] + (w - plan_share_of_tile(tp[b], P, Ttot));
+    int ctx = a.ctx_len[b];
+    if (a.page_size == 0 && ctx > a.cache_len) {
+      if (lane == 0) atomicOr(a.status, kStatusBounds);
+      ctx = (int)a.cache_len;
+    }
+    const long long p_begin = (s0 - tp[b]) * kTile;
+    const long long p_end = min((long long)ctx, (s1 - tp[b]) * kTile);
+
+    float q[kQPerLane];
+#pragma unroll
+    for (int j = 0; j < kQPerLane; ++j) {
+      const int f = lane + 32 * j;
+      q[j] = f < D ? to_f(qg[((long long)b * a.n_h + h) * D + f]) : 0.f;
+    }
+    float o[kOPerLane];
+#pragma unroll
+    for (int j = 0; j < kOPerLane; ++j) o[j] = 0.f;
+    float m = -CUDART_INF_F, l = 0.f;
+
+    for (long long p = p_begin; p < p_end; ++p) {
+      const long long row = cache_row(b, p, a.cache_len, a.block_table, a.max_blocks, a.page_size);
+      if (row < 0) {
+        if (lane == 0) atomicOr(a.status, kStatusBounds);
+        continue;
+      }
+      const T *r = cache + row * D;
+      float part = 0.f;
+#pragma unroll
+      for (int j = 0; j < kQPerLane; ++j) {
+        const int f = lane + 32 * j;
+        if (f < D) part += q[j] * to_f(r[f]);
+      }
+      const float s = warp_sum(part) * a.scale_log2;   // score in log2 units
+      const float m_new = fmaxf(m, s);
+      const float corr = exp2f(m - m_new);
+      const float pr = exp2f(s - m_new);
+      l = l * corr + pr;
+#pragma unroll
+      for (int j = 0; j < kOPerLane; ++j) {
+        const int f = lane + 32 * j;
+        if (f < a.d_c) o[j] = o[j] * corr + pr * to_f(r[f]);
+      }
+      m = m_new;
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float *dst = opart + (piece * a.n_h + h) * (long long)a.d_c;
+#pragma unroll
+    for (int j = 0; j < kOPerLane; ++j) {
+      const int f = lane + 32 * j;
+      if (f < a.d_c) dst[f] = o[j] * inv;
+    }
+    if (lane == 0)
+      lse[piece * a.n_h + h] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// log-sum-exp combine: one block per (sequence, head)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) combine_kernel(const char *ws, WsLayout L, int n_h, int d_c,
+                                                      T *ctx_lat, float *lse_out) {
+  const int b = blockIdx.x, h = blockIdx.y;
+  const long long *pb = reinterpret_cast<const long long *>(ws + L.piece_base_off);
+  const float *lse = reinterpret_cast<const float *>(ws + L.lse_off);
+  const float *op = reinterpret_cast<const float *>(ws + L.opart_off);
+  const long long p0 = pb[b], p1 = pb[b + 1];
+  float m = -CUDART_INF_F;
+  for (long long p = p0; p < p1; ++p) m = fmaxf(m, lse[p * n_h + h]);
+  T *dst = ctx_lat + ((long long)b * n_h + h) * d_c;
+  if (m == -CUDART_INF_F) {
+    for (int f = threadIdx.x; f < d_c; f += blockDim.x) dst[f] = from_f<T>(0.f);
+    if (lse_out && threadIdx.x == 0) lse_out[(long long)b * n_h + h] = -CUDART_INF_F;
+    return;
+  }
+  float tot = 0.f;
+  for (long long p = p0; p < p1; ++p) tot += expf(lse[p * n_h + h] - m);
+  const float inv = 1.f / tot;
+  for (int f = threadIdx.x; f < d_c; f += blockDim.x) {
+    float acc = 0.f;
+    for (long long p = p0; p < p1; ++p)
+      acc += expf(lse[p * n_h + h] - m) * op[(p * n_h + h) * (long long)d_c + f];
+    dst[f] = from_f<T>(acc * inv);
+  }
+  if (lse_out && threadIdx.x == 0) lse_out[(long long)b * n_h + h] = m + logf(tot);
+}
+
+// ---------------------------------------------------------------------------
+// cache append: one block per token; each warp computes a pair of features
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) append_simt_kernel(
+    const T *h, int T_new, int d, int d_c, int d_r, const int *start_pos, const T *w_dkv,
+    const T *w_kr, T *cache, long long cache_len, const int *block_table, int max_blocks,
+    int page_size, const double *theta, unsigned *status) {
+  extern __shared__ float sh[];
+  const long long tok = blockIdx.x;
+  const int b = (int)(tok / T_new), t = (int)(tok % T_new);
+  for (int k = threadIdx.x; k < d; k += blockDim.x) sh[k] = to_f(h[tok * d + k]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int D = d_c + d_r;
+  const int f0 = 2 * (blockIdx.y * (blockDim.x >> 5) + warp);
+  if (f0 >= D) return;
+  const T *w0 = f0 < d_c ? w_dkv + (long long)f0 * d : w_kr + (long long)(f0 - d_c) * d;
+  const T *w1 = w0 + d;
+  float a0 = 0.f, a1 = 0.f;
+  for (int k = lane; k < d; k += 32) {
+    a0 += to_f(w0[k]) * sh[k];
+    a1 += to_f(w1[k]) * sh[k];
+  }
+  a0 = warp_sum(a0);
+  a1 = warp_sum(a1);
+  if (lane != 0) return;
+  const long long p = (long long)start_pos[b] + t;
+  if (f0 >= d_c) {
+    double sn, cs;
+    sincos((double)p * theta[(f0 - d_c) >> 1], &sn, &cs);
+    const float c = (float)cs, s = (float)sn;
+    const float r0 = a0 * c - a1 * s, r1 = a0 * s + a1 * c;
+    a0 = r0;
+    a1 = r1;
+  }
+  const long long row = cache_row(b, p, cache_len, block_table, max_blocks, page_size);
+  if (row < 0) {
+    atomicOr(status, kStatusBounds);
+    return;
+  }
+  cache[row * D + f0] = from_f<T>(a0);
+  cache[row * D + f0 + 1] = from_f<T>(a1);
+}
+
+// ---------------------------------------------------------------------------
+// query absorption: one block per (sequence, head)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) absorb_simt_kernel(const T *q_nope, const T *q_rope,
+                                                          const int *pos, const T *w_uk, T *q_abs,
+                                                          int n_h, int d_h, int d_c, int d_r,
+                                                          const double *theta) {
+  extern __shared__ float sq[];
+  const int b = blockIdx.x, i = blockIdx.y;
+  const long long bi = (long long)b * n_h + i;
+  for (int r = threadIdx.x; r < d_h; r += blockDim.x) sq[r] = to_f(q_nope[bi * d_h + r]);
+  __syncthreads();
+  const int D = d_c + d_r;
+  for (int m = threadIdx.x; m < d_c; m += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < d_h; ++r) acc += to_f(w_uk[((long long)i * d_h + r) * d_c + m]) * sq[r];
+    q_abs[bi * D + m] = from_f<T>(acc);
+  }
+  const double p = (double)pos[b];
+  for (int k = threadIdx.x; k < d_r / 2; k += blockDim.x) {
+    const float x0 = to_f(q_rope[bi * d_r + 2 * k]), x1 = to_f(q_rope[bi * d_r + 2 * k + 1]);
+    double sn, cs;
+    sincos(p * theta[k], &sn, &cs);
+    const float c = (float)cs, s = (float)sn;
+    q_abs[bi * D + d_c + 2 * k] = from_f<T>(x0 * c - x1 * s);
+    q_abs[bi * D + d_c + 2 * k + 1] = from_f<T>(x0 * s + x1 * c);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// output projection: one block per (sequence, head), one warp per output
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) outproj_simt_kernel(const T *ctx, const T *w_uv, T *o,
+                                                           int n_h, int d_h, int d_c) {
+  const int b = blockIdx.x, i = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const T *c = ctx + ((long long)b * n_h + i) * d_c;
+  for (int r = warp; r < d_h; r += nw) {
+    const T *wr = w_uv + ((long long)i * d_h + r) * d_c;
+    float acc = 0.f;
+    for (int k = lane; k < d_c; k += 32) acc += to_f(wr[k]) * to_f(c[k]);
+    acc = warp_sum(acc);
+    if (lane == 0) o[((long long)b * n_h + i) * d_h + r] = from_f<T>(acc);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) wo_simt_kernel(const T *o, const T *w_o, T *u, int K, int d) {
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.y * (blockDim.x >> 5) + warp;
+  if (j >= d) return;
+  const T *wr = w_o + (long long)j * K;
+  const T *x = o + (long long)b * K;
+  float acc = 0.f;
+  for (int k = lane; k < K; k += 32) acc += to_f(wr[k]) * to_f(x[k]);
+  acc = warp_sum(acc);
+  if (lane == 0) u[(long long)b * d + j] = from_f<T>(acc);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_plan(const int *ctx_len, int B, int P, char *ws, const WsLayout &L,
+                        unsigned *status, cudaStream_t s) {
+  plan_kernel<<<1, 1024, 0, s>>>(ctx_len, B, P, ws, L, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s) {
+  if (a.d_c + a.d_r > kSimtMaxD || a.d_c > kSimtMaxC) return cudaErrorNotSupported;
+  const int warps = a.n_h < 8 ? a.n_h : 8;
+  dim3 grid(P, (a.n_h + warps - 1) / warps);
+  if (fp32) attn_simt_kernel<float><<<grid, warps * 32, 0, s>>>(a);
+  else attn_simt_kernel<__nv_bfloat16><<<grid, warps * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
+                           void *ctx_lat, float *lse, cudaStream_t s) {
+  dim3 grid(B, cfg.n_h);
+  if (cfg.dtype == MLA_FP32)
+    combine_kernel<float><<<grid, 128, 0, s>>>(ws, L, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
+  else
+    combine_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(ws, L, cfg.n_h, cfg.d_c,
+                                                       (__nv_bfloat16 *)ctx_lat, lse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int T,
+                               const int *start_pos, const void *w_dkv, const void *w_kr,
+                               void *cache, long long cache_len, const int *block_table,
+                               int max_blocks, const double *theta, unsigned *status,
+                               cudaStream_t s) {
+  const int D = cfg.d_c + cfg.d_r;
+  dim3 grid((unsigned)((long long)B * T), (D / 2 + 7) / 8);
+  const size_t smem = sizeof(float) * cfg.d_model;
+  if (smem > 48 * 1024) return cudaErrorNotSupported;
+  if (cfg.dtype == MLA_FP32)
+    append_simt_kernel<float><<<grid, 256, smem, s>>>(
+        (const float *)h, T, cfg.d_model, cfg.d_c, cfg.d_r, start_pos, (const float *)w_dkv,
+        (const float *)w_kr, (float *)cache, cache_len, block_table, max_blocks, cfg.page_size,
+        theta, status);
+  else
+    append_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
+        (const __nv_bfloat16 *)h, T, cfg.d_model, cfg.d_c, cfg.d_r, start_pos,
+        (const __nv_bfloat16 *)w_dkv, (const __nv_bfloat16 *)w_kr, (__nv_bfloat16 *)cache,
+        cache_len, block_table, max_blocks, cfg.page_size, theta, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_absorb_simt(const mla_config &cfg, const void *q_nope, const void *q_rope,
+                               const int *pos, const void *w_uk, void *q_abs, int B,
+                               const double *theta, cudaStream_t s) {
+  dim3 grid(B, cfg.n_h);
+  const size_t smem = sizeof(float) * cfg.d_h;
+  if (cfg.dtype == MLA_FP32)
+    absorb_simt_kernel<float><<<grid, 256, smem, s>>>(
+        (const float *)q_nope, (const float *)q_rope, pos, (const float *)w_uk, (float *)q_abs,
+        cfg.n_h, cfg.d_h, cfg.d_c, cfg.d_r, theta);
+  else
+    absorb_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
+        (const __nv_bfloat16 *)q_nope, (const __nv_bfloat16 *)q_rope, pos,
+        (const __nv_bfloat16 *)w_uk, (__nv_bfloat16 *)q_abs, cfg.n_h, cfg.d_h, cfg.d_c, cfg.d_r,
+        theta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_outproj_simt(const mla_config &cfg, const void *ctx_lat, const void *w_uv,
+                                void *o, int B, cudaStream_t s) {
+  dim3 grid(B, cfg.n_h);
+  if (cfg.dtype == MLA_FP32)
+    outproj_simt_kernel<float><<<grid, 256, 0, s>>>((const float *)ctx_lat, (const float *)w_uv,
+                                                    (float *)o, cfg.n_h, cfg.d_h, cfg.d_c);
+  else
+    outproj_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        (const __nv_bfloat16 *)ctx_lat, (const __nv_bfloat16 *)w_uv, (__nv_bfloat16 *)o, cfg.n_h,
+        cfg.d_h, cfg.d_c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wo_simt(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
+                           cudaStream_t s) {
+  const int K = cfg.n_h * cfg.d_h;
+  dim3 grid(B, (cfg.d_model + 7) / 8);
+  if (cfg.dtype == MLA_FP32)
+    wo_simt_kernel<float><<<grid, 256, 0, s>>>((const float *)o, (const float *)w_o, (float *)u, K,
+                                               cfg.d_model);
+  else
+    wo_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)w_o, (__nv_bfloat16 *)u, K, cfg.d_model);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

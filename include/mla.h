@@ -1,0 +1,181 @@
+/*
+ * mla.h -- C ABI of a decode-time Multi-head Latent Attention (MLA) library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (the method's equations):
+ *   "DeepSeek-V3 Technical Report" reading note (dogely.com), MLA section:
+ *     c^KV_t = W^DKV h_t,  k^R_t = RoPE(W^KR h_t),  k_{t,i} = [W^UK_i c^KV_t ; k^R_t],
+ *     v_{t,i} = W^UV_i c^KV_t,
+ *     o_{t,i} = sum_{j<=t} Softmax_j(q_{t,i}^T k_{j,i} / sqrt(d_h + d_h^R)) v_{j,i},
+ *     u_t = W^O [o_{t,1}; ...; o_{t,n_h}].
+ *   "DeepSeek-V2: Strong, Economical, Efficient" (translation), §2.1.2-§2.1.3
+ *     (only [c^KV_t ; k^R_t] is cached: d_c + d_h^R elements per token per layer)
+ *     and Appendix C (W^UK is absorbed into the query and W^UV into the output
+ *     side, so attention runs on the cached rows directly).
+ *
+ * The decode step is five calls, all asynchronous on the caller's stream:
+ *   mla_cache_append    write [c^KV ; k^R] rows for new tokens
+ *   mla_absorb_q        q_abs_i = [W^UK_i^T q^C_i ; RoPE(q^R_i, pos)]
+ *   mla_decode_attn     split-KV softmax over the latent rows -> partials
+ *   mla_combine_splits  log-sum-exp merge of the partials -> ctx_lat
+ *   mla_out_proj        o_i = W^UV_i ctx_lat_i  (and optionally u = W^O o)
+ *
+ * Conventions for every call
+ *   - Tensor pointers are DEVICE memory owned by the caller, row-major and
+ *     contiguous, element type = cfg.dtype (bf16 or fp32), unless stated.
+ *     Integer tensors (positions, lengths, block tables) are device int32.
+ *   - Weights are row-major [out_features, in_features]:
+ *       W_DKV [d_c, d_model]     W_KR [d_r, d_model]
+ *       W_UK, W_UV [n_h*d_h, d_c] (rows i*d_h .. i*d_h+d_h-1 belong to head i)
+ *       W_O [d_model, n_h*d_h]
+ *   - The latent cache row of a token is D = d_c + d_r elements [c^KV | k^R].
+ *     Contiguous cache (cfg.page_size == 0): cache = [B, cache_len, D], where
+ *       cache_len is the per-sequence capacity in tokens; block_table = NULL.
+ *     Paged cache (cfg.page_size > 0): cache = pool [cache_len, page_size, D],
+ *       cache_len = number of blocks in the pool; block_table = [B,
+ *       max_blocks_per_seq] int32 block ids; token p of sequence b lives in block
+ *       block_table[b*max_blocks_per_seq + p/page_size], row p%page_size.
+ *   - RoPE rotates consecutive pairs (x_2k, x_2k+1) of the d_r-wide rotary part
+ *     by angle pos*theta_k, theta_k = rope_base^(-2k/d_r) (RoFormer form; the
+ *     angle is formed in double precision).
+ *   - Host-side argument checks return an error before anything is launched.
+ *     Checks that need device data (positions, lengths, block ids beyond the
+ *     table or pool) are made in the kernels: an offending access is skipped
+ *     and a flag is set in the handle's status word, which
+ *     mla_get_device_status() reports.  Every device-side wait is bounded; a
+ *     wait that runs out sets MLA_ERR_TIMEOUT in the same word.
+ *   - The library allocates device memory only in mla_create (the handle's
+ *     status word and RoPE table).  The decode calls use the caller's workspace.
+ *   - A sequence with ctx_len = 0 produces a zero ctx_lat row and lse = -inf.
+ *   - Results are deterministic for a fixed num_parts (no floating-point atomics).
+ *   - A handle may be used from one host thread at a time.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Identical to cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *mla_stream_t;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,   /* a host-checked argument is out of range or NULL */
+  MLA_ERR_UNSUPPORTED = 2,   /* shape or dtype this build has no kernel for */
+  MLA_ERR_WORKSPACE = 3,     /* workspace pointer NULL, misaligned or too small */
+  MLA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  MLA_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
+  MLA_ERR_DEVICE_BOUNDS = 6  /* a device-side index check failed (access skipped) */
+} mla_status;
+
+typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;
+
+typedef struct {
+  int n_h;          /* attention heads */
+  int d_h;          /* per-head width of q^C / v */
+  int d_c;          /* KV compression width (latent c^KV) */
+  int d_r;          /* decoupled RoPE width d_h^R (even) */
+  int d_model;      /* model width d */
+  int page_size;    /* 0 = contiguous cache; else tokens per block (64 for the fast paths) */
+  double rope_base; /* RoPE base, e.g. 10000 */
+  int dtype;        /* mla_dtype: storage and input type of every tensor */
+} mla_config;
+
+typedef struct mla_handle mla_handle;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char *mla_status_string(int status);
+
+/* Host-only check of a configuration (no CUDA calls): MLA_OK,
+ * MLA_ERR_INVALID_ARG (non-positive or odd d_r, NULL) or MLA_ERR_UNSUPPORTED. */
+int mla_config_validate(const mla_config *cfg);
+
+/* Create a handle on the current CUDA device.  Allocates the status word and
+ * the RoPE frequency table (theta_k in double precision).  On failure *out is
+ * NULL.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int mla_create(const mla_config *cfg, mla_handle **out);
+
+/* Release a handle (synchronises nothing; the caller must not have work in
+ * flight that uses it).  NULL is accepted. */
+void mla_destroy(mla_handle *handle);
+
+/* Cache append (V3 note, MLA equations: c^KV_t = W^DKV h_t, k^R_t = RoPE(W^KR h_t);
+ * V2 §2.1.3: the cached row is [c^KV_t ; k^R_t]).
+ *   h          [B, T, d_model] hidden states of T new tokens per sequence
+ *   start_pos  device int32 [B]: token t of sequence b is written at position
+ *              start_pos[b] + t and rotated by that position
+ *   w_dkv      [d_c, d_model], w_kr [d_r, d_model]
+ *   cache, cache_len, block_table, max_blocks_per_seq: see the conventions above
+ * Positions outside the cache (or unmapped blocks) are skipped and flagged
+ * MLA_ERR_DEVICE_BOUNDS.  T may be large (bulk fill) or 1 (decode step). */
+int mla_cache_append(mla_handle *handle, const void *h, int B, int T, const int *start_pos,
+                     const void *w_dkv, const void *w_kr, void *cache, long long cache_len,
+                     const int *block_table, int max_blocks_per_seq, mla_stream_t stream);
+
+/* Query absorption (V2 Appendix C; V3 note q_{t,i} = [q^C_{t,i} ; q^R_{t,i}]):
+ *   q_abs[b,i,:d_c]  = W^UK_i^T q_nope[b,i,:]        (W^UK_i = rows i*d_h.. of W^UK)
+ *   q_abs[b,i,d_c:]  = RoPE(q_rope[b,i,:], pos[b])
+ *   q_nope [B, n_h, d_h], q_rope [B, n_h, d_r] (before rotation), pos device int32 [B]
+ *   (the query's own position, normally ctx_len-1), q_abs [B, n_h, d_c+d_r]. */
+int mla_absorb_q(mla_handle *handle, const void *q_nope, const void *q_rope, const int *pos,
+                 const void *w_uk, void *q_abs, int B, mla_stream_t stream);
+
+/* Bytes of workspace mla_decode_attn/mla_combine_splits need for batch B with
+ * num_parts work partitions (0 = the default for this handle's kernel).
+ * Returns 0 on invalid arguments. */
+size_t mla_decode_workspace_size(const mla_handle *handle, int B, int num_parts);
+
+/* Default number of work partitions for this handle (depends on the kernel
+ * selected for the configuration and on the device's SM count). */
+int mla_default_num_parts(const mla_handle *handle);
+
+/* Split-KV decode attention over the latent cache (V3 note: o_{t,i} with the
+ * softmax over j = 1..t, scale 1/sqrt(d_h + d_r); absorbed form of V2 App. C).
+ * The batch's KV tokens, in 64-token tiles, are cut into num_parts equal shares;
+ * each share is processed by one worker (one CTA, or one CTA pair for 128
+ * heads) and yields, per (sequence, share) piece, the normalised partial
+ * ctx_lat and its log-sum-exp, written into the workspace.
+ *   q_abs   [B, n_h, d_c+d_r] absorbed queries
+ *   ctx_len device int32 [B], ctx_len[b] tokens of sequence b are attended
+ *   workspace >= mla_decode_workspace_size(handle, B, num_parts) bytes, 256-byte
+ *   aligned, device memory; its contents are overwritten. */
+int mla_decode_attn(mla_handle *handle, const void *q_abs, const void *cache, long long cache_len,
+                    const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
+                    int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream);
+
+/* Merge the partials of the preceding mla_decode_attn on the same workspace:
+ * m = max_s lse_s, ctx_lat = sum_s e^(lse_s - m) O_s / sum_s e^(lse_s - m),
+ * lse = m + log sum_s e^(lse_s - m).
+ *   ctx_lat [B, n_h, d_c] (cfg.dtype), lse [B, n_h] float32 or NULL.
+ * B and num_parts must equal those given to mla_decode_attn. */
+int mla_combine_splits(mla_handle *handle, const void *workspace, size_t ws_bytes, int B,
+                       int num_parts, void *ctx_lat, float *lse, mla_stream_t stream);
+
+/* Output projection (V2 App. C, W^UV absorbed to the output side; V3 note u_t):
+ *   o[b,i,:] = W^UV_i ctx_lat[b,i,:]      o [B, n_h, d_h]
+ *   if w_o != NULL: u[b,:] = W^O o[b,:,:] (flattened)   u [B, d_model]
+ * w_uv [n_h*d_h, d_c], w_o [d_model, n_h*d_h] or NULL (then u is ignored). */
+int mla_out_proj(mla_handle *handle, const void *ctx_lat, const void *w_uv, const void *w_o,
+                 void *o, void *u, int B, mla_stream_t stream);
+
+/* Synchronise `stream`, read and clear the handle's device status word.
+ * Returns MLA_OK, MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_BOUNDS or MLA_ERR_CUDA. */
+int mla_get_device_status(mla_handle *handle, mla_stream_t stream);
+
+/* Host mirror of the split plan mla_decode_attn uses (no CUDA calls).
+ *   ctx_len host int32 [B]; num_parts as for mla_decode_attn (must be > 0 here).
+ *   piece_base host int64 [B+1] (out): pieces of sequence b are
+ *   piece_base[b] .. piece_base[b+1]-1.  Returns the total number of pieces,
+ *   or -1 on invalid arguments. */
+long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *piece_base);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,127 @@
+"""The C ABI without a GPU: the library builds for sm_100a, loads, exports every
+symbol include/mla.h declares, and its host-only logic (configuration checks,
+status strings, the split plan) behaves as documented."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import head_latent_attention_09_b200 as M
+from head_latent_attention_09_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "mla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return M.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in mla.h but not exported"
+    assert set(names) == set(M.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "MLA_OK"), (1, "MLA_ERR_INVALID_ARG"), (5, "MLA_ERR_TIMEOUT"),
+                       (6, "MLA_ERR_DEVICE_BOUNDS")]:
+        assert M.mla_status_string(code) == name
+    assert M.mla_status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def _cfg(**kw):
+    base = dict(n_h=128, d_h=128, d_c=512, d_r=64, d_model=5120, page_size=0, rope_base=10000.0,
+                dtype=M.MLA_BF16)
+    base.update(kw)
+    return M.mla_config(**base)
+
+
+def test_config_validation(lib):
+    assert M.mla_config_validate(_cfg()) == M.MLA_OK
+    assert M.mla_config_validate(_cfg(dtype=M.MLA_FP32, n_h=4, d_h=32, d_c=128, d_r=16,
+                                      d_model=256)) == M.MLA_OK
+    assert M.mla_config_validate(_cfg(d_r=63)) == M.MLA_ERR_INVALID_ARG
+    assert M.mla_config_validate(_cfg(n_h=0)) == M.MLA_ERR_INVALID_ARG
+    assert M.mla_config_validate(_cfg(rope_base=0.0)) == M.MLA_ERR_INVALID_ARG
+    assert M.mla_config_validate(_cfg(dtype=7)) == M.MLA_ERR_INVALID_ARG
+    assert M.mla_config_validate(_cfg(page_size=-1)) == M.MLA_ERR_INVALID_ARG
+    assert M.mla_config_validate(_cfg(d_c=1024)) == M.MLA_ERR_UNSUPPORTED
+    assert lib.mla_config_validate(None) == M.MLA_ERR_INVALID_ARG
+
+
+def test_create_without_device_fails_cleanly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    h = ctypes.c_void_p(123)
+    st = lib.mla_create(ctypes.byref(_cfg()), ctypes.byref(h))
+    assert st == M.MLA_ERR_CUDA and h.value is None
+    lib.mla_destroy(None)
+    # NULL handles are rejected before any CUDA call
+    assert lib.mla_decode_workspace_size(None, 4, 0) == 0
+    assert lib.mla_get_device_status(None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_absorb_q(None, None, None, None, None, None, 1, None) == M.MLA_ERR_INVALID_ARG
+
+
+def python_plan(ctx, P):
+    """Independent restatement of the split plan for checking the library's."""
+    tiles = [(c + 63) // 64 for c in ctx]
+    starts = np.concatenate([[0], np.cumsum(tiles)]).astype(int)
+    total = int(starts[-1])
+    P = min(P, total)
+    if total == 0:
+        return 0, [0] * (len(ctx) + 1), []
+    share = [(w * total // P, (w + 1) * total // P) for w in range(P)]
+    pieces = []
+    for w, (a, b) in enumerate(share):
+        for s in range(len(ctx)):
+            lo, hi = max(a, starts[s]), min(b, starts[s + 1])
+            if lo < hi:
+                pieces.append((s, w, lo, hi))
+    pieces.sort()
+    base, k = [], 0
+    for s in range(len(ctx)):
+        base.append(k)
+        k += sum(1 for p in pieces if p[0] == s)
+    base.append(k)
+    return len(pieces), base, share
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_plan_matches_independent_restatement(lib, seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 40))
+    ctx = rng.integers(0, 3000, size=B)
+    ctx[rng.random(B) < 0.2] = 0
+    for P in (1, 3, 74, 148, 1000):
+        n, base = M.mla_plan_pieces(ctx.tolist(), P)
+        n2, base2, share = python_plan(ctx.tolist(), P)
+        assert n == n2 and base == base2
+        assert n <= P + B
+        # equal shares: sizes differ by at most one tile
+        if share:
+            sizes = [b - a for a, b in share]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+def test_plan_v2_workload(lib):
+    n, base = M.mla_plan_pieces([8192] * 64, 74)
+    assert n <= 74 + 64 and base[-1] == n
+    # every sequence is split: 74 shares of 110.7 tiles over 128-tile sequences
+    assert all(base[b + 1] - base[b] >= 1 for b in range(64))
+    assert M.mla_plan_pieces([], 5)[0] == 0
+    assert lib.mla_plan_pieces(None, 0, 1, None) == -1

@@ -1,0 +1,187 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the CPU
+oracle on the same seeded inputs.
+
+* Full decode steps of every workload at its full size, in the launch
+  configuration the benchmark times (default number of work partitions),
+  checked on sampled sequences the oracle computes one by one.
+* The attention step alone on directly drawn caches, at sizes that span many
+  tiles and ragged tails, with every split count from 1 to more shares than
+  tiles.
+* Edge cases: empty and one-token contexts, contexts that end inside a tile,
+  NaN garbage beyond each context, paged caches, the output projection W^O.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import head_latent_attention_09_b200 as M
+from oracle import mla_oracle as O
+from tests.gpu_harness import (compare, config_of, oracle_step, run_decode_step, to_dev, to_host,
+                               torch_dtype)
+from workloads import WORKLOADS, ctx_lengths, random_cache
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from head_latent_attention_09_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def _check_step(wl, got, seqs, with_wo=False, explicit_heads=None):
+    want = oracle_step(wl, seqs, with_wo=with_wo, explicit_heads=explicit_heads)
+    compare(got["cache_new_rows"], want["cache_new_rows"], wl, "cache row", seqs)
+    compare(got["q_abs"], want["q_abs"], wl, "q_abs", seqs)
+    compare(got["ctx_lat"], want["ctx_lat"], wl, "ctx_lat", seqs)
+    compare(got["lse"], want["lse"], wl, "lse", seqs)
+    compare(got["o"], want["o"], wl, "o", seqs)
+    if with_wo:
+        compare(got["u"], want["u"], wl, "u", seqs)
+    if explicit_heads is not None:
+        g = {b: got["o"][b][list(explicit_heads)] for b in seqs}
+        compare(g, want["o_explicit"], wl, "o (explicit per-head keys)", seqs)
+
+
+# ---------------------------------------------------------------------------
+# full decode steps of the five workloads
+# ---------------------------------------------------------------------------
+
+def test_tiny_fp32_full_step():
+    wl = WORKLOADS["tiny_fp32"]
+    got = run_decode_step(wl, with_wo=True)
+    _check_step(wl, got, [0, 1], with_wo=True, explicit_heads=range(wl.n_h))
+
+
+@pytest.mark.parametrize("parts", [1, 2, 5])
+def test_tiny_fp32_split_counts(parts):
+    wl = WORKLOADS["tiny_fp32"]
+    got = run_decode_step(wl, num_parts=parts)
+    _check_step(wl, got, [0, 1])
+
+
+def test_v2lite_b32_ctx4k_full():
+    wl = WORKLOADS["v2lite_b32_ctx4k"]
+    got = run_decode_step(wl)
+    _check_step(wl, got, [0, 13, 31], explicit_heads=range(0, 16, 5))
+
+
+def test_v2_b64_ctx8k_full():
+    wl = WORKLOADS["v2_b64_ctx8k"]
+    got = run_decode_step(wl)
+    _check_step(wl, got, [0, 37, 63], explicit_heads=[0, 64, 127])
+
+
+def test_ragged_paged_full():
+    wl = WORKLOADS["v2lite_paged_ragged_b128"]
+    ctx = ctx_lengths(wl)
+    got = run_decode_step(wl)
+    seqs = sorted({int(np.argmin(ctx)), int(np.argmax(ctx)), 5, 77})
+    _check_step(wl, got, seqs, explicit_heads=[3, 11])
+
+
+def test_128k_full():
+    wl = WORKLOADS["v2lite_b4_ctx128k"]
+    got = run_decode_step(wl)
+    rng = np.random.default_rng(wl.seed)
+    heads = sorted(rng.choice(wl.n_h, 8, replace=False).tolist())
+    _check_step(wl, got, [2], explicit_heads=heads)     # 8 heads explicit, all 16 absorbed
+
+
+# ---------------------------------------------------------------------------
+# small shapes of the fast paths: ragged, empty, one-token contexts, W^O
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,ctx", [
+    ("v2_b64_ctx8k", (1, 63, 64, 65, 200, 0, 129)),
+    ("v2lite_b32_ctx4k", (1, 2, 64, 100, 0, 1000, 4097)),
+])
+def test_small_ragged_steps(name, ctx):
+    wl = WORKLOADS[name].with_(B=len(ctx), ctx=ctx)
+    got = run_decode_step(wl, with_wo=True)
+    seqs = [b for b in range(wl.B) if ctx[b] > 0]
+    _check_step(wl, got, seqs, with_wo=True)
+    for b in range(wl.B):
+        if ctx[b] == 0:
+            assert np.all(got["ctx_lat"][b] == 0) and np.all(np.isneginf(got["lse"][b]))
+
+
+def test_paged_small():
+    wl = WORKLOADS["v2lite_paged_ragged_b128"].with_(B=6, ctx=(1, 64, 65, 300, 1, 130))
+    got = run_decode_step(wl)
+    _check_step(wl, got, list(range(6)))
+
+
+# ---------------------------------------------------------------------------
+# the attention step alone on drawn caches
+# ---------------------------------------------------------------------------
+
+def _attention_only(wl, ctx, parts, q_scale=0.5, cache_std=1.0, plant=None):
+    cfg = config_of(wl)
+    handle = M.mla_create(cfg)
+    try:
+        ctx = np.asarray(ctx)
+        B, T = len(ctx), int(max(1, ctx.max()))
+        w2 = wl.with_(B=B)
+        rows = random_cache(w2, T, cache_std)                       # [B, T, D]
+        rng = np.random.default_rng(1234)
+        q = rng.standard_normal((B, wl.n_h, wl.D)).astype(np.float32) * q_scale
+        if plant is not None:
+            plant(rows, q)
+        from workloads import bf16_round
+        if wl.dtype == "bf16":
+            q = bf16_round(q)
+        for b in range(B):                                         # garbage past each context
+            rows[b, ctx[b]:] = np.nan
+        cache = to_dev(rows, wl)
+        q_d = to_dev(q, wl)
+        ctx_d = torch.from_numpy(ctx.astype(np.int32)).cuda()
+        ws_bytes = M.mla_decode_workspace_size(handle, B, parts)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        out = torch.empty((B, wl.n_h, wl.d_c), dtype=torch_dtype(wl), device="cuda")
+        lse = torch.empty((B, wl.n_h), dtype=torch.float32, device="cuda")
+        M.mla_decode_attn(handle, q_d, cache, T, None, 0, ctx_d, B, parts, ws, ws_bytes)
+        M.mla_combine_splits(handle, ws, ws_bytes, B, parts, out, lse)
+        assert M.mla_get_device_status(handle) == M.MLA_OK
+        got_ctx, got_lse = to_host(out), to_host(lse)
+    finally:
+        M.mla_destroy(handle)
+    scale = O.softmax_scale(wl.d_h, wl.d_r)
+    want_ctx, want_lse = {}, {}
+    for b in range(B):
+        want_ctx[b], want_lse[b] = O.latent_attention(q[b], rows[b, :ctx[b]], d_c=wl.d_c,
+                                                      scale=scale)
+    return got_ctx, got_lse, want_ctx, want_lse
+
+
+@pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k", "tiny_fp32"])
+@pytest.mark.parametrize("parts", [1, 3, 16, 74, 148, 5000])
+def test_attention_split_counts(name, parts):
+    wl = WORKLOADS[name]
+    ctx = [700, 1, 64, 0, 129, 2000, 63]
+    gc, gl, wc, wlse = _attention_only(wl, ctx, parts)
+    seqs = [b for b in range(len(ctx)) if ctx[b] > 0]
+    compare(gc, wc, wl, f"ctx_lat parts={parts}", seqs)
+    compare(gl, wlse, wl, f"lse parts={parts}", seqs)
+    assert np.all(gc[3] == 0) and np.all(np.isneginf(gl[3]))
+
+
+@pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k"])
+def test_attention_late_dominant_key(name):
+    """A key far above the others late in the sequence forces the running
+    maximum to jump (the rescale path)."""
+    wl = WORKLOADS[name]
+
+    def plant(rows, q):
+        rows[:, 1500, :] = 0.0
+        rows[:, 1500, 0] = 30.0
+        rows[:, 1500, 1] = 5.0
+        q[:, :, :] *= 0.1
+        q[:, :, 0] = 4.0
+
+    ctx = [1800, 1600]
+    gc, gl, wc, wlse = _attention_only(wl, ctx, 7, plant=plant)
+    compare(gc, wc, wl, "ctx_lat dominant", [0, 1])
+    compare(gl, wlse, wl, "lse dominant", [0, 1])
