@@ -1,0 +1,559 @@
+// Split-KV decode attention over the latent cache for 128 heads (DeepSeek-V2
+// shapes: d_c = 512, d_h^R = 64, bf16), on pairs of SMs.
+//
+// What it computes (absorbed MLA, "DeepSeek-V2", Appendix C; softmax of the
+// "DeepSeek-V3" note's o_{t,i}): for every (sequence, share) piece,
+//   s_j   = q_abs_i . [c_j ; k^R_j] / sqrt(d_h + d_h^R)
+//   ctx_i = sum_j softmax_j(s) c_j      and   lse_i = log sum_j e^{s_j}
+// over the piece's tokens, written as fp32 partials for the log-sum-exp merge.
+//
+// Why a pair: the output accumulator of 128 heads x 512 latent columns in fp32
+// is 256 KB -- all of one SM's tensor memory -- so it is split across the two
+// SMs of a cluster, 64 heads each, and the MMAs are pair MMAs
+// (tcgen05.mma.cta_group::2, M = 128).  A pair MMA takes half of A's rows and
+// half of B's columns from each CTA's shared memory:
+//   S = Q K^T  (N = 128 tokens): CTA r holds Q rows 64r.. and tokens 64r.. of
+//               the tile; each CTA receives S for its 64 heads x 128 tokens,
+//               folded into 128 lanes x 64 columns (lanes 64.. = tokens 64..).
+//   O += P V   (N = 256 latent columns per MMA, two MMAs): CTA r holds P for
+//               its heads and columns 128r.. of each 256-column group; each CTA
+//               accumulates O for its 64 heads x 512 columns in 256 columns.
+// The cache is therefore staged twice per CTA -- once token-split for S, once
+// column-split for O -- which doubles L2->SM traffic but reads HBM once and
+// needs no exchange of partial scores.
+//
+// Warp roles per CTA (192 threads): warp 0 TMA producer, warp 1 tensor-memory
+// allocation and (leader CTA only) MMA issue, warps 2-5 softmax, O rescale and
+// epilogue (one thread per tensor-memory lane).
+//
+// Every wait is bounded; a wait that runs out flags MLA_ERR_TIMEOUT and the
+// kernel winds down without further waits.
+#include <math_constants.h>
+
+#include "ptx.cuh"
+
+namespace mla {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kNS = 12;                 // ring stages
+constexpr int kStage = 8192;            // bytes per ring stage
+constexpr int kQBytes = 9 * 8192;       // 64 heads x 576 bf16, nine 64-column chunks
+constexpr int kPBytes = 16384;          // 64 heads x 128 tokens bf16 (two 64-token chunks)
+constexpr int kTileTok = 128;           // tokens per MMA tile
+constexpr float kRescale = 8.0f;        // rescale O only when the running max grows by > 2^8
+
+constexpr int kOffQ = 0;
+constexpr int kOffRing = kOffQ + kQBytes;
+constexpr int kOffP = kOffRing + kNS * kStage;
+constexpr int kOffRed = kOffP + 2 * kPBytes;            // float red_m[2][128], red_l[128]
+constexpr int kOffBar = kOffRed + 3 * 128 * 4;
+// barriers
+constexpr int kBarFull = 0;                 // [kNS]  leader: 2 arrivals + tx
+constexpr int kBarEmpty = kBarFull + kNS;   // [kNS]  both: pair commit
+constexpr int kBarQFull = kBarEmpty + kNS;  // leader: 2 arrivals + tx
+constexpr int kBarQEmpty = kBarQFull + 1;   // both: pair commit
+constexpr int kBarSFull = kBarQEmpty + 1;   // [2] both: pair commit
+constexpr int kBarPFull = kBarSFull + 2;    // [2] leader: 8 warp arrivals
+constexpr int kBarPFree = kBarPFull + 2;    // [2] both: pair commit
+constexpr int kBarODone = kBarPFree + 2;    // both: pair commit after each PV
+constexpr int kBarOFree = kBarODone + 1;    // leader: 8 warp arrivals
+constexpr int kBarXchg = kBarOFree + 1;     // [2] local: 4 softmax-warp arrivals (row-max exchange)
+constexpr int kBarLsum = kBarXchg + 2;      // local: 4 softmax-warp arrivals (row-sum exchange)
+constexpr int kNumBars = kBarLsum + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 16;
+constexpr int kSmemAlloc = kSmemBytes + 1024;
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+
+constexpr uint32_t kTmemCols = 512;         // S: cols 0..127 (2 x 64), O: cols 128..383
+constexpr uint32_t kColO = 128;
+
+constexpr uint32_t kIdescQK = idesc_bf16(128, kTileTok, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16(128, 256, false, true);
+
+struct Piece {
+  int b;
+  long long piece;     // global piece index
+  int tok_begin;       // first token of the piece in sequence b
+  int tok_end;         // one past the last token attended by this piece
+  int ctx;             // the sequence's context length (clamped to the cache)
+  int ntiles;          // 128-token MMA tiles
+};
+
+struct Walk {
+  const long long *tp;
+  const long long *pb;
+  long long P, Ttot, t0, t1;
+  int b;
+  int B;
+};
+
+__device__ __forceinline__ void walk_init(Walk &w, const AttnArgs &a, int share) {
+  const WsHeader *hd = reinterpret_cast<const WsHeader *>(a.ws);
+  w.P = hd->P;
+  w.Ttot = hd->Ttot;
+  w.tp = reinterpret_cast<const long long *>(a.ws + a.L.tile_prefix_off);
+  w.pb = reinterpret_cast<const long long *>(a.ws + a.L.piece_base_off);
+  w.B = a.B;
+  if (share >= w.P) {
+    w.b = a.B;
+    return;
+  }
+  w.t0 = plan_begin(share, w.P, w.Ttot);
+  w.t1 = plan_begin(share + 1, w.P, w.Ttot);
+  int lo = 0, hi = a.B;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (w.tp[mid + 1] <= w.t0) lo = mid + 1; else hi = mid;
+  }
+  w.b = lo;
+}
+
+// Next piece of this share; false when done.
+__device__ __forceinline__ bool walk_next(Walk &w, const AttnArgs &a, int share, Piece &pc) {
+  while (w.b < w.B && w.tp[w.b] < w.t1) {
+    const int b = w.b++;
+    const long long s0 = w.t0 > w.tp[b] ? w.t0 : w.tp[b];
+    const long long s1 = w.t1 < w.tp[b + 1] ? w.t1 : w.tp[b + 1];
+    if (s0 >= s1) continue;
+    int ctx = a.ctx_len[b];
+    if (a.page_size == 0 && ctx > a.cache_len) ctx = (int)a.cache_len;
+    pc.b = b;
+    pc.piece = w.pb[b] + (share - plan_share_of_tile(w.tp[b], w.P, w.Ttot));
+    pc.tok_begin = (int)((s0 - w.tp[b]) * kTile);
+    const long long e = (s1 - w.tp[b]) * kTile;
+    pc.tok_end = (int)(e < ctx ? e : ctx);
+    pc.ctx = ctx;
+    pc.ntiles = (pc.tok_end - pc.tok_begin + kTileTok - 1) / kTileTok;
+    return true;
+  }
+  return false;
+}
+
+// Cache row of token t of sequence b, or -1 (unmapped / outside the cache).
+__device__ __forceinline__ long long kv_row(const AttnArgs &a, int b, int t) {
+  if (a.page_size == 0) return (long long)b * a.cache_len + t;
+  const int bi = t / kTile;
+  if (bi >= a.max_blocks) return -1;
+  const int blk = a.block_table[(long long)b * a.max_blocks + bi];
+  if (blk < 0 || blk >= a.cache_len) return -1;
+  return (long long)blk * kTile + (t % kTile);
+}
+
+struct Bars {
+  uint64_t *b;
+  __device__ uint64_t *full(int s) { return b + kBarFull + s; }
+  __device__ uint64_t *empty(int s) { return b + kBarEmpty + s; }
+  __device__ uint64_t *qfull() { return b + kBarQFull; }
+  __device__ uint64_t *qempty() { return b + kBarQEmpty; }
+  __device__ uint64_t *sfull(int i) { return b + kBarSFull + i; }
+  __device__ uint64_t *pfull(int i) { return b + kBarPFull + i; }
+  __device__ uint64_t *pfree(int i) { return b + kBarPFree + i; }
+  __device__ uint64_t *odone() { return b + kBarODone; }
+  __device__ uint64_t *ofree() { return b + kBarOFree; }
+  __device__ uint64_t *xchg(int i) { return b + kBarXchg + i; }
+  __device__ uint64_t *lsum() { return b + kBarLsum; }
+};
+
+// Warp-uniform bounded wait: lane 0 waits, the result is broadcast, the other
+// lanes then observe the completed phase themselves (acquire).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned *status,
+                                          volatile int *abort) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, status, abort, true);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok && (threadIdx.x & 31) != 0) ptx::mbar_try_wait_cluster(bar, parity);
+  __syncwarp();
+  return ok;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                     const __grid_constant__ CUtensorMap mapV, const AttnArgs a, const long long kv_rows) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = sm + kOffQ;
+  uint8_t *sRing = sm + kOffRing;
+  uint8_t *sP = sm + kOffP;
+  float *red_m = reinterpret_cast<float *>(sm + kOffRed);   // [2][128]
+  float *red_l = red_m + 256;                                 // [128]
+  Bars bars{reinterpret_cast<uint64_t *>(sm + kOffBar)};
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int share = blockIdx.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      ptx::mbar_init(bars.full(s), 2);
+      ptx::mbar_init(bars.empty(s), 1);
+    }
+    ptx::mbar_init(bars.qfull(), 2);
+    ptx::mbar_init(bars.qempty(), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bars.sfull(i), 1);
+      ptx::mbar_init(bars.pfull(i), 8);
+      ptx::mbar_init(bars.pfree(i), 1);
+    }
+    ptx::mbar_init(bars.odone(), 1);
+    ptx::mbar_init(bars.ofree(), 8);
+    ptx::mbar_init(bars.xchg(0), 4);
+    ptx::mbar_init(bars.xchg(1), 4);
+    ptx::mbar_init(bars.lsum(), 4);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync_all();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint32_t lq = ptx::leader_addr(bars.qfull());
+    Walk w;
+    walk_init(w, a, share);
+    Piece pc;
+    int sc = 0, npc = 0;
+    bool have_prev = false, ok = true;
+    Piece prev;
+    int prev_tok0 = 0;
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&mapQ);
+      ptx::tma_prefetch_desc(&mapK);
+      ptx::tma_prefetch_desc(&mapV);
+    }
+    auto acquire_stage = [&](int &s) -> bool {
+      s = sc % kNS;
+      if (sc >= kNS && !warp_wait(bars.empty(s), ((sc / kNS) - 1) & 1, a.status, abort_flag)) return false;
+      return true;
+    };
+    // arm the leader's full barrier for stage s: tx bytes from both CTAs (or 0)
+    auto arm = [&](int s, uint32_t bytes_both) {
+      if (lane == 0) {
+        if (leader) ptx::mbar_arrive_expect_tx(bars.full(s), bytes_both);
+        else ptx::mbar_arrive_remote_addr(ptx::leader_addr(bars.full(s)));
+      }
+    };
+    auto produce_v = [&](const Piece &p, int tile_tok0) -> bool {
+      for (int g = 0; g < 2; ++g) {
+        for (int kb = 0; kb < 4; ++kb) {
+          int s;
+          if (!acquire_stage(s)) return false;
+          uint8_t *dst = sRing + s * kStage;
+          const int tok0 = tile_tok0 + 32 * kb;
+          const int feat0 = 256 * g + 128 * (int)rank;
+          if (tok0 < p.tok_end && tok0 + 32 > p.ctx) {
+            // The block runs past the sequence: copy the valid rows by hand and
+            // zero the rest, so that no unwritten cache row (possibly NaN)
+            // reaches the P.V product.  128-byte rows, 16-byte units swizzled
+            // by row (the layout a 128-byte-swizzled TMA load would produce).
+            for (int u = lane; u < 2 * 32 * 8; u += 32) {
+              const int half = u >> 8, row = (u >> 3) & 31, c = u & 7;
+              const int t = tok0 + row;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (t < p.ctx) {
+                const long long r = kv_row(a, p.b, t);
+                if (r >= 0) {
+                  const uint4 *src = reinterpret_cast<const uint4 *>(
+                      reinterpret_cast<const __nv_bfloat16 *>(a.cache) + r * 576 + feat0 + 64 * half + 8 * c);
+                  v = *src;
+                } else {
+                  atomicOr(a.status, kStatusBounds);
+                }
+              }
+              *reinterpret_cast<uint4 *>(dst + half * 4096 + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            arm(s, 0);
+          } else {
+            int y = (int)kv_rows;   // out of range: TMA fills zeros
+            if (tok0 < p.tok_end) {
+              const long long r = kv_row(a, p.b, tok0);
+              if (r >= 0) y = (int)r;
+              else if (lane == 0) atomicOr(a.status, kStatusBounds);
+            }
+            arm(s, 2 * kStage);
+            if (lane == 0) {
+              const uint32_t lb = ptx::leader_addr(bars.full(s));
+              ptx::tma_load_2d_pair(dst, &mapV, lb, feat0, y);
+              ptx::tma_load_2d_pair(dst + 4096, &mapV, lb, feat0 + 64, y);
+            }
+          }
+          ++sc;
+        }
+      }
+      return true;
+    };
+
+    while (ok && walk_next(w, a, share, pc)) {
+      if (npc > 0 && !warp_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (lane == 0) {
+        if (leader) ptx::mbar_arrive_expect_tx(bars.qfull(), 2 * kQBytes);
+        else ptx::mbar_arrive_remote_addr(lq);
+        for (int c = 0; c < 9; ++c)
+          ptx::tma_load_2d_pair(sQ + c * 8192, &mapQ, lq, 64 * c, pc.b * 128 + 64 * (int)rank);
+      }
+      for (int k = 0; k < pc.ntiles && ok; ++k) {
+        const int tile_tok0 = pc.tok_begin + kTileTok * k;
+        const int half_tok0 = tile_tok0 + 64 * (int)rank;
+        int y = (int)kv_rows;
+        if (half_tok0 < pc.tok_end) {
+          const long long r = kv_row(a, pc.b, half_tok0);
+          if (r >= 0) y = (int)r;
+          else if (lane == 0) atomicOr(a.status, kStatusBounds);
+        }
+        for (int c = 0; c < 9; ++c) {
+          int s;
+          if (!acquire_stage(s)) { ok = false; break; }
+          arm(s, 2 * kStage);
+          if (lane == 0) ptx::tma_load_2d_pair(sRing + s * kStage, &mapK, ptx::leader_addr(bars.full(s)), 64 * c, y);
+          ++sc;
+        }
+        if (!ok) break;
+        if (have_prev && !produce_v(prev, prev_tok0)) { ok = false; break; }
+        prev = pc;
+        prev_tok0 = tile_tok0;
+        have_prev = true;
+      }
+      ++npc;
+    }
+    if (ok && have_prev) produce_v(prev, prev_tok0);
+    if (*abort_flag) {
+      // let loads already issued into this CTA's shared memory land
+      const unsigned long long t0 = ptx::globaltimer();
+      while (ptx::globaltimer() - t0 < 100000ull) {}
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (leader && lane == 0) {
+      Walk w;
+      walk_init(w, a, share);
+      Piece pc;
+      int sc = 0, npc = 0, i = 0;
+      bool ok = true;
+      struct PrevTile { int i, first, npc; } prev{0, 0, 0};
+      bool have_prev = false;
+      const uint32_t q0 = ptx::smem_u32(sQ), r0 = ptx::smem_u32(sRing), p0 = ptx::smem_u32(sP);
+      auto pv = [&](const PrevTile &t) -> bool {
+        if (t.first && t.npc > 0 &&
+            !ptx::mbar_wait(bars.ofree(), (t.npc - 1) & 1, a.status, abort_flag, true))
+          return false;
+        if (!ptx::mbar_wait(bars.pfull(t.i & 1), (t.i >> 1) & 1, a.status, abort_flag, true)) return false;
+        ptx::tc_fence_after();
+        const uint32_t pbase = p0 + (t.i & 1) * kPBytes;
+        for (int g = 0; g < 2; ++g) {
+          for (int kb = 0; kb < 4; ++kb) {
+            const int s = sc % kNS;
+            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag, true)) return false;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int tau = 32 * kb + 16 * j;
+              const uint64_t ad = ptx::sdesc(pbase + (tau >> 6) * 8192 + ((tau & 63) >> 4) * 32, 16, 1024, 2);
+              const uint64_t bd = ptx::sdesc(r0 + s * kStage + j * 2048, 4096, 1024, 2);
+              ptx::mma_bf16_ss_pair(tmem + kColO + 128 * g, ad, bd, kIdescPV,
+                                    (t.first && kb == 0 && j == 0) ? 0u : 1u);
+            }
+            ptx::mma_commit_pair_both(bars.empty(s));
+            ++sc;
+          }
+        }
+        ptx::mma_commit_pair_both(bars.pfree(t.i & 1));
+        ptx::mma_commit_pair_both(bars.odone());
+        return true;
+      };
+      while (ok && walk_next(w, a, share, pc)) {
+        if (!ptx::mbar_wait(bars.qfull(), npc & 1, a.status, abort_flag, true)) { ok = false; break; }
+        for (int k = 0; k < pc.ntiles && ok; ++k) {
+          for (int c = 0; c < 9; ++c) {
+            const int s = sc % kNS;
+            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag, true)) { ok = false; break; }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t ad = ptx::sdesc(q0 + c * 8192 + 32 * j, 16, 1024, 2);
+              const uint64_t bd = ptx::sdesc(r0 + s * kStage + 32 * j, 16, 1024, 2);
+              ptx::mma_bf16_ss_pair(tmem + (i & 1) * 64, ad, bd, kIdescQK, (c | j) != 0 ? 1u : 0u);
+            }
+            ptx::mma_commit_pair_both(bars.empty(s));
+            ++sc;
+          }
+          if (!ok) break;
+          ptx::mma_commit_pair_both(bars.sfull(i & 1));
+          if (k == pc.ntiles - 1) ptx::mma_commit_pair_both(bars.qempty());
+          if (have_prev && !pv(prev)) { ok = false; break; }
+          prev = {i, k == 0 ? 1 : 0, npc};
+          have_prev = true;
+          ++i;
+        }
+        ++npc;
+      }
+      if (ok && have_prev) pv(prev);
+    }
+  } else {
+    // ------------------------------------------- softmax, rescale, epilogue
+    const int q = warp & 3;
+    const int l = q * 32 + lane;          // tensor-memory lane of this thread
+    const int h = l & 63, th = l >> 6;    // local head, token half
+    const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+    const uint32_t leader_pfull0 = ptx::leader_addr(bars.pfull(0));
+    const uint32_t leader_ofree = ptx::leader_addr(bars.ofree());
+    float *opart = reinterpret_cast<float *>(a.ws + a.L.opart_off);
+    float *lse_out = reinterpret_cast<float *>(a.ws + a.L.lse_off);
+    Walk w;
+    walk_init(w, a, share);
+    Piece pc;
+    int i = 0, npc_s = 0;
+    bool ok = true;
+    while (ok && walk_next(w, a, share, pc)) {
+      float m_run = -CUDART_INF_F, l_part = 0.f;
+      for (int k = 0; k < pc.ntiles; ++k, ++i) {
+        const int base = pc.tok_begin + kTileTok * k + 64 * th;
+        const int nvalid = min(max(pc.tok_end - base, 0), 64);
+        if (!warp_wait(bars.sfull(i & 1), (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        float s[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[16];
+          ptx::tmem_ld16(lane_addr + (i & 1) * 64 + 16 * c, r);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(r[j]);
+        }
+        float mloc = -CUDART_INF_F;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          s[j] = j < nvalid ? s[j] * a.scale_log2 : -CUDART_INF_F;
+          mloc = fmaxf(mloc, s[j]);
+        }
+        red_m[(i & 1) * 128 + l] = mloc;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bars.xchg(i & 1));
+        if (!warp_wait(bars.xchg(i & 1), (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+        const float m_tile = fmaxf(mloc, red_m[(i & 1) * 128 + (l ^ 64)]);
+        bool rescale = false;
+        float alpha = 1.f;
+        if (m_tile > m_run + kRescale) {
+          alpha = exp2f(m_run - m_tile);       // 0 when m_run = -inf
+          m_run = m_tile;
+          l_part *= alpha;
+          rescale = k > 0;
+        }
+        uint32_t pk[32];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float p0 = exp2f(s[2 * j] - m_run), p1 = exp2f(s[2 * j + 1] - m_run);
+          sum += p0 + p1;
+          __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
+          pk[j] = *reinterpret_cast<uint32_t *>(&v);
+        }
+        l_part += sum;
+        if (i >= 2 && !warp_wait(bars.pfree(i & 1), ((i >> 1) - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+        uint8_t *prow = sP + (i & 1) * kPBytes + th * 8192 + h * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        if (rescale) {
+          if (!warp_wait(bars.odone(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t r[16];
+            ptx::tmem_ld16(lane_addr + kColO + 16 * c, r);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+            ptx::tmem_st16(lane_addr + kColO + 16 * c, r);
+          }
+          ptx::tmem_st_wait();
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_remote_addr(leader_pfull0 + 8 * (i & 1));
+      }
+      if (!ok) break;
+      // ---- epilogue of the piece: O / l and the log-sum-exp
+      red_l[l] = l_part;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bars.lsum());
+      if (!warp_wait(bars.lsum(), npc_s & 1, a.status, abort_flag)) { ok = false; break; }
+      ++npc_s;
+      const float lsum = l_part + red_l[l ^ 64];
+      if (!warp_wait(bars.odone(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const int head = 64 * (int)rank + h;
+      float *dst = opart + (pc.piece * a.n_h + head) * (long long)a.d_c + 128 * th;
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {
+        uint32_t r[16];
+        ptx::tmem_ld16(lane_addr + kColO + 16 * c, r);
+        ptx::tmem_ld_wait();
+        float *d = dst + (c >> 3) * 256 + (c & 7) * 16;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4 *>(d + j) =
+              make_float4(__uint_as_float(r[j]) * inv, __uint_as_float(r[j + 1]) * inv,
+                          __uint_as_float(r[j + 2]) * inv, __uint_as_float(r[j + 3]) * inv);
+      }
+      if (th == 0)
+        lse_out[pc.piece * a.n_h + head] =
+            lsum > 0.f ? (m_run + log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_remote_addr(leader_ofree);
+      // red_l is rewritten only after the next piece's per-tile exchanges
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  ptx::tc_fence_before();
+  __syncwarp();
+  ptx::cluster_sync_all();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
+  if (a.n_h != 128 || a.d_c != 512 || a.d_r != 64) return cudaErrorNotSupported;
+  if (a.page_size != 0 && a.page_size != kTile) return cudaErrorNotSupported;
+  const long long rows = a.page_size ? a.cache_len * kTile : (long long)a.B * a.cache_len;
+  if (rows <= 0 || rows >= (1ll << 31) - 256) return cudaErrorNotSupported;
+  CUtensorMap mq, mk, mv;
+  const uint64_t dq[2] = {576, (uint64_t)a.B * 128};
+  const uint64_t dkv[2] = {576, (uint64_t)rows};
+  const uint64_t st[1] = {576 * 2};
+  const uint32_t bq[2] = {64, 64}, bk[2] = {64, 64}, bv[2] = {64, 32};
+  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mk, a.cache, 2, dkv, st, bk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mv, a.cache, 2, dkv, st, bv, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorNotSupported;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  attn_pair_kernel<<<2 * P, kThreads, kSmemAlloc, s>>>(mq, mk, mv, a, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace mla
