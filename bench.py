@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--num-parts", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the batch size (small cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -221,6 +223,8 @@ def run_ours(args):
     M.load()
 
     wl = WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(B=args.batch, ctx=(wl.ctx[0],) * args.batch)
     B, H, D, d = wl.B, wl.n_h, wl.D, wl.d_model
     ctx = np.asarray(wl.ctx, dtype=np.int64)
     cfg = M.mla_config(n_h=H, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, d_model=d,
@@ -263,16 +267,24 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
-    def step(ev_pair=None):
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
         M.mla_cache_append(handle, h_new, B, 1, pos, w_dkv, w_kr, cache, cap, None, 0, sh)
+        if ev is not None:
+            ev[1].record(stream)
         M.mla_absorb_q(handle, q_nope, q_rope, pos, w_uk, q_abs, B, sh)
-        if ev_pair is not None:
-            ev_pair[0].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
         M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, ctx_d, B, P, ws, ws_bytes, sh)
-        if ev_pair is not None:
-            ev_pair[1].record(stream)
+        if ev is not None:
+            ev[3].record(stream)
         M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
+        if ev is not None:
+            ev[4].record(stream)
         M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+        if ev is not None:
+            ev[5].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -283,22 +295,24 @@ def run_ours(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
+    call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t_start.record(stream)
     for i in range(args.steps):
-        step(attn_ev[i])
+        step(call_ev[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_ev]))
+    names = ["cache_append", "absorb_q", "decode_attn", "combine_splits", "out_proj"]
+    per_call = {n: float(np.mean([ev[j].elapsed_time(ev[j + 1]) for ev in call_ev])) * 1e3
+                for j, n in enumerate(names)}
+    attn_ms = per_call["decode_attn"] * 1e-3
     st = M.mla_get_device_status(handle, sh)
     if st != M.MLA_OK:
         raise M.MlaError(st, "device status after timing")
@@ -379,6 +393,7 @@ def run_ours(args):
         "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 6 * args.steps,
+        "per_call_us": per_call,
         "clocks": clk,
         "cpu_baseline": cpu,
     }

@@ -466,9 +466,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        if (rescale) {
+        // P.V of the previous tile of this piece must be complete before O is
+        // touched.  o_done completes once per P.V and a parity wait may lag by
+        // at most one phase, so every completion is observed here in order
+        // (the first tile of a piece relies on the previous piece's epilogue).
+        if (k > 0) {
           if (!warp_wait(bars.odone(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
           ptx::tc_fence_after();
+        }
+        if (rescale) {
 #pragma unroll 1
           for (int c = 0; c < 16; ++c) {
             uint32_t r[16];
