@@ -83,15 +83,32 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  On time-out sets the
 // status word's timeout bit and `*abort`, and returns false.  If `*abort` is
 // already set the wait gives up at once.
+//
+// The wait polls with the non-blocking test_wait: a suspended try_wait was
+// measured to resume microseconds after phases completed by tcgen05.commit
+// arrivals, which serialised the pipelines.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *status,
-                                          volatile int *abort, bool cluster_scope = false) {
-  if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+                                          volatile int *abort) {
+  if (mbar_test_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
@@ -271,9 +288,29 @@ __device__ __forceinline__ void mma_commit_pair_both(uint64_t *bar) {
           smem_u32(bar))
       : "memory");
 }
-// Remote arrive on a barrier given by its shared::cluster address.
+// Arrive on a barrier given by its shared::cluster address (possibly the peer
+// CTA's).  Default (CTA-scope) release semantics: a cluster-scope release acts
+// as a heavyweight fence; ordering of shared-memory data the tensor core reads
+// is provided by fence.proxy.async before the arrive.
 __device__ __forceinline__ void mbar_arrive_remote_addr(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+
+// shared::cluster address of this CTA's shared-memory address `a` in CTA `cta`.
+__device__ __forceinline__ uint32_t mapa_peer(uint32_t a, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(cta));
+  return r;
+}
+__device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 
 }  // namespace ptx

@@ -49,15 +49,15 @@ constexpr int kOffP = kOffRing + kNS * kStage;
 constexpr int kOffRed = kOffP + 2 * kPBytes;            // float red_m[2][128], red_l[128]
 constexpr int kOffBar = kOffRed + 3 * 128 * 4;
 // barriers
-constexpr int kBarFull = 0;                 // [kNS]  leader: 2 arrivals + tx
+constexpr int kBarFull = 0;                 // [kNS]  leader: 1 arrival (+ tx bytes of both CTAs)
 constexpr int kBarEmpty = kBarFull + kNS;   // [kNS]  both: pair commit
-constexpr int kBarQFull = kBarEmpty + kNS;  // leader: 2 arrivals + tx
+constexpr int kBarQFull = kBarEmpty + kNS;  // leader: 1 arrival + tx
 constexpr int kBarQEmpty = kBarQFull + 1;   // both: pair commit
 constexpr int kBarSFull = kBarQEmpty + 1;   // [2] both: pair commit
 constexpr int kBarPFull = kBarSFull + 2;    // [2] leader: 8 warp arrivals
 constexpr int kBarPFree = kBarPFull + 2;    // [2] both: pair commit
-constexpr int kBarODone = kBarPFree + 2;    // both: pair commit after each PV
-constexpr int kBarOFree = kBarODone + 1;    // leader: 8 warp arrivals
+constexpr int kBarODone = kBarPFree + 2;    // [2] both: pair commit after P.V of even / odd tiles
+constexpr int kBarOFree = kBarODone + 2;    // leader: 8 warp arrivals
 constexpr int kBarXchg = kBarOFree + 1;     // [2] local: 4 softmax-warp arrivals (row-max exchange)
 constexpr int kBarLsum = kBarXchg + 2;      // local: 4 softmax-warp arrivals (row-sum exchange)
 constexpr int kNumBars = kBarLsum + 1;
@@ -150,7 +150,7 @@ struct Bars {
   __device__ uint64_t *sfull(int i) { return b + kBarSFull + i; }
   __device__ uint64_t *pfull(int i) { return b + kBarPFull + i; }
   __device__ uint64_t *pfree(int i) { return b + kBarPFree + i; }
-  __device__ uint64_t *odone() { return b + kBarODone; }
+  __device__ uint64_t *odone(int i) { return b + kBarODone + i; }
   __device__ uint64_t *ofree() { return b + kBarOFree; }
   __device__ uint64_t *xchg(int i) { return b + kBarXchg + i; }
   __device__ uint64_t *lsum() { return b + kBarLsum; }
@@ -161,9 +161,9 @@ struct Bars {
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned *status,
                                           volatile int *abort) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, status, abort, true);
+  if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, status, abort);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  if (ok && (threadIdx.x & 31) != 0) ptx::mbar_try_wait_cluster(bar, parity);
+  if (ok && (threadIdx.x & 31) != 0) ptx::mbar_test_wait(bar, parity);
   __syncwarp();
   return ok;
 }
@@ -189,17 +189,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
-      ptx::mbar_init(bars.full(s), 2);
+      ptx::mbar_init(bars.full(s), 1);
       ptx::mbar_init(bars.empty(s), 1);
     }
-    ptx::mbar_init(bars.qfull(), 2);
+    ptx::mbar_init(bars.qfull(), 1);
     ptx::mbar_init(bars.qempty(), 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bars.sfull(i), 1);
       ptx::mbar_init(bars.pfull(i), 8);
       ptx::mbar_init(bars.pfree(i), 1);
     }
-    ptx::mbar_init(bars.odone(), 1);
+    ptx::mbar_init(bars.odone(0), 1);
+    ptx::mbar_init(bars.odone(1), 1);
     ptx::mbar_init(bars.ofree(), 8);
     ptx::mbar_init(bars.xchg(0), 4);
     ptx::mbar_init(bars.xchg(1), 4);
@@ -218,7 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    const uint32_t lq = ptx::leader_addr(bars.qfull());
+    const uint32_t lq = ptx::leader_addr(bars.qfull());   // Q bytes of both CTAs count here
     Walk w;
     walk_init(w, a, share);
     Piece pc;
@@ -236,12 +237,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (sc >= kNS && !warp_wait(bars.empty(s), ((sc / kNS) - 1) & 1, a.status, abort_flag)) return false;
       return true;
     };
-    // arm the leader's full barrier for stage s: tx bytes from both CTAs (or 0)
+    // The leader arms its full barrier with the bytes both CTAs' loads bring;
+    // the peer's TMA loads count on the leader's barrier directly.
     auto arm = [&](int s, uint32_t bytes_both) {
-      if (lane == 0) {
-        if (leader) ptx::mbar_arrive_expect_tx(bars.full(s), bytes_both);
-        else ptx::mbar_arrive_remote_addr(ptx::leader_addr(bars.full(s)));
-      }
+      if (lane == 0 && leader) ptx::mbar_arrive_expect_tx(bars.full(s), bytes_both);
     };
     auto produce_v = [&](const Piece &p, int tile_tok0) -> bool {
       for (int g = 0; g < 2; ++g) {
@@ -252,29 +251,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int tok0 = tile_tok0 + 32 * kb;
           const int feat0 = 256 * g + 128 * (int)rank;
           if (tok0 < p.tok_end && tok0 + 32 > p.ctx) {
-            // The block runs past the sequence: copy the valid rows by hand and
-            // zero the rest, so that no unwritten cache row (possibly NaN)
-            // reaches the P.V product.  128-byte rows, 16-byte units swizzled
-            // by row (the layout a 128-byte-swizzled TMA load would produce).
-            for (int u = lane; u < 2 * 32 * 8; u += 32) {
-              const int half = u >> 8, row = (u >> 3) & 31, c = u & 7;
-              const int t = tok0 + row;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (t < p.ctx) {
-                const long long r = kv_row(a, p.b, t);
-                if (r >= 0) {
-                  const uint4 *src = reinterpret_cast<const uint4 *>(
-                      reinterpret_cast<const __nv_bfloat16 *>(a.cache) + r * 576 + feat0 + 64 * half + 8 * c);
-                  v = *src;
-                } else {
-                  atomicOr(a.status, kStatusBounds);
+            // The block runs past the sequence: the leader copies the valid rows
+            // of both CTAs' column halves by hand and zeroes the rest, so that
+            // no unwritten cache row (possibly NaN) reaches the P.V product.
+            // 128-byte rows, 16-byte units swizzled by row (the layout a
+            // 128-byte-swizzled TMA load produces).  The peer skips the stage.
+            if (leader) {
+              const uint32_t own = ptx::smem_u32(dst), peer = ptx::mapa_peer(own, 1);
+              for (int u = lane; u < 2 * 2 * 32 * 8; u += 32) {
+                const int cta = u >> 9, half = (u >> 8) & 1, row = (u >> 3) & 31, c = u & 7;
+                const int t = tok0 + row;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (t < p.ctx) {
+                  const long long r = kv_row(a, p.b, t);
+                  if (r >= 0)
+                    v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.cache) + r * 576 +
+                                                         256 * g + 128 * cta + 64 * half + 8 * c);
+                  else
+                    atomicOr(a.status, kStatusBounds);
                 }
+                const uint32_t off = half * 4096 + row * 128 + ((c ^ (row & 7)) << 4);
+                ptx::st_shared_cluster_v4(cta ? peer + off : own + off, v);
               }
-              *reinterpret_cast<uint4 *>(dst + half * 4096 + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+              ptx::fence_acq_rel_cluster();
+              ptx::fence_proxy_async_cluster();
+              __syncwarp();
+              if (lane == 0) ptx::mbar_arrive(bars.full(s));
             }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            arm(s, 0);
           } else {
             int y = (int)kv_rows;   // out of range: TMA fills zeros
             if (tok0 < p.tok_end) {
@@ -299,7 +302,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (npc > 0 && !warp_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
       if (lane == 0) {
         if (leader) ptx::mbar_arrive_expect_tx(bars.qfull(), 2 * kQBytes);
-        else ptx::mbar_arrive_remote_addr(lq);
         for (int c = 0; c < 9; ++c)
           ptx::tma_load_2d_pair(sQ + c * 8192, &mapQ, lq, 64 * c, pc.b * 128 + 64 * (int)rank);
       }
@@ -346,15 +348,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t q0 = ptx::smem_u32(sQ), r0 = ptx::smem_u32(sRing), p0 = ptx::smem_u32(sP);
       auto pv = [&](const PrevTile &t) -> bool {
         if (t.first && t.npc > 0 &&
-            !ptx::mbar_wait(bars.ofree(), (t.npc - 1) & 1, a.status, abort_flag, true))
+            !ptx::mbar_wait(bars.ofree(), (t.npc - 1) & 1, a.status, abort_flag))
           return false;
-        if (!ptx::mbar_wait(bars.pfull(t.i & 1), (t.i >> 1) & 1, a.status, abort_flag, true)) return false;
+        if (!ptx::mbar_wait(bars.pfull(t.i & 1), (t.i >> 1) & 1, a.status, abort_flag)) return false;
         ptx::tc_fence_after();
         const uint32_t pbase = p0 + (t.i & 1) * kPBytes;
         for (int g = 0; g < 2; ++g) {
           for (int kb = 0; kb < 4; ++kb) {
             const int s = sc % kNS;
-            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag, true)) return false;
+            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag)) return false;
             ptx::tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -369,15 +371,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         ptx::mma_commit_pair_both(bars.pfree(t.i & 1));
-        ptx::mma_commit_pair_both(bars.odone());
+        ptx::mma_commit_pair_both(bars.odone(t.i & 1));
         return true;
       };
       while (ok && walk_next(w, a, share, pc)) {
-        if (!ptx::mbar_wait(bars.qfull(), npc & 1, a.status, abort_flag, true)) { ok = false; break; }
+        if (!ptx::mbar_wait(bars.qfull(), npc & 1, a.status, abort_flag)) { ok = false; break; }
         for (int k = 0; k < pc.ntiles && ok; ++k) {
           for (int c = 0; c < 9; ++c) {
             const int s = sc % kNS;
-            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag, true)) { ok = false; break; }
+            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -466,15 +468,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        // P.V of the previous tile of this piece must be complete before O is
-        // touched.  o_done completes once per P.V and a parity wait may lag by
-        // at most one phase, so every completion is observed here in order
-        // (the first tile of a piece relies on the previous piece's epilogue).
-        if (k > 0) {
-          if (!warp_wait(bars.odone(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+        // The rescale (tensor-memory loads and stores, .sync.aligned) is done by
+        // the whole warp when any of its rows needs it; other rows use alpha = 1.
+        if (__any_sync(0xffffffffu, rescale)) {
+          // P.V of the previous tile must be complete before O is rescaled.
+          // o_done[b] completes for the P.V of tiles b, b+2, ...; since S of
+          // this tile is complete, every P.V up to tile i-2 is too (MMAs of
+          // one thread complete in order), so the wait below is never more
+          // than one phase away from the barrier's state.
+          if (!warp_wait(bars.odone((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
           ptx::tc_fence_after();
-        }
-        if (rescale) {
 #pragma unroll 1
           for (int c = 0; c < 16; ++c) {
             uint32_t r[16];
@@ -499,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!warp_wait(bars.lsum(), npc_s & 1, a.status, abort_flag)) { ok = false; break; }
       ++npc_s;
       const float lsum = l_part + red_l[l ^ 64];
-      if (!warp_wait(bars.odone(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (!warp_wait(bars.odone((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       const int head = 64 * (int)rank + h;

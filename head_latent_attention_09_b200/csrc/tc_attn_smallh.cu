@@ -39,7 +39,7 @@ struct Cfg {
   static constexpr int kOffBar = kOffRed + 12 * H * 4;
   // barriers
   static constexpr int bFull = 0, bEmpty = kNS, bQFull = 2 * kNS, bQEmpty = bQFull + 1, bSFull = bQEmpty + 1,
-                       bPFull = bSFull + 2, bPFree = bPFull + 2, bODone = bPFree + 2, bOFree = bODone + 1,
+                       bPFull = bSFull + 2, bPFree = bPFull + 2, bODone = bPFree + 2, bOFree = bODone + 2,
                        bXchg = bOFree + 1, bLsum = bXchg + 2, kNumBars = bLsum + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;
@@ -114,7 +114,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, status, abort);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  if (ok && (threadIdx.x & 31) != 0) ptx::mbar_try_wait(bar, parity);
+  if (ok && (threadIdx.x & 31) != 0) ptx::mbar_test_wait(bar, parity);
   __syncwarp();
   return ok;
 }
@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar + C::bXchg + i, 4);
     }
     ptx::mbar_init(bar + C::bODone, 1);
+    ptx::mbar_init(bar + C::bODone + 1, 1);
     ptx::mbar_init(bar + C::bOFree, 4);
     ptx::mbar_init(bar + C::bLsum, 4);
     *abort_flag = 0;
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int c = 0; c < 9; ++c) ptx::mma_commit(bar + C::bEmpty + (t.slot0 + c) % NS);
         ptx::mma_commit(bar + C::bPFree + (t.i & 1));
-        ptx::mma_commit(bar + C::bODone);
+        ptx::mma_commit(bar + C::bODone + (t.i & 1));
         return true;
       };
       while (ok && walk_next(w, a, share, pc)) {
@@ -386,14 +387,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<__nv_bfloat16 *>(pt + hh * 128 + ((unit ^ (hh & 7)) << 4) + inunit) =
                 __float2bfloat16_rn(p[hh]);
         }
-        // Observe every completion of o_done in order (a parity wait may lag by
-        // at most one phase); the first tile of a piece relies on the
-        // previous piece's epilogue wait.
-        if (k > 0) {
-          if (!warp_wait(bar + C::bODone, (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
-          ptx::tc_fence_after();
-        }
         if (any_rescale) {
+          // P.V of the previous tile must be complete before O^T is rescaled.
+          // o_done[b] completes for the P.V of tiles b, b+2, ...; S^T of this
+          // tile being complete implies every P.V up to tile i-2 is (MMAs of
+          // one thread complete in order), so this wait is never more than
+          // one phase away from the barrier's state.
+          if (!warp_wait(bar + C::bODone + ((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
 #pragma unroll 1
           for (int f = 0; f < 8; ++f) {
 #pragma unroll
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (q == 0 && lane == 0)
           lse_out[pc.piece * a.n_h + hh] = l > 0.f ? (m_run[hh] + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
       }
-      if (!warp_wait(bar + C::bODone, (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (!warp_wait(bar + C::bODone + ((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
 #pragma unroll 1
       for (int f = 0; f < 8; ++f) {
