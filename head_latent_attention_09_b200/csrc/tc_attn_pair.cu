@@ -22,9 +22,14 @@
 // column-split for O -- which doubles L2->SM traffic but reads HBM once and
 // needs no exchange of partial scores.
 //
-// Warp roles per CTA (192 threads): warp 0 TMA producer, warp 1 tensor-memory
+// Staging: the cache tiles for S (K stages, 3 x 64 latent columns of 64
+// tokens, 24 KB) and for O (V stages, 64 tokens x 128 columns, 16 KB) flow
+// through separate rings with their own producer warps, so V stages waiting
+// for the softmax never hold back the next tile's K stages.
+//
+// Warp roles per CTA (224 threads): warp 0 K/Q producer, warp 1 tensor-memory
 // allocation and (leader CTA only) MMA issue, warps 2-5 softmax, O rescale and
-// epilogue (one thread per tensor-memory lane).
+// epilogue (one thread per tensor-memory lane), warp 6 V producer.
 //
 // Every wait is bounded; a wait that runs out flags MLA_ERR_TIMEOUT and the
 // kernel winds down without further waits.
@@ -35,36 +40,41 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kNS = 12;                 // ring stages
-constexpr int kStage = 8192;            // bytes per ring stage
+constexpr int kThreads = 224;
+constexpr int kKSlots = 3;              // K ring: 3 x 24 KB (one tile's nine 64-column chunks)
+constexpr int kKSlot = 3 * 8192;
+constexpr int kVSlots = 3;              // V ring: 3 x 16 KB
+constexpr int kVSlot = 2 * 8192;
 constexpr int kQBytes = 9 * 8192;       // 64 heads x 576 bf16, nine 64-column chunks
 constexpr int kPBytes = 16384;          // 64 heads x 128 tokens bf16 (two 64-token chunks)
 constexpr int kTileTok = 128;           // tokens per MMA tile
 constexpr float kRescale = 8.0f;        // rescale O only when the running max grows by > 2^8
 
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kNS * kStage;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kKSlots * kKSlot;
+constexpr int kOffP = kOffV + kVSlots * kVSlot;
 constexpr int kOffRed = kOffP + 2 * kPBytes;            // float red_m[2][128], red_l[128]
 constexpr int kOffBar = kOffRed + 3 * 128 * 4;
 // barriers
-constexpr int kBarFull = 0;                 // [kNS]  leader: 1 arrival (+ tx bytes of both CTAs)
-constexpr int kBarEmpty = kBarFull + kNS;   // [kNS]  both: pair commit
-constexpr int kBarQFull = kBarEmpty + kNS;  // leader: 1 arrival + tx
-constexpr int kBarQEmpty = kBarQFull + 1;   // both: pair commit
-constexpr int kBarSFull = kBarQEmpty + 1;   // [2] both: pair commit
-constexpr int kBarPFull = kBarSFull + 2;    // [2] leader: 8 warp arrivals
-constexpr int kBarPFree = kBarPFull + 2;    // [2] both: pair commit
-constexpr int kBarODone = kBarPFree + 2;    // [2] both: pair commit after P.V of even / odd tiles
-constexpr int kBarOFree = kBarODone + 2;    // leader: 8 warp arrivals
-constexpr int kBarXchg = kBarOFree + 1;     // [2] local: 4 softmax-warp arrivals (row-max exchange)
-constexpr int kBarLsum = kBarXchg + 2;      // local: 4 softmax-warp arrivals (row-sum exchange)
+constexpr int kBarKFull = 0;                    // [3] leader: 1 arrival + tx bytes of both CTAs
+constexpr int kBarKEmpty = kBarKFull + kKSlots; // [3] both: pair commit
+constexpr int kBarVFull = kBarKEmpty + kKSlots; // [3] leader
+constexpr int kBarVEmpty = kBarVFull + kVSlots; // [3] both
+constexpr int kBarQFull = kBarVEmpty + kVSlots; // leader: 1 arrival + tx
+constexpr int kBarQEmpty = kBarQFull + 1;       // both: pair commit
+constexpr int kBarSFull = kBarQEmpty + 1;       // [2] both: pair commit
+constexpr int kBarPFull = kBarSFull + 2;        // [2] leader: 8 warp arrivals
+constexpr int kBarPFree = kBarPFull + 2;        // [2] both: pair commit
+constexpr int kBarODone = kBarPFree + 2;        // [2] both: pair commit after P.V of even / odd tiles
+constexpr int kBarOFree = kBarODone + 2;        // leader: 8 warp arrivals
+constexpr int kBarXchg = kBarOFree + 1;         // [2] local: 4 softmax-warp arrivals (row-max exchange)
+constexpr int kBarLsum = kBarXchg + 2;          // local: 4 softmax-warp arrivals (row-sum exchange)
 constexpr int kNumBars = kBarLsum + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
-static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;         // S: cols 0..127 (2 x 64), O: cols 128..383
 constexpr uint32_t kColO = 128;
@@ -143,8 +153,10 @@ __device__ __forceinline__ long long kv_row(const AttnArgs &a, int b, int t) {
 
 struct Bars {
   uint64_t *b;
-  __device__ uint64_t *full(int s) { return b + kBarFull + s; }
-  __device__ uint64_t *empty(int s) { return b + kBarEmpty + s; }
+  __device__ uint64_t *kfull(int s) { return b + kBarKFull + s; }
+  __device__ uint64_t *kempty(int s) { return b + kBarKEmpty + s; }
+  __device__ uint64_t *vfull(int s) { return b + kBarVFull + s; }
+  __device__ uint64_t *vempty(int s) { return b + kBarVEmpty + s; }
   __device__ uint64_t *qfull() { return b + kBarQFull; }
   __device__ uint64_t *qempty() { return b + kBarQEmpty; }
   __device__ uint64_t *sfull(int i) { return b + kBarSFull + i; }
@@ -168,16 +180,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
   return ok;
 }
 
+// Row coordinate of a 64-token block starting at token t0 of the piece's
+// sequence, or an out-of-range row (TMA then fills zeros) when the block lies
+// past the piece.
+__device__ __forceinline__ int block_row(const AttnArgs &a, const Piece &p, int t0, long long kv_rows) {
+  if (t0 >= p.tok_end) return (int)kv_rows;
+  const long long r = kv_row(a, p.b, t0);
+  if (r < 0) {
+    atomicOr(a.status, kStatusBounds);
+    return (int)kv_rows;
+  }
+  return (int)r;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    attn_pair_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                     const __grid_constant__ CUtensorMap mapV, const AttnArgs a, const long long kv_rows) {
+    attn_pair_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapKV,
+                     const AttnArgs a, const long long kv_rows) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + kOffQ;
-  uint8_t *sRing = sm + kOffRing;
+  uint8_t *sK = sm + kOffK;
+  uint8_t *sV = sm + kOffV;
   uint8_t *sP = sm + kOffP;
   float *red_m = reinterpret_cast<float *>(sm + kOffRed);   // [2][128]
-  float *red_l = red_m + 256;                                 // [128]
+  float *red_l = red_m + 256;                                // [128]
   Bars bars{reinterpret_cast<uint64_t *>(sm + kOffBar)};
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
@@ -188,9 +214,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int share = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNS; ++s) {
-      ptx::mbar_init(bars.full(s), 1);
-      ptx::mbar_init(bars.empty(s), 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      ptx::mbar_init(bars.kfull(s), 1);
+      ptx::mbar_init(bars.kempty(s), 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      ptx::mbar_init(bars.vfull(s), 1);
+      ptx::mbar_init(bars.vempty(s), 1);
     }
     ptx::mbar_init(bars.qfull(), 1);
     ptx::mbar_init(bars.qempty(), 1);
@@ -198,12 +228,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bars.sfull(i), 1);
       ptx::mbar_init(bars.pfull(i), 8);
       ptx::mbar_init(bars.pfree(i), 1);
+      ptx::mbar_init(bars.odone(i), 1);
+      ptx::mbar_init(bars.xchg(i), 4);
     }
-    ptx::mbar_init(bars.odone(0), 1);
-    ptx::mbar_init(bars.odone(1), 1);
     ptx::mbar_init(bars.ofree(), 8);
-    ptx::mbar_init(bars.xchg(0), 4);
-    ptx::mbar_init(bars.xchg(1), 4);
     ptx::mbar_init(bars.lsum(), 4);
     *abort_flag = 0;
     ptx::fence_barrier_init();
@@ -218,122 +246,109 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const uint32_t lq = ptx::leader_addr(bars.qfull());   // Q bytes of both CTAs count here
-    Walk w;
-    walk_init(w, a, share);
-    Piece pc;
-    int sc = 0, npc = 0;
-    bool have_prev = false, ok = true;
-    Piece prev;
-    int prev_tok0 = 0;
+    // ------------------------------------------------- Q and K-stage producer
+    // Lane 0 issues; the leader arms each stage with the bytes both CTAs'
+    // loads bring (the peer's loads count on the leader's barrier directly).
     if (lane == 0) {
+      const uint32_t lq = ptx::leader_addr(bars.qfull());
+      const uint32_t lk0 = ptx::leader_addr(bars.kfull(0));
       ptx::tma_prefetch_desc(&mapQ);
-      ptx::tma_prefetch_desc(&mapK);
-      ptx::tma_prefetch_desc(&mapV);
-    }
-    auto acquire_stage = [&](int &s) -> bool {
-      s = sc % kNS;
-      if (sc >= kNS && !warp_wait(bars.empty(s), ((sc / kNS) - 1) & 1, a.status, abort_flag)) return false;
-      return true;
-    };
-    // The leader arms its full barrier with the bytes both CTAs' loads bring;
-    // the peer's TMA loads count on the leader's barrier directly.
-    auto arm = [&](int s, uint32_t bytes_both) {
-      if (lane == 0 && leader) ptx::mbar_arrive_expect_tx(bars.full(s), bytes_both);
-    };
-    auto produce_v = [&](const Piece &p, int tile_tok0) -> bool {
-      for (int g = 0; g < 2; ++g) {
-        for (int kb = 0; kb < 4; ++kb) {
-          int s;
-          if (!acquire_stage(s)) return false;
-          uint8_t *dst = sRing + s * kStage;
-          const int tok0 = tile_tok0 + 32 * kb;
-          const int feat0 = 256 * g + 128 * (int)rank;
-          if (tok0 < p.tok_end && tok0 + 32 > p.ctx) {
-            // The block runs past the sequence: the leader copies the valid rows
-            // of both CTAs' column halves by hand and zeroes the rest, so that
-            // no unwritten cache row (possibly NaN) reaches the P.V product.
-            // 128-byte rows, 16-byte units swizzled by row (the layout a
-            // 128-byte-swizzled TMA load produces).  The peer skips the stage.
-            if (leader) {
-              const uint32_t own = ptx::smem_u32(dst), peer = ptx::mapa_peer(own, 1);
-              for (int u = lane; u < 2 * 2 * 32 * 8; u += 32) {
-                const int cta = u >> 9, half = (u >> 8) & 1, row = (u >> 3) & 31, c = u & 7;
-                const int t = tok0 + row;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (t < p.ctx) {
-                  const long long r = kv_row(a, p.b, t);
-                  if (r >= 0)
-                    v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.cache) + r * 576 +
-                                                         256 * g + 128 * cta + 64 * half + 8 * c);
-                  else
-                    atomicOr(a.status, kStatusBounds);
-                }
-                const uint32_t off = half * 4096 + row * 128 + ((c ^ (row & 7)) << 4);
-                ptx::st_shared_cluster_v4(cta ? peer + off : own + off, v);
-              }
-              ptx::fence_acq_rel_cluster();
-              ptx::fence_proxy_async_cluster();
-              __syncwarp();
-              if (lane == 0) ptx::mbar_arrive(bars.full(s));
-            }
-          } else {
-            int y = (int)kv_rows;   // out of range: TMA fills zeros
-            if (tok0 < p.tok_end) {
-              const long long r = kv_row(a, p.b, tok0);
-              if (r >= 0) y = (int)r;
-              else if (lane == 0) atomicOr(a.status, kStatusBounds);
-            }
-            arm(s, 2 * kStage);
-            if (lane == 0) {
-              const uint32_t lb = ptx::leader_addr(bars.full(s));
-              ptx::tma_load_2d_pair(dst, &mapV, lb, feat0, y);
-              ptx::tma_load_2d_pair(dst + 4096, &mapV, lb, feat0 + 64, y);
-            }
-          }
-          ++sc;
-        }
-      }
-      return true;
-    };
-
-    while (ok && walk_next(w, a, share, pc)) {
-      if (npc > 0 && !warp_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
-      if (lane == 0) {
+      ptx::tma_prefetch_desc(&mapKV);
+      Walk w;
+      walk_init(w, a, share);
+      Piece pc;
+      int sc = 0, npc = 0;
+      bool ok = true;
+      while (ok && walk_next(w, a, share, pc)) {
+        if (npc > 0 && !ptx::mbar_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag)) break;
         if (leader) ptx::mbar_arrive_expect_tx(bars.qfull(), 2 * kQBytes);
         for (int c = 0; c < 9; ++c)
           ptx::tma_load_2d_pair(sQ + c * 8192, &mapQ, lq, 64 * c, pc.b * 128 + 64 * (int)rank);
-      }
-      for (int k = 0; k < pc.ntiles && ok; ++k) {
-        const int tile_tok0 = pc.tok_begin + kTileTok * k;
-        const int half_tok0 = tile_tok0 + 64 * (int)rank;
-        int y = (int)kv_rows;
-        if (half_tok0 < pc.tok_end) {
-          const long long r = kv_row(a, pc.b, half_tok0);
-          if (r >= 0) y = (int)r;
-          else if (lane == 0) atomicOr(a.status, kStatusBounds);
+        for (int k = 0; k < pc.ntiles && ok; ++k) {
+          const int y = block_row(a, pc, pc.tok_begin + kTileTok * k + 64 * (int)rank, kv_rows);
+          for (int kc = 0; kc < 3; ++kc) {
+            const int s = sc % kKSlots;
+            if (sc >= kKSlots && !ptx::mbar_wait(bars.kempty(s), ((sc / kKSlots) - 1) & 1, a.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (leader) ptx::mbar_arrive_expect_tx(bars.kfull(s), 2 * kKSlot);
+            uint8_t *dst = sK + s * kKSlot;
+#pragma unroll
+            for (int cc = 0; cc < 3; ++cc)
+              ptx::tma_load_2d_pair(dst + cc * 8192, &mapKV, lk0 + 8 * s, 64 * (3 * kc + cc), y);
+            ++sc;
+          }
         }
-        for (int c = 0; c < 9; ++c) {
-          int s;
-          if (!acquire_stage(s)) { ok = false; break; }
-          arm(s, 2 * kStage);
-          if (lane == 0) ptx::tma_load_2d_pair(sRing + s * kStage, &mapK, ptx::leader_addr(bars.full(s)), 64 * c, y);
-          ++sc;
-        }
-        if (!ok) break;
-        if (have_prev && !produce_v(prev, prev_tok0)) { ok = false; break; }
-        prev = pc;
-        prev_tok0 = tile_tok0;
-        have_prev = true;
+        ++npc;
       }
-      ++npc;
     }
-    if (ok && have_prev) produce_v(prev, prev_tok0);
-    if (*abort_flag) {
-      // let loads already issued into this CTA's shared memory land
-      const unsigned long long t0 = ptx::globaltimer();
-      while (ptx::globaltimer() - t0 < 100000ull) {}
+  } else if (warp == 6) {
+    // -------------------------------------------------------- V-stage producer
+    // V stage (g, h) of a tile: tokens 64h.. of the tile, latent columns
+    // 256g + 128 * rank .. +128 (this CTA's half of the 256-column group).
+    const uint32_t lv0 = ptx::leader_addr(bars.vfull(0));
+    Walk w;
+    walk_init(w, a, share);
+    Piece pc;
+    int sc = 0;
+    bool ok = true;
+    if (lane == 0) ptx::tma_prefetch_desc(&mapKV);
+    while (ok && walk_next(w, a, share, pc)) {
+      for (int k = 0; k < pc.ntiles && ok; ++k) {
+        for (int g = 0; g < 2 && ok; ++g) {
+          for (int hh = 0; hh < 2; ++hh) {
+            const int s = sc % kVSlots;
+            const int tok0 = pc.tok_begin + kTileTok * k + 64 * hh;
+            const bool manual = tok0 < pc.tok_end && tok0 + 64 > pc.ctx;
+            bool got = true;
+            if (lane == 0 && sc >= kVSlots)
+              got = ptx::mbar_wait(bars.vempty(s), ((sc / kVSlots) - 1) & 1, a.status, abort_flag);
+            if (!(__shfl_sync(0xffffffffu, got ? 1 : 0, 0))) {
+              ok = false;
+              break;
+            }
+            __syncwarp();
+            uint8_t *dst = sV + s * kVSlot;
+            if (manual) {
+              // The block runs past the sequence: the leader copies the valid
+              // rows of both CTAs' column halves by hand and zeroes the rest,
+              // so that no unwritten cache row (possibly NaN) reaches P.V.
+              // 128-byte rows, 16-byte units swizzled by row (the layout a
+              // 128-byte-swizzled TMA load produces).  The peer skips it.
+              if (leader) {
+                const uint32_t own = ptx::smem_u32(dst), peer = ptx::mapa_peer(own, 1);
+                for (int u = lane; u < 2 * 2 * 64 * 8; u += 32) {
+                  const int cta = u >> 10, half = (u >> 9) & 1, row = (u >> 3) & 63, c = u & 7;
+                  const int t = tok0 + row;
+                  uint4 v = make_uint4(0, 0, 0, 0);
+                  if (t < pc.ctx) {
+                    const long long r = kv_row(a, pc.b, t);
+                    if (r >= 0)
+                      v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.cache) +
+                                                           r * 576 + 256 * g + 128 * cta + 64 * half + 8 * c);
+                    else
+                      atomicOr(a.status, kStatusBounds);
+                  }
+                  const uint32_t off = half * 8192 + row * 128 + ((c ^ (row & 7)) << 4);
+                  ptx::st_shared_cluster_v4(cta ? peer + off : own + off, v);
+                }
+                ptx::fence_acq_rel_cluster();
+                ptx::fence_proxy_async_cluster();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bars.vfull(s));
+              }
+            } else if (lane == 0) {
+              const int y = block_row(a, pc, tok0, kv_rows);
+              if (leader) ptx::mbar_arrive_expect_tx(bars.vfull(s), 2 * kVSlot);
+              const int feat0 = 256 * g + 128 * (int)rank;
+              ptx::tma_load_2d_pair(dst, &mapKV, lv0 + 8 * s, feat0, y);
+              ptx::tma_load_2d_pair(dst + 8192, &mapKV, lv0 + 8 * s, feat0 + 64, y);
+            }
+            ++sc;
+          }
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -341,33 +356,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Walk w;
       walk_init(w, a, share);
       Piece pc;
-      int sc = 0, npc = 0, i = 0;
+      int ksc = 0, vsc = 0, npc = 0, i = 0;
       bool ok = true;
       struct PrevTile { int i, first, npc; } prev{0, 0, 0};
       bool have_prev = false;
-      const uint32_t q0 = ptx::smem_u32(sQ), r0 = ptx::smem_u32(sRing), p0 = ptx::smem_u32(sP);
+      // Descriptors are built once; the start address (bits 0-13, 16-byte
+      // units) is advanced by adding offsets.
+      const uint64_t dQ = ptx::sdesc(ptx::smem_u32(sQ), 16, 1024, 2);
+      const uint64_t dK = ptx::sdesc(ptx::smem_u32(sK), 16, 1024, 2);
+      const uint64_t dP = ptx::sdesc(ptx::smem_u32(sP), 16, 1024, 2);
+      const uint64_t dV = ptx::sdesc(ptx::smem_u32(sV), 8192, 1024, 2);
       auto pv = [&](const PrevTile &t) -> bool {
-        if (t.first && t.npc > 0 &&
-            !ptx::mbar_wait(bars.ofree(), (t.npc - 1) & 1, a.status, abort_flag))
+        if (t.first && t.npc > 0 && !ptx::mbar_wait(bars.ofree(), (t.npc - 1) & 1, a.status, abort_flag))
           return false;
         if (!ptx::mbar_wait(bars.pfull(t.i & 1), (t.i >> 1) & 1, a.status, abort_flag)) return false;
         ptx::tc_fence_after();
-        const uint32_t pbase = p0 + (t.i & 1) * kPBytes;
+        const uint32_t pofs = (t.i & 1) * (kPBytes >> 4);
         for (int g = 0; g < 2; ++g) {
-          for (int kb = 0; kb < 4; ++kb) {
-            const int s = sc % kNS;
-            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag)) return false;
+          for (int hh = 0; hh < 2; ++hh) {
+            const int s = vsc % kVSlots;
+            if (!ptx::mbar_wait(bars.vfull(s), (vsc / kVSlots) & 1, a.status, abort_flag)) return false;
             ptx::tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int tau = 32 * kb + 16 * j;
-              const uint64_t ad = ptx::sdesc(pbase + (tau >> 6) * 8192 + ((tau & 63) >> 4) * 32, 16, 1024, 2);
-              const uint64_t bd = ptx::sdesc(r0 + s * kStage + j * 2048, 4096, 1024, 2);
+            for (int j = 0; j < 4; ++j) {
+              // A = P rows (heads) x tokens 64hh + 16j.. (K-major); B = V rows
+              // (tokens 16j..) x 128 columns in two 64-column chunks 8 KB apart.
+              const uint64_t ad = dP + pofs + ((hh * 8192 + j * 32) >> 4);
+              const uint64_t bd = dV + ((s * kVSlot + j * 2048) >> 4);
               ptx::mma_bf16_ss_pair(tmem + kColO + 128 * g, ad, bd, kIdescPV,
-                                    (t.first && kb == 0 && j == 0) ? 0u : 1u);
+                                    (t.first && hh == 0 && j == 0) ? 0u : 1u);
             }
-            ptx::mma_commit_pair_both(bars.empty(s));
-            ++sc;
+            ptx::mma_commit_pair_both(bars.vempty(s));
+            ++vsc;
           }
         }
         ptx::mma_commit_pair_both(bars.pfree(t.i & 1));
@@ -377,18 +397,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (ok && walk_next(w, a, share, pc)) {
         if (!ptx::mbar_wait(bars.qfull(), npc & 1, a.status, abort_flag)) { ok = false; break; }
         for (int k = 0; k < pc.ntiles && ok; ++k) {
-          for (int c = 0; c < 9; ++c) {
-            const int s = sc % kNS;
-            if (!ptx::mbar_wait(bars.full(s), (sc / kNS) & 1, a.status, abort_flag)) { ok = false; break; }
+          for (int kc = 0; kc < 3; ++kc) {
+            const int s = ksc % kKSlots;
+            if (!ptx::mbar_wait(bars.kfull(s), (ksc / kKSlots) & 1, a.status, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint64_t ad = ptx::sdesc(q0 + c * 8192 + 32 * j, 16, 1024, 2);
-              const uint64_t bd = ptx::sdesc(r0 + s * kStage + 32 * j, 16, 1024, 2);
-              ptx::mma_bf16_ss_pair(tmem + (i & 1) * 64, ad, bd, kIdescQK, (c | j) != 0 ? 1u : 0u);
+            for (int cc = 0; cc < 3; ++cc) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint64_t ad = dQ + (((3 * kc + cc) * 8192 + 32 * j) >> 4);
+                const uint64_t bd = dK + ((s * kKSlot + cc * 8192 + 32 * j) >> 4);
+                ptx::mma_bf16_ss_pair(tmem + (i & 1) * 64, ad, bd, kIdescQK, (kc | cc | j) != 0 ? 1u : 0u);
+              }
             }
-            ptx::mma_commit_pair_both(bars.empty(s));
-            ++sc;
+            ptx::mma_commit_pair_both(bars.kempty(s));
+            ++ksc;
           }
           if (!ok) break;
           ptx::mma_commit_pair_both(bars.sfull(i & 1));
@@ -546,14 +569,13 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
   if (a.page_size != 0 && a.page_size != kTile) return cudaErrorNotSupported;
   const long long rows = a.page_size ? a.cache_len * kTile : (long long)a.B * a.cache_len;
   if (rows <= 0 || rows >= (1ll << 31) - 256) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mkv;
   const uint64_t dq[2] = {576, (uint64_t)a.B * 128};
   const uint64_t dkv[2] = {576, (uint64_t)rows};
   const uint64_t st[1] = {576 * 2};
-  const uint32_t bq[2] = {64, 64}, bk[2] = {64, 64}, bv[2] = {64, 32};
-  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mk, a.cache, 2, dkv, st, bk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mv, a.cache, 2, dkv, st, bv, CU_TENSOR_MAP_SWIZZLE_128B))
+  const uint32_t box[2] = {64, 64};
+  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mkv, a.cache, 2, dkv, st, box, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
   static bool configured = false;
   if (!configured) {
@@ -561,7 +583,7 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_pair_kernel<<<2 * P, kThreads, kSmemAlloc, s>>>(mq, mk, mv, a, rows);
+  attn_pair_kernel<<<2 * P, kThreads, kSmemAlloc, s>>>(mq, mkv, a, rows);
   return cudaGetLastError();
 }
 
