@@ -29,7 +29,8 @@ EXPORTED = (
     "mla_status_string", "mla_config_validate", "mla_create", "mla_destroy",
     "mla_cache_append", "mla_absorb_q", "mla_decode_workspace_size",
     "mla_default_num_parts", "mla_decode_attn", "mla_combine_splits", "mla_out_proj",
-    "mla_get_device_status", "mla_plan_pieces",
+    "mla_get_device_status", "mla_plan_pieces", "mla_decode_attn_combine_noalloc",
+    "mla_noalloc_scratch_bytes",
 )
 
 
@@ -72,6 +73,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_out_proj": (i, [vp, vp, vp, vp, vp, vp, i, vp]),
         "mla_get_device_status": (i, [vp, vp]),
         "mla_plan_pieces": (ll, [vp, i, i, vp]),
+        "mla_decode_attn_combine_noalloc": (i, [vp, vp, vp, ll, vp, i, vp, i, i, vp, vp, vp]),
+        "mla_noalloc_scratch_bytes": (sz, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -175,6 +178,21 @@ def mla_out_proj(handle, ctx_lat, w_uv, w_o, o, u, B, stream=None):
 
 def mla_get_device_status(handle, stream=None) -> int:
     return load().mla_get_device_status(handle, _stream(stream))
+
+
+def mla_decode_attn_combine_noalloc(handle, q_abs, cache, cache_len, block_table,
+                                    max_blocks_per_seq, ctx_len, B, num_parts, ctx_lat, lse=None,
+                                    stream=None):
+    """Attention plus combine with the library's fixed scratch array (no
+    device allocation; see include/mla.h)."""
+    _check(load().mla_decode_attn_combine_noalloc(
+        handle, _ptr(q_abs), _ptr(cache), cache_len, _ptr(block_table), max_blocks_per_seq,
+        _ptr(ctx_len), B, num_parts, _ptr(ctx_lat), _ptr(lse), _stream(stream)),
+        "mla_decode_attn_combine_noalloc")
+
+
+def mla_noalloc_scratch_bytes() -> int:
+    return load().mla_noalloc_scratch_bytes()
 
 
 def mla_plan_pieces(ctx_len, num_parts):

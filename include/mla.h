@@ -45,7 +45,9 @@
  *     mla_get_device_status() reports.  Every device-side wait is bounded; a
  *     wait that runs out sets MLA_ERR_TIMEOUT in the same word.
  *   - The library allocates device memory only in mla_create (the handle's
- *     status word and RoPE table).  The decode calls use the caller's workspace.
+ *     status word and RoPE table).  The decode calls use the caller's workspace
+ *     (mla_decode_attn_combine_noalloc uses a fixed array in the device image
+ *     instead; see its declaration).
  *   - A sequence with ctx_len = 0 produces a zero ctx_lat row and lse = -inf.
  *   - Results are deterministic for a fixed num_parts (no floating-point atomics).
  *   - A handle may be used from one host thread at a time.
@@ -173,6 +175,33 @@ int mla_get_device_status(mla_handle *handle, mla_stream_t stream);
  *   piece_base[b] .. piece_base[b+1]-1.  Returns the total number of pieces,
  *   or -1 on invalid arguments. */
 long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *piece_base);
+
+/* Allocation-free variant of mla_decode_attn followed by mla_combine_splits.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory where attention runs (code inside an
+ * allocator or memory-pool callback, runtimes that forbid cudaMalloc after
+ * start-up, embeddings that only lend the library buffers they already own).
+ * Instead of a caller workspace, the split partials live in one fixed scratch
+ * array of mla_noalloc_scratch_bytes() bytes (32 MiB) inside the library's
+ * device image; every GPU that loads the library holds it until exit.
+ *   Arguments as for mla_decode_attn, plus ctx_lat [B, n_h, d_c] (cfg.dtype)
+ *   and lse [B, n_h] float32 or NULL as for mla_combine_splits.
+ *   num_parts = 0 picks the default split count, lowered until the partials
+ *   fit the array; an explicit num_parts (or a batch) whose partials do not
+ *   fit is rejected with MLA_ERR_WORKSPACE before anything is launched.
+ * No cudaMalloc/cudaFree or allocating library call is made.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.
+ * All calls share the array and leave their partials in it; calls whose work
+ * overlaps on the GPU (unordered streams) race on it.  The array needs no
+ * zeroing: each call writes everything it reads. */
+int mla_decode_attn_combine_noalloc(mla_handle *handle, const void *q_abs, const void *cache,
+                                    long long cache_len, const int *block_table,
+                                    int max_blocks_per_seq, const int *ctx_len, int B, int num_parts,
+                                    void *ctx_lat, float *lse, mla_stream_t stream);
+
+/* Size in bytes of the scratch array mla_decode_attn_combine_noalloc uses. */
+size_t mla_noalloc_scratch_bytes(void);
 
 #ifdef __cplusplus
 }
