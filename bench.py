@@ -21,8 +21,6 @@ import argparse
 import json
 import math
 import os
-import signal
-import subprocess
 import sys
 import time
 
@@ -74,55 +72,76 @@ def algorithmic_flops(wl, ctx_sum):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """SM clock and throttle-reason samples taken DURING the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    A thread polls NVML (read-only queries) every millisecond between start()
+    and stop(), so that even a timed region of a few milliseconds gets samples
+    (an `nvidia-smi -lms` loop needs longer than that to print its first line).
+    Without NVML the record says so instead of holding numbers."""
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+    REASONS = (("hw_slowdown", 0x8), ("sw_power_cap", 0x4), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.thread = None
+        self.stop_flag = False
+        self.handle = None
+        self.err = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = "%08X:%02X:%02X.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                        props.pci_device_id)
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception as e:  # noqa: BLE001 - any NVML failure just disables sampling
+            self.err = f"nvml: {e}"
+            self.handle = None
+
+    def _poll(self):
+        nv = self.nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while True:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = int(get_reasons(self.handle))
+                self.samples.append((sm, mx, rs))
+            except Exception as e:  # noqa: BLE001
+                self.err = f"nvml poll: {e}"
+                return
+            if self.stop_flag:
+                return
+            time.sleep(0.001)
 
     def start(self):
-        try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.handle is None:
+            return
+        import threading
+        self.stop_flag = False
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+        while not self.samples and self.thread.is_alive():
+            time.sleep(0.0005)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.send_signal(signal.SIGTERM)
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return None
+        if self.thread is None:
+            return {"samples": 0, "error": self.err or "no sampler"}
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return {"samples": 0, "error": self.err or "no samples"}
+        sm = [x[0] for x in self.samples]
+        mx = [x[1] for x in self.samples]
+        reasons = sorted({n for _, _, r in self.samples for n, bit in self.REASONS if r & bit})
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_min_mhz": float(min(sm)), "reasons": reasons, "samples": len(sm),
+                "source": "nvml"}
 
 
 # ----------------------------------------------------------------------------
@@ -293,7 +312,7 @@ def run_ours(args):
     if st != M.MLA_OK:
         raise M.MlaError(st, "device status after warm-up")
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     clocks.start()
     call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// log-sum-exp combine: one block per (sequence, head)
+// log-sum-exp combine, generic form: one block per (sequence, head)
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(const char *ws, WsLayout L, int n_h, int d_c,
@@ -360,8 +360,92 @@ cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s
   return cudaGetLastError();
 }
 
+// Vectorised combine for d_c a multiple of 4 and at most 512: one warp per
+// (sequence, head), 8 per block.  The warp reduces the pieces' log-sum-exps
+// across its lanes, then each lane accumulates up to four float4 columns of
+// the weighted partials, with the loads of several pieces in flight at once.
+template <typename T>
+__device__ __forceinline__ void store4(T *dst, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float *dst, float4 v) {
+  *reinterpret_cast<float4 *>(dst) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *dst, float4 v) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t *>(&lo);
+  u.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = u;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) combine_vec_kernel(const char *ws, WsLayout L, int B, int n_h, int d_c,
+                                                          T *ctx_lat, float *lse_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + warp;   // = b * n_h + h
+  if (row >= (long long)B * n_h) return;
+  const int b = (int)(row / n_h), h = (int)(row % n_h);
+  const long long *pb = reinterpret_cast<const long long *>(ws + L.piece_base_off);
+  const float *lse = reinterpret_cast<const float *>(ws + L.lse_off);
+  const float *op = reinterpret_cast<const float *>(ws + L.opart_off);
+  const long long p0 = pb[b], p1 = pb[b + 1];
+  float m = -CUDART_INF_F;
+  for (long long p = p0 + lane; p < p1; p += 32) m = fmaxf(m, lse[p * n_h + h]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  T *dst = ctx_lat + row * d_c;
+  const int n4 = d_c / 4;
+  if (m == -CUDART_INF_F) {
+    for (int f = lane; f < n4; f += 32) store4<T>(dst + 4 * f, make_float4(0.f, 0.f, 0.f, 0.f));
+    if (lse_out && lane == 0) lse_out[row] = -CUDART_INF_F;
+    return;
+  }
+  float tot = 0.f;
+  for (long long p = p0 + lane; p < p1; p += 32) tot += expf(lse[p * n_h + h] - m);
+  tot = warp_sum(tot);
+  const float inv = 1.f / tot;
+  float4 acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (long long p = p0; p < p1; ++p) {
+    const float w = expf(lse[p * n_h + h] - m) * inv;
+    const float4 *src = reinterpret_cast<const float4 *>(op + (p * n_h + h) * (long long)d_c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int f = lane + 32 * i;
+      if (f < n4) {
+        const float4 v = __ldg(src + f);
+        acc[i].x += w * v.x;
+        acc[i].y += w * v.y;
+        acc[i].z += w * v.z;
+        acc[i].w += w * v.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int f = lane + 32 * i;
+    if (f < n4) store4<T>(dst + 4 * f, acc[i]);
+  }
+  if (lse_out && lane == 0) lse_out[row] = m + logf(tot);
+}
+
 cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
                            void *ctx_lat, float *lse, cudaStream_t s) {
+  const size_t esz = cfg.dtype == MLA_FP32 ? 4 : 2;
+  if (cfg.d_c % 4 == 0 && cfg.d_c <= 512 && ((uintptr_t)ctx_lat % (4 * esz)) == 0 &&
+      ((uintptr_t)ws % 16) == 0) {
+    const long long rows = (long long)B * cfg.n_h;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (cfg.dtype == MLA_FP32)
+      combine_vec_kernel<float><<<blocks, 256, 0, s>>>(ws, L, B, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
+    else
+      combine_vec_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(ws, L, B, cfg.n_h, cfg.d_c,
+                                                              (__nv_bfloat16 *)ctx_lat, lse);
+    return cudaGetLastError();
+  }
   dim3 grid(B, cfg.n_h);
   if (cfg.dtype == MLA_FP32)
     combine_kernel<float><<<grid, 128, 0, s>>>(ws, L, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);

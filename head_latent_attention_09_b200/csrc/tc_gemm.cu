@@ -60,7 +60,7 @@ bool encode_map_bf16(CUtensorMap *map, const void *base, int rank, const uint64_
 namespace {
 
 constexpr int kGemmThreads = 192;
-constexpr int kGemmStages = 4;
+constexpr int kMaxStages = 8;           // pipeline depth is chosen per launch (<= this)
 constexpr int kKChunk = 64;           // bf16 elements per 128-byte swizzled row
 constexpr int kABytes = 128 * kKChunk * 2;
 
@@ -68,7 +68,9 @@ enum EpiMode : int { kEpiAbsorb = 0, kEpiOutProj = 1, kEpiWo = 2, kEpiAppend = 3
 
 struct GemmParams {
   int mode;
-  int num_k_chunks;
+  int num_k_chunks;   // K / 64 of the whole product
+  int stages;         // pipeline stages of this launch (<= kMaxStages)
+  int ksplit;         // K slices per output tile (1, or a cluster of ksplit CTAs along x)
   int M_valid;        // valid output features (rows of the product)
   int N;              // valid columns (tokens or sequences)
   int a_split_tile;   // m-tiles >= a_split_tile read map A1 (append: W_KR)
@@ -114,21 +116,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(base + kGemmStages * kStage);
-  uint64_t *empty = full + kGemmStages;
-  uint64_t *accf = empty + kGemmStages;
+  const int S = g.stages;
+  const bool split = g.ksplit > 1;
+  // The stage ring; with a K split it is reused afterwards for this CTA's fp32 partial.
+  const int region = split && 128 * BN * 4 > S * kStage ? 128 * BN * 4 : S * kStage;
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + region);
+  uint64_t *empty = full + kMaxStages;
+  uint64_t *accf = empty + kMaxStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  long long *s_row = reinterpret_cast<long long *>(base + kGemmStages * kStage + 128);
+  long long *s_row = reinterpret_cast<long long *>(base + region + 256);
   int *s_pos = reinterpret_cast<int *>(s_row + BN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, nt = blockIdx.y, z = blockIdx.z;
+  // blockIdx.x = m tile * ksplit + K slice; a K split runs as one cluster of
+  // ksplit CTAs along x, so the slice index is also the CTA's cluster rank.
+  const int mt = (int)blockIdx.x / g.ksplit, zs = (int)blockIdx.x % g.ksplit;
+  const int nt = blockIdx.y, z = blockIdx.z;
+  const int per = (g.num_k_chunks + g.ksplit - 1) / g.ksplit;
+  const int kc0 = zs * per;
+  const int nk = max(0, min(g.num_k_chunks, kc0 + per) - kc0);   // K chunks of this CTA
   const int m0 = mt * 128, n0 = nt * BN;
   const bool use_a1 = mt >= g.a_split_tile;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGemmStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
@@ -153,11 +165,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ptx::tma_prefetch_desc(mA);
       ptx::tma_prefetch_desc(&mapB);
       int issued = 0;
-      for (int kc = 0; kc < g.num_k_chunks; ++kc) {
-        const int s = kc % kGemmStages;
-        if (kc >= kGemmStages &&
-            !ptx::mbar_wait(&empty[s], ((kc / kGemmStages) - 1) & 1, g.status, abort_flag))
-          break;
+      for (int kl = 0; kl < nk; ++kl) {
+        const int s = kl % S, kc = kc0 + kl;
+        if (kl >= S && !ptx::mbar_wait(&empty[s], ((kl / S) - 1) & 1, g.status, abort_flag)) break;
         ++issued;
         uint8_t *sa = base + s * kStage;
         uint8_t *sb = sa + kABytes;
@@ -173,17 +183,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         else ptx::tma_load_2d(sb, &mapB, &full[s], kc * kKChunk, n0);
       }
       // Drain: do not leave while loads into this CTA's shared memory are in flight.
-      for (int kc = issued - kGemmStages > 0 ? issued - kGemmStages : 0; kc < issued; ++kc) {
+      for (int kl = issued - S > 0 ? issued - S : 0; kl < issued; ++kl) {
         volatile int no_abort = 0;
-        ptx::mbar_wait(&full[kc % kGemmStages], (kc / kGemmStages) & 1, g.status, &no_abort);
+        ptx::mbar_wait(&full[kl % S], (kl / S) & 1, g.status, &no_abort);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, BN, A_MN, false);
-      for (int kc = 0; kc < g.num_k_chunks; ++kc) {
-        const int s = kc % kGemmStages;
-        if (!ptx::mbar_wait(&full[s], (kc / kGemmStages) & 1, g.status, abort_flag)) break;
+      for (int kl = 0; kl < nk; ++kl) {
+        const int s = kl % S;
+        if (!ptx::mbar_wait(&full[s], (kl / S) & 1, g.status, abort_flag)) break;
         ptx::tc_fence_after();
         const uint32_t sa = ptx::smem_u32(base + s * kStage);
         const uint32_t sb = sa + kABytes;
@@ -194,7 +204,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t ad = A_MN ? ptx::sdesc(sa + j * 2048, kABytes / 2, 1024, 2)
                                    : ptx::sdesc(sa + j * 32, 16, 1024, 2);
           const uint64_t bd = ptx::sdesc(sb + j * 32, 16, 1024, 2);
-          ptx::mma_bf16_ss(tmem, ad, bd, idesc, (kc | j) != 0 ? 1u : 0u);
+          ptx::mma_bf16_ss(tmem, ad, bd, idesc, (kl | j) != 0 ? 1u : 0u);
         }
         ptx::mma_commit(&empty[s]);
       }
@@ -226,7 +236,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int m = m0 + m_local;
     const bool m_ok = m < g.M_valid;
     const bool rope_tile = g.mode == kEpiAppend && use_a1;
-    if (ok) {
+    if (split) {
+      // Partial of this K slice, [BN columns][128 rows] fp32, read by the whole cluster below.
+      float *red = reinterpret_cast<float *>(base);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        const bool have = ok && nk > 0;   // a slice with no K chunks contributes zero
+        if (have) {
+          ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, r);
+          ptx::tmem_ld_wait();
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) red[(c0 + j) * 128 + m_local] = have ? __uint_as_float(r[j]) : 0.f;
+      }
+    } else if (ok) {
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         uint32_t r[16];
@@ -256,7 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-    if (g.mode == kEpiAbsorb && mt == 0) {
+    if (g.mode == kEpiAbsorb && mt == 0 && zs == 0) {
       // rotary part of the absorbed query: q_abs[b, z, d_c + 2k (+1)] = RoPE(q_rope[b, z], pos[b])
       const int npair = g.d_r / 2;
       const int ncol = min(BN, g.N - n0);
@@ -281,34 +305,142 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
+
+  if (split) {
+    // Every CTA of the cluster reaches this point (all waits above are
+    // bounded), so the two cluster barriers always complete.
+    ptx::cluster_sync_all();   // partials of all K slices are written
+    const int ks = g.ksplit;
+    if (ptx::cluster_nctarank() == (uint32_t)ks) {
+      // This CTA sums rows [zs*R, zs*R + R) of the tile over the cluster's
+      // partials, 4 rows (one float4) per item, and writes them out.
+      const int R = 128 / ks, R4 = R / 4;
+      const uint32_t red = ptx::smem_u32(base);
+      for (int idx = threadIdx.x; idx < BN * R4; idx += kGemmThreads) {
+        const int c = idx / R4, ml = zs * R + 4 * (idx % R4);
+        const uint32_t off = (uint32_t)((c * 128 + ml) * 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p = 0; p < ks; ++p) {
+          const float4 v = ptx::ld_shared_cluster_v4f(ptx::mapa_peer(red + off, (uint32_t)p));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int n = n0 + c;
+        if (n >= g.N) continue;
+        float v[4] = {acc.x, acc.y, acc.z, acc.w};
+        if (g.mode == kEpiAppend && use_a1) {
+          // rows (ml, ml+1) and (ml+2, ml+3) are rotary pairs k = ml/2, ml/2 + 1
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const int k = (ml + e) >> 1;
+            if (k < g.d_r / 2) {
+              double sn, cs;
+              sincos((double)s_pos[c] * g.theta[k], &sn, &cs);
+              const float co = (float)cs, si = (float)sn;
+              const float x0 = v[e], x1 = v[e + 1];
+              v[e] = x0 * co - x1 * si;
+              v[e + 1] = x0 * si + x1 * co;
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int m = m0 + ml + e;
+          if (m >= g.M_valid) continue;
+          if (g.mode == kEpiAppend) {
+            const long long row = s_row[c];
+            if (row >= 0) g.out[row * (long long)(g.d_c + g.d_r) + m] = __float2bfloat16_rn(v[e]);
+          } else {
+            g.out[(long long)n * g.out_ld + (long long)z * g.out_z + m] = __float2bfloat16_rn(v[e]);
+          }
+        }
+      }
+    } else if (threadIdx.x == 0) {
+      atomicOr(g.status, kStatusBounds);   // launched without the cluster shape it needs
+    }
+    ptx::cluster_sync_all();   // no CTA leaves while others still read its partial
+  }
+}
+
+constexpr size_t kSmemLimit = 232448;   // opt-in shared memory per block on sm_100
+
+template <int BN>
+constexpr int stage_bytes() { return kABytes + BN * kKChunk * 2; }
+
+template <int BN>
+constexpr size_t smem_tail() { return 256 + (size_t)BN * (8 + 4); }
+
+template <int BN>
+constexpr int max_stages() {
+  return (int)((kSmemLimit - 1024 - smem_tail<BN>()) / stage_bytes<BN>()) < kMaxStages
+             ? (int)((kSmemLimit - 1024 - smem_tail<BN>()) / stage_bytes<BN>())
+             : kMaxStages;
 }
 
 template <int BN, bool A_MN>
-cudaError_t launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
-                        const GemmParams &g, dim3 grid, cudaStream_t s) {
-  constexpr int kStage = kABytes + BN * kKChunk * 2;
-  const size_t smem = 1024 + (size_t)kGemmStages * kStage + 128 + BN * (8 + 4);
+cudaError_t launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, GemmParams g,
+                        int mtiles, int ntiles, int nz, cudaStream_t s) {
+  constexpr int kStage = stage_bytes<BN>();
+  const int per = (g.num_k_chunks + g.ksplit - 1) / g.ksplit;
+  g.stages = per < max_stages<BN>() ? (per > 0 ? per : 1) : max_stages<BN>();
+  size_t region = (size_t)g.stages * kStage;
+  if (g.ksplit > 1 && (size_t)128 * BN * 4 > region) region = (size_t)128 * BN * 4;
+  const size_t smem = 1024 + region + smem_tail<BN>();
+  if (smem > kSmemLimit) return cudaErrorNotSupported;
   auto kern = gemm_tc_kernel<BN, A_MN>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool configured[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev] = true;
   }
-  kern<<<grid, kGemmThreads, smem, s>>>(a0, a1, b, g);
-  return cudaGetLastError();
+  const dim3 grid(mtiles * g.ksplit, ntiles, nz);
+  if (g.ksplit == 1) {
+    kern<<<grid, kGemmThreads, smem, s>>>(a0, a1, b, g);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = g.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, g);
+}
+
+// K split: the smallest power of two (<= 8, the portable cluster size) that
+// gives at least one CTA per SM, while every slice keeps >= 2 K chunks.
+int pick_ksplit(long long ctas, int num_k_chunks) {
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int ks = 1;
+  while (ks < 8 && ctas * ks < sms && num_k_chunks >= 4 * ks) ks *= 2;
+  return ks;
 }
 
 template <bool A_MN>
 cudaError_t dispatch_bn(int N, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
-                        const GemmParams &g, int mtiles, int z, cudaStream_t s, int bn) {
-  const dim3 grid(mtiles, (N + bn - 1) / bn, z);
+                        GemmParams g, int mtiles, int z, cudaStream_t s, int bn) {
+  const int ntiles = (N + bn - 1) / bn;
+  if (g.ksplit == 0) g.ksplit = pick_ksplit((long long)mtiles * ntiles * z, g.num_k_chunks);
   switch (bn) {
-    case 16: return launch_gemm<16, A_MN>(a0, a1, b, g, grid, s);
-    case 32: return launch_gemm<32, A_MN>(a0, a1, b, g, grid, s);
-    case 64: return launch_gemm<64, A_MN>(a0, a1, b, g, grid, s);
-    case 128: return launch_gemm<128, A_MN>(a0, a1, b, g, grid, s);
-    default: return launch_gemm<256, A_MN>(a0, a1, b, g, grid, s);
+    case 16: return launch_gemm<16, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
+    case 32: return launch_gemm<32, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
+    case 64: return launch_gemm<64, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
+    case 128: return launch_gemm<128, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
+    default: return launch_gemm<256, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
   }
 }
 
