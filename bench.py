@@ -145,6 +145,31 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------
+# multi-rank plumbing (one process per GPU; ranks share nothing on the data path)
+# ----------------------------------------------------------------------------
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's synthetic batch: every rank decodes its own sequences."""
+    return 1000 + rank
+
+
+def reduce_max_over_ranks(values, world, device):
+    """Element-wise max over all ranks: the slowest rank sets each time."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_gbs(bytes_per_rank_step, world, ms_per_step):
+    """Whole-job throughput: the bytes all ranks moved in one step over the
+    (max over ranks) step time."""
+    return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
+
+
+# ----------------------------------------------------------------------------
 # CPU oracle timing (the baseline; also the --impl reference arm)
 # ----------------------------------------------------------------------------
 
@@ -250,7 +275,7 @@ def run_ours(args):
                        page_size=wl.page_size, rope_base=wl.rope_base, dtype=M.MLA_BF16)
     handle = M.mla_create(cfg)
     g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
+    g.manual_seed(rank_seed(rank))
     bf = torch.bfloat16
 
     def randn(*shape, std=1.0):
@@ -369,11 +394,9 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
     # ---- reduce over ranks: max time
-    times = torch.tensor([ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)
+    ms, attn_ms, e2e_ms = reduce_max_over_ranks([ms, attn_ms, e2e_ms], world, dev)
     if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
         dist.barrier()
-    ms, attn_ms, e2e_ms = times.tolist()
     M.mla_destroy(handle)
     if world > 1:
         dist.destroy_process_group()
@@ -384,7 +407,7 @@ def run_ours(args):
     step_bytes = algorithmic_bytes(wl, ctx_sum)
     attn_bytes = ctx_sum * D * 2
     hbm_peak, tf_peak, peak_kind = peaks()
-    value = step_bytes * world / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(step_bytes, world, ms)
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
     attn_flops, gemm_flops = algorithmic_flops(wl, ctx_sum)
     cpu = None
@@ -409,7 +432,7 @@ def run_ours(args):
                      "attn_us": attn_ms * 1e3,
                      "frac_of_8TBps": attn_gbs / 8000.0,
                      "tensor_tflops": attn_flops / (attn_ms * 1e-3) / 1e12},
-        "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": whole_job_gbs(step_bytes, world, e2e_ms), "unit": "GB/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 6 * args.steps,
         "per_call_us": per_call,

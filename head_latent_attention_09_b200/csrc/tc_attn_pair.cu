@@ -11,25 +11,30 @@
 // is 256 KB -- all of one SM's tensor memory -- so it is split across the two
 // SMs of a cluster, 64 heads each, and the MMAs are pair MMAs
 // (tcgen05.mma.cta_group::2, M = 128).  A pair MMA takes half of A's rows and
-// half of B's columns from each CTA's shared memory:
-//   S = Q K^T  (N = 128 tokens): CTA r holds Q rows 64r.. and tokens 64r.. of
-//               the tile; each CTA receives S for its 64 heads x 128 tokens,
-//               folded into 128 lanes x 64 columns (lanes 64.. = tokens 64..).
+// half of B's columns from each CTA's shared memory.  Per 256-token tile:
+//   S = Q K^T  (N = 256 tokens): CTA r holds Q rows 64r.. and tokens 128r..
+//               of the tile; each CTA receives S for its 64 heads x 256 tokens,
+//               folded into 128 lanes x 128 columns (lanes 64.. = tokens 128..).
 //   O += P V   (N = 256 latent columns per MMA, two MMAs): CTA r holds P for
 //               its heads and columns 128r.. of each 256-column group; each CTA
 //               accumulates O for its 64 heads x 512 columns in 256 columns.
 // The cache is therefore staged twice per CTA -- once token-split for S, once
-// column-split for O -- which doubles L2->SM traffic but reads HBM once and
-// needs no exchange of partial scores.
+// column-split for O -- which raises L2->SM traffic but reads HBM once and
+// needs no exchange of partial scores between the SMs.
 //
-// Staging: the cache tiles for S (K stages, 3 x 64 latent columns of 64
-// tokens, 24 KB) and for O (V stages, 64 tokens x 128 columns, 16 KB) flow
-// through separate rings with their own producer warps, so V stages waiting
-// for the softmax never hold back the next tile's K stages.
+// Why 256-token tiles: one thread issues the MMAs, and back-to-back
+// tcgen05.mma instructions cost ~55 cycles each however little work they
+// carry; a pair MMA with N = 256 carries 64 cycles of work, so only N = 256
+// keeps the tensor pipe busy.  A 256-token tile does not fit in shared memory
+// beside the resident query (72 KB), so it is streamed: S = Q K^T in nine
+// chunks of 64 columns (this CTA's 128 tokens, 16 KB each), O += P V in eight
+// sub-stages of 64 tokens x 128 columns (16 KB each), all through one ring of
+// 16 KB slots filled in the order the MMAs consume them.
 //
-// Warp roles per CTA (224 threads): warp 0 K/Q producer, warp 1 tensor-memory
-// allocation and (leader CTA only) MMA issue, warps 2-5 softmax, O rescale and
-// epilogue (one thread per tensor-memory lane), warp 6 V producer.
+// Warp roles per CTA (192 threads): warp 0 producer (TMA, and the hand copy
+// of a sequence's last partial block), warp 1 tensor-memory allocation and
+// (leader CTA only) MMA issue, warps 2-5 softmax, O rescale and epilogue (one
+// thread per tensor-memory lane).
 //
 // Every wait is bounded; a wait that runs out flags MLA_ERR_TIMEOUT and the
 // kernel winds down without further waits.
@@ -40,33 +45,30 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 224;
-constexpr int kKSlots = 3;              // K ring: 3 x 24 KB (one tile's nine 64-column chunks)
-constexpr int kKSlot = 3 * 8192;
-constexpr int kVSlots = 3;              // V ring: 3 x 16 KB
-constexpr int kVSlot = 2 * 8192;
+constexpr int kThreads = 192;
+constexpr int kTileTok = 256;           // tokens per pair tile (MMA N of S = Q K^T)
+constexpr int kHalfTok = 128;           // tokens of a tile each CTA stages for S
+constexpr int kSubTok = 64;             // tokens per O += P V sub-stage
+constexpr int kSlot = 16384;            // ring slot: a K chunk (128 rows x 128 B) or a V sub-stage
+constexpr int kSlots = 7;
 constexpr int kQBytes = 9 * 8192;       // 64 heads x 576 bf16, nine 64-column chunks
-constexpr int kPBytes = 16384;          // 64 heads x 128 tokens bf16 (two 64-token chunks)
-constexpr int kTileTok = 128;           // tokens per MMA tile
+constexpr int kPBytes = 4 * 8192;       // 64 heads x 256 tokens bf16, four 64-token chunks
 constexpr float kRescale = 8.0f;        // rescale O only when the running max grows by > 2^8
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKSlots * kKSlot;
-constexpr int kOffP = kOffV + kVSlots * kVSlot;
-constexpr int kOffRed = kOffP + 2 * kPBytes;            // float red_m[2][128], red_l[128]
+constexpr int kOffRing = kOffQ + kQBytes;
+constexpr int kOffP = kOffRing + kSlots * kSlot;
+constexpr int kOffRed = kOffP + kPBytes;                // float red_m[2][128], red_l[128]
 constexpr int kOffBar = kOffRed + 3 * 128 * 4;
 // barriers
-constexpr int kBarKFull = 0;                    // [3] leader: 1 arrival + tx bytes of both CTAs
-constexpr int kBarKEmpty = kBarKFull + kKSlots; // [3] both: pair commit
-constexpr int kBarVFull = kBarKEmpty + kKSlots; // [3] leader
-constexpr int kBarVEmpty = kBarVFull + kVSlots; // [3] both
-constexpr int kBarQFull = kBarVEmpty + kVSlots; // leader: 1 arrival + tx
+constexpr int kBarFull = 0;                     // [7] leader: 1 arrival + tx bytes of both CTAs
+constexpr int kBarEmpty = kBarFull + kSlots;    // [7] both: pair commit
+constexpr int kBarQFull = kBarEmpty + kSlots;   // leader: 1 arrival + tx
 constexpr int kBarQEmpty = kBarQFull + 1;       // both: pair commit
 constexpr int kBarSFull = kBarQEmpty + 1;       // [2] both: pair commit
-constexpr int kBarPFull = kBarSFull + 2;        // [2] leader: 8 warp arrivals
-constexpr int kBarPFree = kBarPFull + 2;        // [2] both: pair commit
-constexpr int kBarODone = kBarPFree + 2;        // [2] both: pair commit after P.V of even / odd tiles
+constexpr int kBarPFull = kBarSFull + 2;        // leader: 8 warp arrivals per tile
+constexpr int kBarPFree = kBarPFull + 1;        // both: pair commit after each tile's P.V
+constexpr int kBarODone = kBarPFree + 1;        // [2] both: pair commit after P.V of even / odd tiles
 constexpr int kBarOFree = kBarODone + 2;        // leader: 8 warp arrivals
 constexpr int kBarXchg = kBarOFree + 1;         // [2] local: 4 softmax-warp arrivals (row-max exchange)
 constexpr int kBarLsum = kBarXchg + 2;          // local: 4 softmax-warp arrivals (row-sum exchange)
@@ -75,9 +77,12 @@ constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kOffRing % 1024 == 0 && kOffP % 1024 == 0 && kSlot % 1024 == 0,
+              "128-byte-swizzled buffers must be 1024-byte aligned");
 
-constexpr uint32_t kTmemCols = 512;         // S: cols 0..127 (2 x 64), O: cols 128..383
-constexpr uint32_t kColO = 128;
+constexpr uint32_t kTmemCols = 512;         // S: 2 x 128 columns, O: columns 256..511
+constexpr uint32_t kColS = 128;
+constexpr uint32_t kColO = 256;
 
 constexpr uint32_t kIdescQK = idesc_bf16(128, kTileTok, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 256, false, true);
@@ -88,7 +93,7 @@ struct Piece {
   int tok_begin;       // first token of the piece in sequence b
   int tok_end;         // one past the last token attended by this piece
   int ctx;             // the sequence's context length (clamped to the cache)
-  int ntiles;          // 128-token MMA tiles
+  int ntiles;          // 256-token MMA tiles
 };
 
 struct Walk {
@@ -153,15 +158,13 @@ __device__ __forceinline__ long long kv_row(const AttnArgs &a, int b, int t) {
 
 struct Bars {
   uint64_t *b;
-  __device__ uint64_t *kfull(int s) { return b + kBarKFull + s; }
-  __device__ uint64_t *kempty(int s) { return b + kBarKEmpty + s; }
-  __device__ uint64_t *vfull(int s) { return b + kBarVFull + s; }
-  __device__ uint64_t *vempty(int s) { return b + kBarVEmpty + s; }
+  __device__ uint64_t *full(int s) { return b + kBarFull + s; }
+  __device__ uint64_t *empty(int s) { return b + kBarEmpty + s; }
   __device__ uint64_t *qfull() { return b + kBarQFull; }
   __device__ uint64_t *qempty() { return b + kBarQEmpty; }
   __device__ uint64_t *sfull(int i) { return b + kBarSFull + i; }
-  __device__ uint64_t *pfull(int i) { return b + kBarPFull + i; }
-  __device__ uint64_t *pfree(int i) { return b + kBarPFree + i; }
+  __device__ uint64_t *pfull() { return b + kBarPFull; }
+  __device__ uint64_t *pfree() { return b + kBarPFree; }
   __device__ uint64_t *odone(int i) { return b + kBarODone + i; }
   __device__ uint64_t *ofree() { return b + kBarOFree; }
   __device__ uint64_t *xchg(int i) { return b + kBarXchg + i; }
@@ -180,9 +183,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
   return ok;
 }
 
-// Row coordinate of a 64-token block starting at token t0 of the piece's
-// sequence, or an out-of-range row (TMA then fills zeros) when the block lies
-// past the piece.
+// Row coordinate of a block of cache rows starting at token t0 of the piece's
+// sequence, or an out-of-range row (TMA then fills zeros) when the block
+// starts past the piece.
 __device__ __forceinline__ int block_row(const AttnArgs &a, const Piece &p, int t0, long long kv_rows) {
   if (t0 >= p.tok_end) return (int)kv_rows;
   const long long r = kv_row(a, p.b, t0);
@@ -193,14 +196,20 @@ __device__ __forceinline__ int block_row(const AttnArgs &a, const Piece &p, int 
   return (int)r;
 }
 
+// O += P V sub-stages of a tile that starts at token t0 of the piece (the
+// sub-stages past the piece's end are skipped by the producer and the MMAs).
+__device__ __forceinline__ int tile_subs(const Piece &p, int t0) {
+  const int n = min(p.tok_end - t0, kTileTok);
+  return (n + kSubTok - 1) / kSubTok;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    attn_pair_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapKV,
-                     const AttnArgs a, const long long kv_rows) {
+    attn_pair_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                     const __grid_constant__ CUtensorMap mapV, const AttnArgs a, const long long kv_rows) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + kOffQ;
-  uint8_t *sK = sm + kOffK;
-  uint8_t *sV = sm + kOffV;
+  uint8_t *sRing = sm + kOffRing;
   uint8_t *sP = sm + kOffP;
   float *red_m = reinterpret_cast<float *>(sm + kOffRed);   // [2][128]
   float *red_l = red_m + 256;                                // [128]
@@ -214,23 +223,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int share = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kKSlots; ++s) {
-      ptx::mbar_init(bars.kfull(s), 1);
-      ptx::mbar_init(bars.kempty(s), 1);
-    }
-    for (int s = 0; s < kVSlots; ++s) {
-      ptx::mbar_init(bars.vfull(s), 1);
-      ptx::mbar_init(bars.vempty(s), 1);
+    for (int s = 0; s < kSlots; ++s) {
+      ptx::mbar_init(bars.full(s), 1);
+      ptx::mbar_init(bars.empty(s), 1);
     }
     ptx::mbar_init(bars.qfull(), 1);
     ptx::mbar_init(bars.qempty(), 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bars.sfull(i), 1);
-      ptx::mbar_init(bars.pfull(i), 8);
-      ptx::mbar_init(bars.pfree(i), 1);
       ptx::mbar_init(bars.odone(i), 1);
       ptx::mbar_init(bars.xchg(i), 4);
     }
+    ptx::mbar_init(bars.pfull(), 8);
+    ptx::mbar_init(bars.pfree(), 1);
     ptx::mbar_init(bars.ofree(), 8);
     ptx::mbar_init(bars.lsum(), 4);
     *abort_flag = 0;
@@ -246,178 +251,200 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------- Q and K-stage producer
-    // Lane 0 issues; the leader arms each stage with the bytes both CTAs'
-    // loads bring (the peer's loads count on the leader's barrier directly).
+    // --------------------------------------------------------------- producer
+    // Fills the ring in the order the MMAs consume it: the nine K chunks of
+    // tile i, then the V sub-stages of tile i-1 (tiles counted across the
+    // share's pieces).  Lane 0 issues TMA; the leader arms each slot with the
+    // bytes both CTAs' loads bring (the peer's loads count on the leader's
+    // barrier directly).
+    const uint32_t lq = ptx::leader_addr(bars.qfull());
+    const uint32_t lf0 = ptx::leader_addr(bars.full(0));
     if (lane == 0) {
-      const uint32_t lq = ptx::leader_addr(bars.qfull());
-      const uint32_t lk0 = ptx::leader_addr(bars.kfull(0));
       ptx::tma_prefetch_desc(&mapQ);
-      ptx::tma_prefetch_desc(&mapKV);
-      Walk w;
-      walk_init(w, a, share);
-      Piece pc;
-      int sc = 0, npc = 0;
-      bool ok = true;
-      while (ok && walk_next(w, a, share, pc)) {
-        if (npc > 0 && !ptx::mbar_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag)) break;
-        if (leader) ptx::mbar_arrive_expect_tx(bars.qfull(), 2 * kQBytes);
-        for (int c = 0; c < 9; ++c)
-          ptx::tma_load_2d_pair(sQ + c * 8192, &mapQ, lq, 64 * c, pc.b * 128 + 64 * (int)rank);
-        for (int k = 0; k < pc.ntiles && ok; ++k) {
-          const int y = block_row(a, pc, pc.tok_begin + kTileTok * k + 64 * (int)rank, kv_rows);
-          for (int kc = 0; kc < 3; ++kc) {
-            const int s = sc % kKSlots;
-            if (sc >= kKSlots && !ptx::mbar_wait(bars.kempty(s), ((sc / kKSlots) - 1) & 1, a.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            if (leader) ptx::mbar_arrive_expect_tx(bars.kfull(s), 2 * kKSlot);
-            uint8_t *dst = sK + s * kKSlot;
-#pragma unroll
-            for (int cc = 0; cc < 3; ++cc)
-              ptx::tma_load_2d_pair(dst + cc * 8192, &mapKV, lk0 + 8 * s, 64 * (3 * kc + cc), y);
-            ++sc;
-          }
-        }
-        ++npc;
-      }
+      ptx::tma_prefetch_desc(&mapK);
+      ptx::tma_prefetch_desc(&mapV);
     }
-  } else if (warp == 6) {
-    // -------------------------------------------------------- V-stage producer
-    // V stage (g, h) of a tile: tokens 64h.. of the tile, latent columns
-    // 256g + 128 * rank .. +128 (this CTA's half of the 256-column group).
-    const uint32_t lv0 = ptx::leader_addr(bars.vfull(0));
     Walk w;
     walk_init(w, a, share);
-    Piece pc;
-    int sc = 0;
+    Piece pc, vpc;            // vpc/vt0: the tile whose V sub-stages are pending
+    int vt0 = 0;
+    bool vpending = false;
+    int sc = 0, npc = 0;
     bool ok = true;
-    if (lane == 0) ptx::tma_prefetch_desc(&mapKV);
-    while (ok && walk_next(w, a, share, pc)) {
-      for (int k = 0; k < pc.ntiles && ok; ++k) {
-        for (int g = 0; g < 2 && ok; ++g) {
-          for (int hh = 0; hh < 2; ++hh) {
-            const int s = sc % kVSlots;
-            const int tok0 = pc.tok_begin + kTileTok * k + 64 * hh;
-            const bool manual = tok0 < pc.tok_end && tok0 + 64 > pc.ctx;
-            bool got = true;
-            if (lane == 0 && sc >= kVSlots)
-              got = ptx::mbar_wait(bars.vempty(s), ((sc / kVSlots) - 1) & 1, a.status, abort_flag);
-            if (!(__shfl_sync(0xffffffffu, got ? 1 : 0, 0))) {
-              ok = false;
-              break;
-            }
-            __syncwarp();
-            uint8_t *dst = sV + s * kVSlot;
-            if (manual) {
-              // The block runs past the sequence: the leader copies the valid
-              // rows of both CTAs' column halves by hand and zeroes the rest,
-              // so that no unwritten cache row (possibly NaN) reaches P.V.
-              // 128-byte rows, 16-byte units swizzled by row (the layout a
-              // 128-byte-swizzled TMA load produces).  The peer skips it.
-              if (leader) {
-                const uint32_t own = ptx::smem_u32(dst), peer = ptx::mapa_peer(own, 1);
-                for (int u = lane; u < 2 * 2 * 64 * 8; u += 32) {
-                  const int cta = u >> 10, half = (u >> 9) & 1, row = (u >> 3) & 63, c = u & 7;
-                  const int t = tok0 + row;
-                  uint4 v = make_uint4(0, 0, 0, 0);
-                  if (t < pc.ctx) {
-                    const long long r = kv_row(a, pc.b, t);
-                    if (r >= 0)
-                      v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.cache) +
-                                                           r * 576 + 256 * g + 128 * cta + 64 * half + 8 * c);
-                    else
-                      atomicOr(a.status, kStatusBounds);
-                  }
-                  const uint32_t off = half * 8192 + row * 128 + ((c ^ (row & 7)) << 4);
-                  ptx::st_shared_cluster_v4(cta ? peer + off : own + off, v);
+    // Acquires the next ring slot (warp-uniform); returns its index or -1.
+    auto acquire = [&]() -> int {
+      const int s = sc % kSlots;
+      bool got = true;
+      if (lane == 0 && sc >= kSlots)
+        got = ptx::mbar_wait(bars.empty(s), ((sc / kSlots) - 1) & 1, a.status, abort_flag);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      __syncwarp();
+      return got ? s : -1;
+    };
+    // V sub-stages of the tile at token t0 of piece p: tokens t0 + 64t..,
+    // latent columns 256g + 128 * rank .. +128.
+    auto issue_v = [&](const Piece &p, int t0) -> bool {
+      const int nsub = tile_subs(p, t0);
+      for (int t = 0; t < nsub; ++t) {
+        for (int g = 0; g < 2; ++g) {
+          const int s = acquire();
+          if (s < 0) return false;
+          uint8_t *dst = sRing + s * kSlot;
+          const int tok0 = t0 + kSubTok * t;
+          if (tok0 + kSubTok > p.ctx) {
+            // The block runs past the sequence: the leader copies the valid
+            // rows of both CTAs' column halves by hand and zeroes the rest,
+            // so that no unwritten cache row (possibly NaN) reaches P.V.
+            // 128-byte rows, 16-byte units swizzled by row (the layout a
+            // 128-byte-swizzled TMA load produces).  The peer skips it.
+            if (leader) {
+              const uint32_t own = ptx::smem_u32(dst), peer = ptx::mapa_peer(own, 1);
+              for (int u = lane; u < 2 * 2 * 64 * 8; u += 32) {
+                const int cta = u >> 10, half = (u >> 9) & 1, row = (u >> 3) & 63, c = u & 7;
+                const int tk = tok0 + row;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (tk < p.ctx) {
+                  const long long r = kv_row(a, p.b, tk);
+                  if (r >= 0)
+                    v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.cache) +
+                                                         r * 576 + 256 * g + 128 * cta + 64 * half + 8 * c);
+                  else
+                    atomicOr(a.status, kStatusBounds);
                 }
-                ptx::fence_acq_rel_cluster();
-                ptx::fence_proxy_async_cluster();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bars.vfull(s));
+                const uint32_t off = half * 8192 + row * 128 + ((c ^ (row & 7)) << 4);
+                ptx::st_shared_cluster_v4(cta ? peer + off : own + off, v);
               }
-            } else if (lane == 0) {
-              const int y = block_row(a, pc, tok0, kv_rows);
-              if (leader) ptx::mbar_arrive_expect_tx(bars.vfull(s), 2 * kVSlot);
-              const int feat0 = 256 * g + 128 * (int)rank;
-              ptx::tma_load_2d_pair(dst, &mapKV, lv0 + 8 * s, feat0, y);
-              ptx::tma_load_2d_pair(dst + 8192, &mapKV, lv0 + 8 * s, feat0 + 64, y);
+              ptx::fence_acq_rel_cluster();
+              ptx::fence_proxy_async_cluster();
+              __syncwarp();
+              if (lane == 0) ptx::mbar_arrive(bars.full(s));
             }
-            ++sc;
+          } else if (lane == 0) {
+            const int y = block_row(a, p, tok0, kv_rows);
+            if (leader) ptx::mbar_arrive_expect_tx(bars.full(s), 2 * kSlot);
+            const int feat0 = 256 * g + 128 * (int)rank;
+            ptx::tma_load_2d_pair(dst, &mapV, lf0 + 8 * s, feat0, y);
+            ptx::tma_load_2d_pair(dst + 8192, &mapV, lf0 + 8 * s, feat0 + 64, y);
           }
+          ++sc;
         }
       }
+      return true;
+    };
+    while (ok && walk_next(w, a, share, pc)) {
+      bool qok = true;
+      if (lane == 0) {
+        if (npc > 0) qok = ptx::mbar_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag);
+        if (qok) {
+          if (leader) ptx::mbar_arrive_expect_tx(bars.qfull(), 2 * kQBytes);
+          for (int c = 0; c < 9; ++c)
+            ptx::tma_load_2d_pair(sQ + c * 8192, &mapQ, lq, 64 * c, pc.b * 128 + 64 * (int)rank);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, qok ? 1 : 0, 0)) break;
+      for (int k = 0; k < pc.ntiles && ok; ++k) {
+        // K chunks of this tile: this CTA's 128 tokens x 64 columns each.
+        const int t0 = pc.tok_begin + kTileTok * k;
+        const int tr = t0 + kHalfTok * (int)rank;
+        int y0 = 0, y1 = 0;
+        if (lane == 0) {
+          y0 = block_row(a, pc, tr, kv_rows);
+          if (a.page_size) y1 = block_row(a, pc, tr + kSubTok, kv_rows);
+        }
+        for (int c = 0; c < 9; ++c) {
+          const int s = acquire();
+          if (s < 0) { ok = false; break; }
+          if (lane == 0) {
+            uint8_t *dst = sRing + s * kSlot;
+            if (leader) ptx::mbar_arrive_expect_tx(bars.full(s), 2 * kSlot);
+            if (a.page_size == 0) {
+              ptx::tma_load_2d_pair(dst, &mapK, lf0 + 8 * s, 64 * c, y0);
+            } else {
+              // 64-token pages: two 64-row boxes.
+              ptx::tma_load_2d_pair(dst, &mapV, lf0 + 8 * s, 64 * c, y0);
+              ptx::tma_load_2d_pair(dst + 8192, &mapV, lf0 + 8 * s, 64 * c, y1);
+            }
+          }
+          ++sc;
+        }
+        if (!ok) break;
+        if (vpending && !issue_v(vpc, vt0)) { ok = false; break; }
+        vpc = pc;
+        vt0 = t0;
+        vpending = true;
+      }
+      ++npc;
     }
+    if (ok && vpending) issue_v(vpc, vt0);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (leader && lane == 0) {
       Walk w;
       walk_init(w, a, share);
       Piece pc;
-      int ksc = 0, vsc = 0, npc = 0, i = 0;
+      int sc = 0, npc = 0, i = 0;
       bool ok = true;
-      struct PrevTile { int i, first, npc; } prev{0, 0, 0};
+      struct PrevTile { int i, first, npc, nsub; } prev{0, 0, 0, 0};
       bool have_prev = false;
       // Descriptors are built once; the start address (bits 0-13, 16-byte
       // units) is advanced by adding offsets.
       const uint64_t dQ = ptx::sdesc(ptx::smem_u32(sQ), 16, 1024, 2);
-      const uint64_t dK = ptx::sdesc(ptx::smem_u32(sK), 16, 1024, 2);
+      const uint64_t dK = ptx::sdesc(ptx::smem_u32(sRing), 16, 1024, 2);
+      const uint64_t dV = ptx::sdesc(ptx::smem_u32(sRing), 8192, 1024, 2);
       const uint64_t dP = ptx::sdesc(ptx::smem_u32(sP), 16, 1024, 2);
-      const uint64_t dV = ptx::sdesc(ptx::smem_u32(sV), 8192, 1024, 2);
+      auto slot_wait = [&]() -> int {
+        const int s = sc % kSlots;
+        if (!ptx::mbar_wait(bars.full(s), (sc / kSlots) & 1, a.status, abort_flag)) return -1;
+        ptx::tc_fence_after();
+        return s;
+      };
       auto pv = [&](const PrevTile &t) -> bool {
         if (t.first && t.npc > 0 && !ptx::mbar_wait(bars.ofree(), (t.npc - 1) & 1, a.status, abort_flag))
           return false;
-        if (!ptx::mbar_wait(bars.pfull(t.i & 1), (t.i >> 1) & 1, a.status, abort_flag)) return false;
+        if (!ptx::mbar_wait(bars.pfull(), t.i & 1, a.status, abort_flag)) return false;
         ptx::tc_fence_after();
-        const uint32_t pofs = (t.i & 1) * (kPBytes >> 4);
-        for (int g = 0; g < 2; ++g) {
-          for (int hh = 0; hh < 2; ++hh) {
-            const int s = vsc % kVSlots;
-            if (!ptx::mbar_wait(bars.vfull(s), (vsc / kVSlots) & 1, a.status, abort_flag)) return false;
-            ptx::tc_fence_after();
+        for (int tt = 0; tt < t.nsub; ++tt) {
+          for (int g = 0; g < 2; ++g) {
+            const int s = slot_wait();
+            if (s < 0) return false;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              // A = P rows (heads) x tokens 64hh + 16j.. (K-major); B = V rows
-              // (tokens 16j..) x 128 columns in two 64-column chunks 8 KB apart.
-              const uint64_t ad = dP + pofs + ((hh * 8192 + j * 32) >> 4);
-              const uint64_t bd = dV + ((s * kVSlot + j * 2048) >> 4);
+              // A = P rows (heads) x tokens 64tt + 16j.. (K-major); B = V rows
+              // (tokens 16j.. of the sub-stage) x 128 columns in two 64-column
+              // chunks 8 KB apart.
+              const uint64_t ad = dP + ((tt * 8192 + j * 32) >> 4);
+              const uint64_t bd = dV + ((s * kSlot + j * 2048) >> 4);
               ptx::mma_bf16_ss_pair(tmem + kColO + 128 * g, ad, bd, kIdescPV,
-                                    (t.first && hh == 0 && j == 0) ? 0u : 1u);
+                                    (t.first && tt == 0 && j == 0) ? 0u : 1u);
             }
-            ptx::mma_commit_pair_both(bars.vempty(s));
-            ++vsc;
+            ptx::mma_commit_pair_both(bars.empty(s));
+            ++sc;
           }
         }
-        ptx::mma_commit_pair_both(bars.pfree(t.i & 1));
+        ptx::mma_commit_pair_both(bars.pfree());
         ptx::mma_commit_pair_both(bars.odone(t.i & 1));
         return true;
       };
       while (ok && walk_next(w, a, share, pc)) {
         if (!ptx::mbar_wait(bars.qfull(), npc & 1, a.status, abort_flag)) { ok = false; break; }
         for (int k = 0; k < pc.ntiles && ok; ++k) {
-          for (int kc = 0; kc < 3; ++kc) {
-            const int s = ksc % kKSlots;
-            if (!ptx::mbar_wait(bars.kfull(s), (ksc / kKSlots) & 1, a.status, abort_flag)) { ok = false; break; }
-            ptx::tc_fence_after();
+          for (int c = 0; c < 9; ++c) {
+            const int s = slot_wait();
+            if (s < 0) { ok = false; break; }
 #pragma unroll
-            for (int cc = 0; cc < 3; ++cc) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint64_t ad = dQ + (((3 * kc + cc) * 8192 + 32 * j) >> 4);
-                const uint64_t bd = dK + ((s * kKSlot + cc * 8192 + 32 * j) >> 4);
-                ptx::mma_bf16_ss_pair(tmem + (i & 1) * 64, ad, bd, kIdescQK, (kc | cc | j) != 0 ? 1u : 0u);
-              }
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t ad = dQ + ((c * 8192 + 32 * j) >> 4);
+              const uint64_t bd = dK + ((s * kSlot + 32 * j) >> 4);
+              ptx::mma_bf16_ss_pair(tmem + (i & 1) * kColS, ad, bd, kIdescQK, (c | j) != 0 ? 1u : 0u);
             }
-            ptx::mma_commit_pair_both(bars.kempty(s));
-            ++ksc;
+            ptx::mma_commit_pair_both(bars.empty(s));
+            ++sc;
           }
           if (!ok) break;
           ptx::mma_commit_pair_both(bars.sfull(i & 1));
           if (k == pc.ntiles - 1) ptx::mma_commit_pair_both(bars.qempty());
           if (have_prev && !pv(prev)) { ok = false; break; }
-          prev = {i, k == 0 ? 1 : 0, npc};
+          prev = {i, k == 0 ? 1 : 0, npc, tile_subs(pc, pc.tok_begin + kTileTok * k)};
           have_prev = true;
           ++i;
         }
@@ -431,10 +458,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int l = q * 32 + lane;          // tensor-memory lane of this thread
     const int h = l & 63, th = l >> 6;    // local head, token half
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
-    const uint32_t leader_pfull0 = ptx::leader_addr(bars.pfull(0));
+    const uint32_t leader_pfull = ptx::leader_addr(bars.pfull());
     const uint32_t leader_ofree = ptx::leader_addr(bars.ofree());
     float *opart = reinterpret_cast<float *>(a.ws + a.L.opart_off);
     float *lse_out = reinterpret_cast<float *>(a.ws + a.L.lse_off);
+    uint8_t *prow = sP + h * 128;         // row h of each 64-token P chunk
     Walk w;
     walk_init(w, a, share);
     Piece pc;
@@ -443,24 +471,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (ok && walk_next(w, a, share, pc)) {
       float m_run = -CUDART_INF_F, l_part = 0.f;
       for (int k = 0; k < pc.ntiles; ++k, ++i) {
-        const int base = pc.tok_begin + kTileTok * k + 64 * th;
-        const int nvalid = min(max(pc.tok_end - base, 0), 64);
+        const int base = pc.tok_begin + kTileTok * k + kHalfTok * th;
+        const int nvalid = min(max(pc.tok_end - base, 0), kHalfTok);
+        const uint32_t scol = lane_addr + (i & 1) * kColS;
         if (!warp_wait(bars.sfull(i & 1), (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
-        float s[64];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        // pass 1: this row's maximum over its 128 tokens (log2 units)
+        float mloc = -CUDART_INF_F;
+#pragma unroll 2
+        for (int c = 0; c < kHalfTok / 16; ++c) {
           uint32_t r[16];
-          ptx::tmem_ld16(lane_addr + (i & 1) * 64 + 16 * c, r);
+          ptx::tmem_ld16(scol + 16 * c, r);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(r[j]);
-        }
-        float mloc = -CUDART_INF_F;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          s[j] = j < nvalid ? s[j] * a.scale_log2 : -CUDART_INF_F;
-          mloc = fmaxf(mloc, s[j]);
+          for (int j = 0; j < 16; ++j)
+            if (16 * c + j < nvalid) mloc = fmaxf(mloc, __uint_as_float(r[j]) * a.scale_log2);
         }
         red_m[(i & 1) * 128 + l] = mloc;
         __syncwarp();
@@ -475,22 +500,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           l_part *= alpha;
           rescale = k > 0;
         }
-        uint32_t pk[32];
+        // P of the previous tile must have been read by its P.V.
+        if (i >= 1 && !warp_wait(bars.pfree(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+        // pass 2: probabilities, their sum, and P (bf16) in shared memory:
+        // tokens 128 th + 16c.. are 16-byte units 2(c&3), 2(c&3)+1 of row h
+        // of P chunk 2 th + (c >> 2) (128-byte swizzle by row).
         float sum = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < kHalfTok / 16; ++c) {
+          uint32_t r[16];
+          ptx::tmem_ld16(scol + 16 * c, r);
+          ptx::tmem_ld_wait();
+          uint32_t pk[8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = exp2f(s[2 * j] - m_run), p1 = exp2f(s[2 * j + 1] - m_run);
-          sum += p0 + p1;
-          __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
-          pk[j] = *reinterpret_cast<uint32_t *>(&v);
+          for (int j = 0; j < 8; ++j) {
+            const int t = 16 * c + 2 * j;
+            const float p0 = t < nvalid ? exp2f(__uint_as_float(r[2 * j]) * a.scale_log2 - m_run) : 0.f;
+            const float p1 = t + 1 < nvalid ? exp2f(__uint_as_float(r[2 * j + 1]) * a.scale_log2 - m_run) : 0.f;
+            sum += p0 + p1;
+            __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
+            pk[j] = *reinterpret_cast<uint32_t *>(&v);
+          }
+          uint8_t *chunk = prow + (2 * th + (c >> 2)) * 8192;
+          const int u0 = 2 * (c & 3);
+          *reinterpret_cast<uint4 *>(chunk + ((u0 ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4 *>(chunk + (((u0 + 1) ^ (h & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
         l_part += sum;
-        if (i >= 2 && !warp_wait(bars.pfree(i & 1), ((i >> 1) - 1) & 1, a.status, abort_flag)) { ok = false; break; }
-        uint8_t *prow = sP + (i & 1) * kPBytes + th * 8192 + h * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         // The rescale (tensor-memory loads and stores, .sync.aligned) is done by
         // the whole warp when any of its rows needs it; other rows use alpha = 1.
         if (__any_sync(0xffffffffu, rescale)) {
@@ -515,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_remote_addr(leader_pfull0 + 8 * (i & 1));
+        if (lane == 0) ptx::mbar_arrive_remote_addr(leader_pfull);
       }
       if (!ok) break;
       // ---- epilogue of the piece: O / l and the log-sum-exp
@@ -569,13 +605,16 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
   if (a.page_size != 0 && a.page_size != kTile) return cudaErrorNotSupported;
   const long long rows = a.page_size ? a.cache_len * kTile : (long long)a.B * a.cache_len;
   if (rows <= 0 || rows >= (1ll << 31) - 256) return cudaErrorNotSupported;
-  CUtensorMap mq, mkv;
+  CUtensorMap mq, mk, mv;
   const uint64_t dq[2] = {576, (uint64_t)a.B * 128};
   const uint64_t dkv[2] = {576, (uint64_t)rows};
   const uint64_t st[1] = {576 * 2};
-  const uint32_t box[2] = {64, 64};
-  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mkv, a.cache, 2, dkv, st, box, CU_TENSOR_MAP_SWIZZLE_128B))
+  const uint32_t boxq[2] = {64, 64};
+  const uint32_t boxk[2] = {64, kHalfTok};
+  const uint32_t boxv[2] = {64, kSubTok};
+  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, boxq, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mk, a.cache, 2, dkv, st, boxk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mv, a.cache, 2, dkv, st, boxv, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
   static bool configured = false;
   if (!configured) {
@@ -583,7 +622,7 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_pair_kernel<<<2 * P, kThreads, kSmemAlloc, s>>>(mq, mkv, a, rows);
+  attn_pair_kernel<<<2 * P, kThreads, kSmemAlloc, s>>>(mq, mk, mv, a, rows);
   return cudaGetLastError();
 }
 
