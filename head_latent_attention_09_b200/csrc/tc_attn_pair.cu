@@ -271,14 +271,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool vpending = false;
     int sc = 0, npc = 0;
     bool ok = true;
+    int ws_ = 0;               // ring slot of the next job
+    int wround = 0;            // how many times the ring has been filled before
     // Acquires the next ring slot (warp-uniform); returns its index or -1.
+    // In round r >= 1 a slot is free once the MMAs of round r-1 released it.
     auto acquire = [&]() -> int {
-      const int s = sc % kSlots;
+      const int s = ws_;
       bool got = true;
-      if (lane == 0 && sc >= kSlots)
-        got = ptx::mbar_wait(bars.empty(s), ((sc / kSlots) - 1) & 1, a.status, abort_flag);
+      if (lane == 0 && wround > 0) got = ptx::mbar_wait(bars.empty(s), (wround - 1) & 1, a.status, abort_flag);
       got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
       __syncwarp();
+      if (++ws_ == kSlots) {
+        ws_ = 0;
+        ++wround;
+      }
       return got ? s : -1;
     };
     // V sub-stages of the tile at token t0 of piece p: tokens t0 + 64t..,
@@ -382,20 +388,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Walk w;
       walk_init(w, a, share);
       Piece pc;
-      int sc = 0, npc = 0, i = 0;
+      int npc = 0, i = 0;
+      int rs = 0;                 // ring slot of the next job
+      uint32_t rph = 0;           // its full-barrier phase parity
       bool ok = true;
       struct PrevTile { int i, first, npc, nsub; } prev{0, 0, 0, 0};
       bool have_prev = false;
       // Descriptors are built once; the start address (bits 0-13, 16-byte
-      // units) is advanced by adding offsets.
+      // units) is advanced by adding offsets.  The issue loop is kept lean:
+      // one thread issues every MMA, and its own instruction latency, not the
+      // tensor pipe, bounds the rate when the loop does more than it must.
       const uint64_t dQ = ptx::sdesc(ptx::smem_u32(sQ), 16, 1024, 2);
       const uint64_t dK = ptx::sdesc(ptx::smem_u32(sRing), 16, 1024, 2);
       const uint64_t dV = ptx::sdesc(ptx::smem_u32(sRing), 8192, 1024, 2);
       const uint64_t dP = ptx::sdesc(ptx::smem_u32(sP), 16, 1024, 2);
+      // Waits for the next ring job; returns its slot or -1.
       auto slot_wait = [&]() -> int {
-        const int s = sc % kSlots;
-        if (!ptx::mbar_wait(bars.full(s), (sc / kSlots) & 1, a.status, abort_flag)) return -1;
+        const int s = rs;
+        if (!ptx::mbar_wait(bars.full(s), rph, a.status, abort_flag)) return -1;
         ptx::tc_fence_after();
+        if (++rs == kSlots) {
+          rs = 0;
+          rph ^= 1u;
+        }
         return s;
       };
       auto pv = [&](const PrevTile &t) -> bool {
@@ -404,21 +419,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bars.pfull(), t.i & 1, a.status, abort_flag)) return false;
         ptx::tc_fence_after();
         for (int tt = 0; tt < t.nsub; ++tt) {
+          const uint64_t ad = dP + (uint64_t)((tt * 8192) >> 4);
+          const uint32_t acc0 = (t.first && tt == 0) ? 0u : 1u;
+#pragma unroll
           for (int g = 0; g < 2; ++g) {
             const int s = slot_wait();
             if (s < 0) return false;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              // A = P rows (heads) x tokens 64tt + 16j.. (K-major); B = V rows
-              // (tokens 16j.. of the sub-stage) x 128 columns in two 64-column
-              // chunks 8 KB apart.
-              const uint64_t ad = dP + ((tt * 8192 + j * 32) >> 4);
-              const uint64_t bd = dV + ((s * kSlot + j * 2048) >> 4);
-              ptx::mma_bf16_ss_pair(tmem + kColO + 128 * g, ad, bd, kIdescPV,
-                                    (t.first && tt == 0 && j == 0) ? 0u : 1u);
-            }
+            // A = P rows (heads) x tokens 64tt + 16j.. (K-major); B = V rows
+            // (tokens 16j.. of the sub-stage) x 128 columns in two 64-column
+            // chunks 8 KB apart.
+            const uint64_t bd = dV + (uint64_t)((s * kSlot) >> 4);
+            const uint32_t d = tmem + kColO + 128 * g;
+            ptx::mma_bf16_ss_pair(d, ad, bd, kIdescPV, acc0);
+            ptx::mma_bf16_ss_pair(d, ad + 2, bd + 128, kIdescPV, 1u);
+            ptx::mma_bf16_ss_pair(d, ad + 4, bd + 256, kIdescPV, 1u);
+            ptx::mma_bf16_ss_pair(d, ad + 6, bd + 384, kIdescPV, 1u);
             ptx::mma_commit_pair_both(bars.empty(s));
-            ++sc;
           }
         }
         ptx::mma_commit_pair_both(bars.pfree());
@@ -428,17 +444,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (ok && walk_next(w, a, share, pc)) {
         if (!ptx::mbar_wait(bars.qfull(), npc & 1, a.status, abort_flag)) { ok = false; break; }
         for (int k = 0; k < pc.ntiles && ok; ++k) {
+          const uint32_t dS = tmem + (i & 1) * kColS;
+#pragma unroll
           for (int c = 0; c < 9; ++c) {
             const int s = slot_wait();
             if (s < 0) { ok = false; break; }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint64_t ad = dQ + ((c * 8192 + 32 * j) >> 4);
-              const uint64_t bd = dK + ((s * kSlot + 32 * j) >> 4);
-              ptx::mma_bf16_ss_pair(tmem + (i & 1) * kColS, ad, bd, kIdescQK, (c | j) != 0 ? 1u : 0u);
-            }
+            // A = Q chunk c (64-column chunks 8 KB apart), B = this slot's
+            // 128 tokens x 64 columns; k steps of 16 columns are 32 B apart.
+            const uint64_t ad = dQ + (uint64_t)((c * 8192) >> 4);
+            const uint64_t bd = dK + (uint64_t)((s * kSlot) >> 4);
+            ptx::mma_bf16_ss_pair(dS, ad, bd, kIdescQK, c != 0 ? 1u : 0u);
+            ptx::mma_bf16_ss_pair(dS, ad + 2, bd + 2, kIdescQK, 1u);
+            ptx::mma_bf16_ss_pair(dS, ad + 4, bd + 4, kIdescQK, 1u);
+            ptx::mma_bf16_ss_pair(dS, ad + 6, bd + 6, kIdescQK, 1u);
             ptx::mma_commit_pair_both(bars.empty(s));
-            ++sc;
           }
           if (!ok) break;
           ptx::mma_commit_pair_both(bars.sfull(i & 1));
@@ -476,17 +495,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t scol = lane_addr + (i & 1) * kColS;
         if (!warp_wait(bars.sfull(i & 1), (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
-        // pass 1: this row's maximum over its 128 tokens (log2 units)
-        float mloc = -CUDART_INF_F;
-#pragma unroll 2
-        for (int c = 0; c < kHalfTok / 16; ++c) {
-          uint32_t r[16];
-          ptx::tmem_ld16(scol + 16 * c, r);
-          ptx::tmem_ld_wait();
+        // This row's 128 scores, in log2 units, invalid tokens at -inf.
+        float v[kHalfTok];
+        ptx::tmem_ld64_sync(scol, reinterpret_cast<uint32_t *>(v));
+        ptx::tmem_ld64_sync(scol + 64, reinterpret_cast<uint32_t *>(v) + 64);
+        float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (16 * c + j < nvalid) mloc = fmaxf(mloc, __uint_as_float(r[j]) * a.scale_log2);
+        for (int j = 0; j < kHalfTok; ++j) {
+          v[j] = j < nvalid ? v[j] * a.scale_log2 : -CUDART_INF_F;
+          mx[j & 3] = fmaxf(mx[j & 3], v[j]);
         }
+        const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         red_m[(i & 1) * 128 + l] = mloc;
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bars.xchg(i & 1));
@@ -500,31 +519,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           l_part *= alpha;
           rescale = k > 0;
         }
+        // Probabilities (bf16 pairs) and their sum, before waiting for the
+        // previous tile's P.V, so that only the store below waits for it.
+        uint32_t pk[kHalfTok / 2];
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < kHalfTok / 2; ++j) {
+          const float p0 = ptx::exp2_approx(v[2 * j] - m_run), p1 = ptx::exp2_approx(v[2 * j + 1] - m_run);
+          ps[j & 7] += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[j] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         // P of the previous tile must have been read by its P.V.
         if (i >= 1 && !warp_wait(bars.pfree(), (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
-        // pass 2: probabilities, their sum, and P (bf16) in shared memory:
-        // tokens 128 th + 16c.. are 16-byte units 2(c&3), 2(c&3)+1 of row h
-        // of P chunk 2 th + (c >> 2) (128-byte swizzle by row).
-        float sum = 0.f;
-#pragma unroll 2
-        for (int c = 0; c < kHalfTok / 16; ++c) {
-          uint32_t r[16];
-          ptx::tmem_ld16(scol + 16 * c, r);
-          ptx::tmem_ld_wait();
-          uint32_t pk[8];
+        // Tokens 128 th + 16c.. are 16-byte units 2(c&3), 2(c&3)+1 of row h of
+        // P chunk 2 th + (c >> 2) (128-byte swizzle by row).
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int t = 16 * c + 2 * j;
-            const float p0 = t < nvalid ? exp2f(__uint_as_float(r[2 * j]) * a.scale_log2 - m_run) : 0.f;
-            const float p1 = t + 1 < nvalid ? exp2f(__uint_as_float(r[2 * j + 1]) * a.scale_log2 - m_run) : 0.f;
-            sum += p0 + p1;
-            __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
-            pk[j] = *reinterpret_cast<uint32_t *>(&v);
-          }
+        for (int c = 0; c < kHalfTok / 16; ++c) {
           uint8_t *chunk = prow + (2 * th + (c >> 2)) * 8192;
           const int u0 = 2 * (c & 3);
-          *reinterpret_cast<uint4 *>(chunk + ((u0 ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4 *>(chunk + (((u0 + 1) ^ (h & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          *reinterpret_cast<uint4 *>(chunk + ((u0 ^ (h & 7)) << 4)) =
+              make_uint4(pk[8 * c], pk[8 * c + 1], pk[8 * c + 2], pk[8 * c + 3]);
+          *reinterpret_cast<uint4 *>(chunk + (((u0 + 1) ^ (h & 7)) << 4)) =
+              make_uint4(pk[8 * c + 4], pk[8 * c + 5], pk[8 * c + 6], pk[8 * c + 7]);
         }
         l_part += sum;
         // The rescale (tensor-memory loads and stores, .sync.aligned) is done by
