@@ -256,7 +256,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // tile i, then the V sub-stages of tile i-1 (tiles counted across the
     // share's pieces).  Lane 0 issues TMA; the leader arms each slot with the
     // bytes both CTAs' loads bring (the peer's loads count on the leader's
-    // barrier directly).
+    // barrier directly).  One producer takes every job in order, so a slot's
+    // empty barrier is never more than one phase behind the phase waited for
+    // (a parity wait cannot tell one phase behind from three); two producers
+    // splitting the jobs would each need to wait for the other to pass the
+    // slot's previous job first, and measured no faster.
     const uint32_t lq = ptx::leader_addr(bars.qfull());
     const uint32_t lf0 = ptx::leader_addr(bars.full(0));
     if (lane == 0) {
