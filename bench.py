@@ -55,6 +55,25 @@ def peaks():
         return 6650.0, 1400.0, "fallback"
 
 
+def measured_traffic(workload_name):
+    """DRAM bytes per attention launch from the committed ncu record
+    (profiles/attn_pair_traffic.json), scaled there to this workload; None
+    when the record is for another workload or the kernel source has changed
+    since the capture (a stale counter is not reported)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_pair_traffic.json")) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "head_latent_attention_09_b200", "csrc", "tc_attn_pair.cu")
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except Exception:
+        return None
+    if workload_name != WORKLOAD or rec.get("kernel_source_sha256") != sha:
+        return None
+    return float(rec["traffic_per_bench_launch"])
+
+
 def algorithmic_bytes(wl, ctx_sum, with_wo=False):
     """Bytes one step must move at least: the latent cache once (sum ctx * D *
     2) plus every weight once (W_DKV, W_KR, W_UK, W_UV [, W_O])."""
@@ -427,7 +446,8 @@ def run_ours(args):
                    "l2": "inputs larger than L2 (latent cache %.0f MB per rank)" % (attn_bytes / 1e6),
                    "parallelism": f"dp{world} (independent batches, no collective)"},
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": attn_gbs / hbm_peak, "traffic": None,
+                     "frac": attn_gbs / hbm_peak,
+                     "traffic": measured_traffic(wl.name) if not args.batch else None,
                      "peak_kind": peak_kind, "kernel": "mla_decode_attn (plan + attention)",
                      "attn_us": attn_ms * 1e3,
                      "frac_of_8TBps": attn_gbs / 8000.0,
