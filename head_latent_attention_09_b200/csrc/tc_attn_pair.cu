@@ -50,7 +50,7 @@ constexpr int kTileTok = 256;           // tokens per pair tile (MMA N of S = Q 
 constexpr int kHalfTok = 128;           // tokens of a tile each CTA stages for S
 constexpr int kSubTok = 64;             // tokens per O += P V sub-stage
 constexpr int kSlot = 16384;            // ring slot: a K chunk (128 rows x 128 B) or a V sub-stage
-constexpr int kSlots = 7;
+constexpr int kSlots = 7;               // 112 KB of ring: what is left beside Q (72 KB) and P (32 KB)
 constexpr int kQBytes = 9 * 8192;       // 64 heads x 576 bf16, nine 64-column chunks
 constexpr int kPBytes = 4 * 8192;       // 64 heads x 256 tokens bf16, four 64-token chunks
 constexpr float kRescale = 8.0f;        // rescale O only when the running max grows by > 2^8
