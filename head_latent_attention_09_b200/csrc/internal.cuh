@@ -29,6 +29,46 @@ enum GemmKind : int { kGemmSimt = 0, kGemmTc = 1 };
 
 }  // namespace mla
 
+namespace mla {
+
+// Programmatic dependent launch.  Kernels of this library are launched so
+// that the next kernel in the stream may begin while the current one
+// finishes (its set-up overlapping the tail); each kernel signals that its
+// dependents may launch, and waits for the kernels before it to complete
+// before it touches memory they write or read.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launches kern(args...) with programmatic stream serialization (and a
+// cluster shape when cluster_x > 1).  Only kernels that call pdl_wait()
+// before their first dependent memory access may be launched this way.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_x,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
+}  // namespace mla
+
 struct mla_handle {
   mla_config cfg;
   int device;

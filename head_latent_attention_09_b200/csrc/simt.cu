@@ -61,6 +61,8 @@ __device__ long long block_exclusive_scan(long long v, long long *smem, long lon
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, int P_req, char *ws,
                                                     WsLayout L, unsigned *status) {
+  pdl_trigger();
+  pdl_wait();   // the workspace may still be read by the previous step's combine
   __shared__ long long scan[1024];
   long long *tile_prefix = reinterpret_cast<long long *>(ws + L.tile_prefix_off);
   long long *piece_base = reinterpret_cast<long long *>(ws + L.piece_base_off);
@@ -208,6 +210,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(const char *ws, WsLayout L, int n_h, int d_c,
                                                       T *ctx_lat, float *lse_out) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x, h = blockIdx.y;
   const long long *pb = reinterpret_cast<const long long *>(ws + L.piece_base_off);
   const float *lse = reinterpret_cast<const float *>(ws + L.lse_off);
@@ -347,8 +351,7 @@ __global__ void __launch_bounds__(256) wo_simt_kernel(const T *o, const T *w_o, 
 // ---------------------------------------------------------------------------
 cudaError_t launch_plan(const int *ctx_len, int B, int P, char *ws, const WsLayout &L,
                         unsigned *status, cudaStream_t s) {
-  plan_kernel<<<1, 1024, 0, s>>>(ctx_len, B, P, ws, L, status);
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_len, B, P, ws, L, status);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s) {
@@ -382,6 +385,8 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *dst, float4
 template <typename T>
 __global__ void __launch_bounds__(256) combine_vec_kernel(const char *ws, WsLayout L, int B, int n_h, int d_c,
                                                           T *ctx_lat, float *lse_out) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * 8 + warp;   // = b * n_h + h
   if (row >= (long long)B * n_h) return;
@@ -440,19 +445,18 @@ cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout
     const long long rows = (long long)B * cfg.n_h;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     if (cfg.dtype == MLA_FP32)
-      combine_vec_kernel<float><<<blocks, 256, 0, s>>>(ws, L, B, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
+      return launch_pdl(combine_vec_kernel<float>, dim3(blocks), dim3(256), 0, s, 1, ws, L, B, cfg.n_h, cfg.d_c,
+                        (float *)ctx_lat, lse);
     else
-      combine_vec_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(ws, L, B, cfg.n_h, cfg.d_c,
-                                                              (__nv_bfloat16 *)ctx_lat, lse);
-    return cudaGetLastError();
+      return launch_pdl(combine_vec_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, s, 1, ws, L, B, cfg.n_h,
+                        cfg.d_c, (__nv_bfloat16 *)ctx_lat, lse);
   }
   dim3 grid(B, cfg.n_h);
   if (cfg.dtype == MLA_FP32)
-    combine_kernel<float><<<grid, 128, 0, s>>>(ws, L, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
+    return launch_pdl(combine_kernel<float>, grid, dim3(128), 0, s, 1, ws, L, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
   else
-    combine_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(ws, L, cfg.n_h, cfg.d_c,
-                                                       (__nv_bfloat16 *)ctx_lat, lse);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(128), 0, s, 1, ws, L, cfg.n_h, cfg.d_c,
+                      (__nv_bfloat16 *)ctx_lat, lse);
 }
 
 cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int T,

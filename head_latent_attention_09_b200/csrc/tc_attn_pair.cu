@@ -221,6 +221,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = ptx::cluster_ctarank();
   const bool leader = rank == 0;
   const int share = blockIdx.x >> 1;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
@@ -249,6 +250,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   ptx::cluster_sync_all();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The set-up above overlaps the previous kernel; from here on the plan,
+  // the query and the cache it wrote are read.
+  pdl_wait();
 
   if (warp == 0) {
     // --------------------------------------------------------------- producer
@@ -644,8 +648,7 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_pair_kernel<<<2 * P, kThreads, kSmemAlloc, s>>>(mq, mk, mv, a, rows);
-  return cudaGetLastError();
+  return launch_pdl(attn_pair_kernel, dim3(2 * P), dim3(kThreads), kSmemAlloc, s, 1, mq, mk, mv, a, rows);
 }
 
 }  // namespace mla

@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int share = blockIdx.x;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -168,6 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The set-up above overlaps the previous kernel; from here on the plan,
+  // the query and the cache it wrote are read.
+  pdl_wait();
 
   if (warp == 0) {
     // -------------------------------------------------------------- producer
@@ -499,8 +503,7 @@ cudaError_t launch_h(const AttnArgs &a, int P, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_smallh_kernel<H><<<P, kThreads, C::kSmem, s>>>(mq, mkv, a, rows);
-  return cudaGetLastError();
+  return launch_pdl(attn_smallh_kernel<H>, dim3(P), dim3(kThreads), C::kSmem, s, 1, mq, mkv, a, rows);
 }
 
 }  // namespace

@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool use_a1 = mt >= g.a_split_tile;   // (only with MT = 1)
   uint32_t tmem_cols = 32;
   while (tmem_cols < (uint32_t)(MT * BN)) tmem_cols <<= 1;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -170,13 +171,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t a_bytes = use_a1 ? (uint32_t)g.a1_rows * 128u : (uint32_t)kABytes;
       ptx::tma_prefetch_desc(mA);
       ptx::tma_prefetch_desc(&mapB);
-      int issued = 0;
-      for (int kl = 0; kl < nk; ++kl) {
+      // The weights (A) never depend on earlier kernels: the first stages'
+      // A tiles are requested before waiting for those kernels, the
+      // activations (B) after.
+      const int pre = nk < S ? nk : S;
+      auto load_a = [&](int kl) {
         const int s = kl % S, kc = kc0 + kl;
-        if (kl >= S && !ptx::mbar_wait(&empty[s], ((kl / S) - 1) & 1, g.status, abort_flag)) break;
-        ++issued;
         uint8_t *sa = base + s * kStage;
-        uint8_t *sb = sa + MT * kABytes;
         ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)mcount * a_bytes + (uint32_t)kBBytes);
         for (int t = 0; t < mcount; ++t) {
           uint8_t *st = sa + t * kABytes;
@@ -188,8 +189,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::tma_load_2d(st, mA, &full[s], kc * kKChunk, z * g.a_row_per_z + a_m0 + 128 * t);
           }
         }
+      };
+      auto load_b = [&](int kl) {
+        const int s = kl % S, kc = kc0 + kl;
+        uint8_t *sb = base + s * kStage + MT * kABytes;
         if (g.b_is_3d) ptx::tma_load_3d(sb, &mapB, &full[s], kc * kKChunk, z, n0);
         else ptx::tma_load_2d(sb, &mapB, &full[s], kc * kKChunk, n0);
+      };
+      for (int kl = 0; kl < pre; ++kl) load_a(kl);
+      pdl_wait();
+      for (int kl = 0; kl < pre; ++kl) load_b(kl);
+      int issued = pre;
+      for (int kl = pre; kl < nk; ++kl) {
+        const int s = kl % S;
+        if (!ptx::mbar_wait(&empty[s], ((kl / S) - 1) & 1, g.status, abort_flag)) break;
+        ++issued;
+        load_a(kl);
+        load_b(kl);
       }
       // Drain: do not leave while loads into this CTA's shared memory are in flight.
       for (int kl = issued - S > 0 ? issued - S : 0; kl < issued; ++kl) {
@@ -224,6 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();
     const int et = threadIdx.x - 64;  // 0..127
     if (g.mode == kEpiAppend) {
       for (int j = et; j < BN; j += 128) {
@@ -326,6 +343,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (split) {
     // Every CTA of the cluster reaches this point (all waits above are
     // bounded), so the two cluster barriers always complete.
+    pdl_wait();                // every thread below writes outputs
     ptx::cluster_sync_all();   // partials of all K slices are written
     const int ks = g.ksplit;
     if (ptx::cluster_nctarank() == (uint32_t)ks) {
@@ -418,23 +436,7 @@ cudaError_t launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUte
   }
   const int groups = (mtiles + g.mt_per_cta - 1) / g.mt_per_cta;
   const dim3 grid(groups * g.ksplit, ntiles, nz);
-  if (g.ksplit == 1) {
-    kern<<<grid, kGemmThreads, smem, s>>>(a0, a1, b, g);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = g.ksplit;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, g);
+  return launch_pdl(kern, grid, dim3(kGemmThreads), smem, s, g.ksplit, a0, a1, b, g);
 }
 
 // K split: the smallest power of two (<= 8, the portable cluster size) that
