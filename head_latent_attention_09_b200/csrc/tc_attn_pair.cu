@@ -31,10 +31,11 @@
 // sub-stages of 64 tokens x 128 columns (16 KB each), all through one ring of
 // 16 KB slots filled in the order the MMAs consume them.
 //
-// Warp roles per CTA (192 threads): warp 0 producer (TMA, and the hand copy
-// of a sequence's last partial block), warp 1 tensor-memory allocation and
-// (leader CTA only) MMA issue, warps 2-5 softmax, O rescale and epilogue (one
-// thread per tensor-memory lane).
+// Warp roles per CTA (224 threads): warps 0 and 6 producers (TMA, and the
+// hand copy of a sequence's last partial block; each owns half the ring's
+// slots), warp 1 tensor-memory allocation and (leader CTA only) MMA issue,
+// warps 2-5 softmax, O rescale and epilogue (one thread per tensor-memory
+// lane).
 //
 // Every wait is bounded; a wait that runs out flags MLA_ERR_TIMEOUT and the
 // kernel winds down without further waits.
@@ -45,7 +46,7 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kTileTok = 256;           // tokens per pair tile (MMA N of S = Q K^T)
 constexpr int kHalfTok = 128;           // tokens of a tile each CTA stages for S
 constexpr int kSubTok = 64;             // tokens per O += P V sub-stage
@@ -254,17 +255,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // the query and the cache it wrote are read.
   pdl_wait();
 
-  if (warp == 0) {
-    // --------------------------------------------------------------- producer
-    // Fills the ring in the order the MMAs consume it: the nine K chunks of
+  if (warp == 0 || warp == 6) {
+    // -------------------------------------------------------------- producers
+    // Fill the ring in the order the MMAs consume it: the nine K chunks of
     // tile i, then the V sub-stages of tile i-1 (tiles counted across the
-    // share's pieces).  Lane 0 issues TMA; the leader arms each slot with the
-    // bytes both CTAs' loads bring (the peer's loads count on the leader's
-    // barrier directly).  One producer takes every job in order, so a slot's
-    // empty barrier is never more than one phase behind the phase waited for
-    // (a parity wait cannot tell one phase behind from three); two producers
-    // splitting the jobs would each need to wait for the other to pass the
-    // slot's previous job first, and measured no faster.
+    // share's pieces).  Job j goes to slot j % kSlots; warp 0 owns the even
+    // slots and warp 6 the odd ones, so two warps keep TMA loads in flight at
+    // once (one issuing warp tops out near 40 GB/s per SM), while every slot
+    // still has one producer that visits its jobs in order: its empty barrier
+    // is never more than one phase behind the phase waited for (a parity wait
+    // cannot tell one phase behind from three).  Lane 0 issues TMA; the
+    // leader arms each slot with the bytes both CTAs' loads bring (the peer's
+    // loads count on the leader's barrier directly).  Warp 0 also loads Q.
+    const int pid = warp == 0 ? 0 : 1;
     const uint32_t lq = ptx::leader_addr(bars.qfull());
     const uint32_t lf0 = ptx::leader_addr(bars.full(0));
     if (lane == 0) {
@@ -281,18 +284,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     int ws_ = 0;               // ring slot of the next job
     int wround = 0;            // how many times the ring has been filled before
-    // Acquires the next ring slot (warp-uniform); returns its index or -1.
-    // In round r >= 1 a slot is free once the MMAs of round r-1 released it.
+    // Next ring job: returns its slot if this warp owns it (after waiting,
+    // in round r >= 1, until the MMAs of round r-1 released it), -2 if the
+    // other producer owns it, -1 on a failed wait.  Warp-uniform.
     auto acquire = [&]() -> int {
       const int s = ws_;
-      bool got = true;
-      if (lane == 0 && wround > 0) got = ptx::mbar_wait(bars.empty(s), (wround - 1) & 1, a.status, abort_flag);
-      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-      __syncwarp();
+      const int r = wround;
       if (++ws_ == kSlots) {
         ws_ = 0;
         ++wround;
       }
+      if ((s & 1) != pid) return -2;
+      bool got = true;
+      if (lane == 0 && r > 0) got = ptx::mbar_wait(bars.empty(s), (r - 1) & 1, a.status, abort_flag);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      __syncwarp();
       return got ? s : -1;
     };
     // V sub-stages of the tile at token t0 of piece p: tokens t0 + 64t..,
@@ -302,6 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int t = 0; t < nsub; ++t) {
         for (int g = 0; g < 2; ++g) {
           const int s = acquire();
+          if (s == -2) continue;
           if (s < 0) return false;
           uint8_t *dst = sRing + s * kSlot;
           const int tok0 = t0 + kSubTok * t;
@@ -348,8 +355,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (ok && walk_next(w, a, share, pc)) {
       bool qok = true;
       if (lane == 0) {
-        if (npc > 0) qok = ptx::mbar_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag);
-        if (qok) {
+        if (pid == 0 && npc > 0) qok = ptx::mbar_wait(bars.qempty(), (npc - 1) & 1, a.status, abort_flag);
+        if (pid == 0 && qok) {
           if (leader) ptx::mbar_arrive_expect_tx(bars.qfull(), 2 * kQBytes);
           for (int c = 0; c < 9; ++c)
             ptx::tma_load_2d_pair(sQ + c * 8192, &mapQ, lq, 64 * c, pc.b * 128 + 64 * (int)rank);
@@ -367,6 +374,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         for (int c = 0; c < 9; ++c) {
           const int s = acquire();
+          if (s == -2) continue;
           if (s < 0) { ok = false; break; }
           if (lane == 0) {
             uint8_t *dst = sRing + s * kSlot;
