@@ -30,7 +30,7 @@ EXPORTED = (
     "mla_cache_append", "mla_absorb_q", "mla_decode_workspace_size",
     "mla_default_num_parts", "mla_decode_attn", "mla_combine_splits", "mla_out_proj",
     "mla_get_device_status", "mla_plan_pieces", "mla_decode_attn_combine_noalloc",
-    "mla_noalloc_scratch_bytes",
+    "mla_noalloc_scratch_bytes", "mla_set_rope_scaling",
 )
 
 
@@ -75,6 +75,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_plan_pieces": (ll, [vp, i, i, vp]),
         "mla_decode_attn_combine_noalloc": (i, [vp, vp, vp, ll, vp, i, vp, i, i, vp, vp, vp]),
         "mla_noalloc_scratch_bytes": (sz, []),
+        "mla_set_rope_scaling": (i, [vp, ctypes.c_double, i, ctypes.c_double, ctypes.c_double,
+                                     ctypes.c_double]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -136,6 +138,11 @@ def mla_create(cfg: mla_config) -> int:
 
 def mla_destroy(handle: int) -> None:
     load().mla_destroy(handle)
+
+
+def mla_set_rope_scaling(handle, factor, original_ctx, alpha, beta, mscale_coef) -> None:
+    _check(load().mla_set_rope_scaling(handle, float(factor), int(original_ctx), float(alpha),
+                                       float(beta), float(mscale_coef)), "mla_set_rope_scaling")
 
 
 def mla_cache_append(handle, h, B, T, start_pos, w_dkv, w_kr, cache, cache_len,

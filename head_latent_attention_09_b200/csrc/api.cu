@@ -3,6 +3,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cmath>
+
 #include "internal.cuh"
 
 using namespace mla;
@@ -89,6 +91,7 @@ int mla_create(const mla_config *cfg, mla_handle **out) {
   }
   h->attn_kind = choose_attn(*cfg);
   h->gemm_kind = choose_gemm(*cfg);
+  h->score_mult = 1.0;
   if ((h->attn_kind != kAttnSimt || h->gemm_kind != kGemmSimt) && !tma_available()) {
     free(h);
     return MLA_ERR_CUDA;
@@ -114,6 +117,35 @@ void mla_destroy(mla_handle *h) {
   if (h->d_status) cudaFree(h->d_status);
   if (h->d_theta) cudaFree(h->d_theta);
   free(h);
+}
+
+int mla_set_rope_scaling(mla_handle *h, double factor, int original_ctx, double alpha, double beta,
+                         double mscale_coef) {
+  if (!h || !(factor >= 1.0) || original_ctx <= 0 || !(alpha >= 0.0) || !(beta > alpha) ||
+      !(mscale_coef >= 0.0) || !std::isfinite(factor) || !std::isfinite(beta) || !std::isfinite(mscale_coef))
+    return MLA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev != h->device) return MLA_ERR_INVALID_ARG;
+  const int d_r = h->cfg.d_r, nth = d_r / 2;
+  double *theta = (double *)malloc(sizeof(double) * (nth > 0 ? nth : 1));
+  if (!theta) return MLA_ERR_CUDA;
+  for (int k = 0; k < nth; ++k) {
+    const double th = pow(h->cfg.rope_base, -2.0 * k / (double)d_r);
+    double keep = 1.0;   // share of the original frequency (1: unchanged, 0: slowed by the factor)
+    if (factor > 1.0) {
+      const double turns = (double)original_ctx * th / (2.0 * 3.14159265358979323846);
+      keep = (turns - alpha) / (beta - alpha);
+      keep = keep < 0.0 ? 0.0 : (keep > 1.0 ? 1.0 : keep);
+    }
+    theta[k] = keep * th + (1.0 - keep) * th / factor;
+  }
+  const cudaError_t e = cudaMemcpy(h->d_theta, theta, sizeof(double) * nth, cudaMemcpyHostToDevice);
+  free(theta);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  const double m = factor > 1.0 ? mscale_coef * log(factor) + 1.0 : 1.0;
+  h->score_mult = m * m;
+  return MLA_OK;
 }
 
 int mla_cache_append(mla_handle *h, const void *x, int B, int T, const int *start_pos,
@@ -187,7 +219,7 @@ int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long lo
   a.n_h = c.n_h;
   a.d_c = c.d_c;
   a.d_r = c.d_r;
-  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)(c.d_h + c.d_r)));
+  a.scale_log2 = (float)(1.4426950408889634 * h->score_mult / sqrt((double)(c.d_h + c.d_r)));
   a.ws = (char *)workspace;
   a.L = L;
   a.status = h->d_status;

@@ -75,6 +75,7 @@ struct mla_handle {
   int num_sms;
   unsigned *d_status;  // device status word (kStatus* bits)
   double *d_theta;     // device [d_r/2] RoPE frequencies theta_k
+  double score_mult;   // YaRN temperature t multiplying every score (1 without scaling)
   int attn_kind;       // mla::AttnKind
   int gemm_kind;       // mla::GemmKind
 };

@@ -106,6 +106,26 @@ int mla_create(const mla_config *cfg, mla_handle **out);
  * flight that uses it).  NULL is accepted. */
 void mla_destroy(mla_handle *handle);
 
+/* Long-context scaling of the rotary part (YaRN): V2 §3.2.4 extends the 4K
+ * window to 128K with YaRN on the decoupled key k^R only, s = 40, alpha = 1,
+ * beta = 32, and a length-scaling factor sqrt(t) = c ln s + 1 (c = 0.0707 in
+ * the V2 paper, 0.1 in the V3 note's context-extension section).
+ *   factor        s >= 1 (1 turns the scaling off: plain RoPE, t = 1)
+ *   original_ctx  the window the frequencies were trained on (> 0)
+ *   alpha, beta   0 <= alpha < beta: a rotary pair that turns more than beta
+ *                 times over original_ctx keeps its frequency, one that turns
+ *                 fewer than alpha times is slowed by s, linear in between
+ *   mscale_coef   c >= 0; every score (content and rotary part) is multiplied
+ *                 by t = (c ln s + 1)^2, i.e. sqrt(t) scales query and key
+ * Replaces the handle's frequency table (synchronously, on the handle's
+ * device) and its score scale; applies to the calls made afterwards on this
+ * handle (mla_cache_append, mla_absorb_q, mla_decode_attn).  Rows already in
+ * a cache were rotated with the previous table, so set the scaling before
+ * filling the cache.  Errors: INVALID_ARG (NULL handle, bad values, wrong
+ * current device), CUDA. */
+int mla_set_rope_scaling(mla_handle *handle, double factor, int original_ctx, double alpha,
+                         double beta, double mscale_coef);
+
 /* Cache append (V3 note, MLA equations: c^KV_t = W^DKV h_t, k^R_t = RoPE(W^KR h_t);
  * V2 §2.1.3: the cached row is [c^KV_t ; k^R_t]).
  *   h          [B, T, d_model] hidden states of T new tokens per sequence

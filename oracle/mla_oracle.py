@@ -31,6 +31,16 @@ Readings of points the pages leave open (each is listed in the design doc):
 * ctx = 0 yields a zero output and log-sum-exp = -inf.
 * The log-sum-exp reported with an output is over the scaled scores
   s_j = q^T k_j / sqrt(d_h + d_h^R), in natural-log units.
+* Long-context RoPE scaling ("DeepSeek-V2", §3.2.4; the "DeepSeek-V3" note's
+  context-extension section) names YaRN (Peng et al.) with s = 40, alpha = 1,
+  beta = 32 over a 4K original window, applied to the decoupled rotary part,
+  and a length-scaling factor sqrt(t) = c ln s + 1 with c = 0.0707 in the V2
+  paper and c = 0.1 in the V3 note.  Reading: YaRN's per-frequency ramp (a
+  pair that turns more than beta times over the original window keeps its
+  frequency, one that turns fewer than alpha times is slowed by s, linear in
+  between), and sqrt(t) scaling both the query and the key, i.e. every score
+  (content and rotary part) multiplied by t = (c ln s + 1)^2; c is a
+  parameter, 0.0707 by default.  s = 1 is plain RoPE.
 
 Parity pins: every function below is pinned by tests/test_oracle_pins.py
 (closed forms, invariants, brute force, the pages' printed cache sizes).
@@ -39,6 +49,7 @@ Parity pins: every function below is pinned by tests/test_oracle_pins.py
 from __future__ import annotations
 
 import math
+from dataclasses import dataclass
 
 import numpy as np
 
@@ -49,16 +60,54 @@ F64 = np.float64
 # RoPE (decoupled part only)
 # ----------------------------------------------------------------------------
 
-def rope_theta(d_r: int, base: float) -> np.ndarray:
-    """theta_k = base^(-2k/d_r) for k = 0 .. d_r/2 - 1 (RoFormer frequencies)."""
+@dataclass(frozen=True)
+class RopeSpec:
+    """RoPE frequencies with optional YaRN scaling.  Every function that takes
+    ``base`` accepts either a plain base (float) or a RopeSpec."""
+    base: float = 10000.0
+    factor: float = 1.0          # s: context-extension ratio (1 = plain RoPE)
+    original_ctx: int = 4096     # the window the frequencies were trained on
+    alpha: float = 1.0           # below alpha turns over the window: fully slowed by s
+    beta: float = 32.0           # above beta turns: unchanged
+    mscale_coef: float = 0.0707  # c in sqrt(t) = c ln s + 1
+
+
+def _spec(base) -> RopeSpec:
+    return base if isinstance(base, RopeSpec) else RopeSpec(base=float(base))
+
+
+def rope_theta(d_r: int, base) -> np.ndarray:
+    """Rotation frequency of each pair k = 0 .. d_r/2 - 1.
+
+    Plain RoPE (RoFormer): theta_k = base^(-2k/d_r).  With YaRN (s > 1): the
+    pair turns r_k = L / (2 pi / theta_k) times over the original window L;
+    gamma_k = clip((r_k - alpha) / (beta - alpha), 0, 1) blends the slowed
+    frequency theta_k / s (gamma = 0) with the original one (gamma = 1)."""
+    spec = _spec(base)
     k = np.arange(d_r // 2, dtype=F64)
-    return np.power(F64(base), -2.0 * k / F64(d_r))
+    theta = np.power(F64(spec.base), -2.0 * k / F64(d_r))
+    if spec.factor <= 1.0:
+        return theta
+    turns = F64(spec.original_ctx) * theta / (2.0 * math.pi)
+    gamma = np.clip((turns - spec.alpha) / (spec.beta - spec.alpha), 0.0, 1.0)
+    return (1.0 - gamma) * theta / F64(spec.factor) + gamma * theta
+
+
+def attention_temperature(base) -> float:
+    """Multiplier t of every score: (c ln s + 1)^2 with YaRN (sqrt(t) scales
+    both the query and the key), 1 for plain RoPE."""
+    spec = _spec(base)
+    if spec.factor <= 1.0:
+        return 1.0
+    m = spec.mscale_coef * math.log(spec.factor) + 1.0
+    return m * m
 
 
 def rope(x: np.ndarray, pos, base: float) -> np.ndarray:
     """Rotate consecutive pairs of the last axis of ``x`` by pos * theta_k.
 
-    ``pos`` is a scalar or an array broadcastable to x.shape[:-1].
+    ``pos`` is a scalar or an array broadcastable to x.shape[:-1]; ``base``
+    is a plain base or a RopeSpec.
     """
     x = np.asarray(x, dtype=F64)
     d_r = x.shape[-1]
@@ -165,6 +214,12 @@ def softmax_scale(d_h: int, d_r: int) -> float:
     return 1.0 / math.sqrt(d_h + d_r)
 
 
+def attention_scale(d_h: int, d_r: int, base) -> float:
+    """The factor every score q . k is multiplied by: the softmax scale times
+    the YaRN temperature (1 for plain RoPE)."""
+    return softmax_scale(d_h, d_r) * attention_temperature(base)
+
+
 def mla_decode_explicit(q_nope, q_rope_raw, pos: int, rows, w_uk, w_uv, *, n_h, d_h, d_c,
                         d_r, base, heads=None):
     """One decode step for one sequence in the explicit form.
@@ -174,7 +229,7 @@ def mla_decode_explicit(q_nope, q_rope_raw, pos: int, rows, w_uk, w_uv, *, n_h, 
     qr = rope(np.asarray(q_rope_raw, F64)[heads], pos, base)
     q = np.concatenate([np.asarray(q_nope, F64)[heads], qr], axis=1)
     k, v = explicit_keys_values(rows, w_uk, w_uv, n_h, d_h, d_c, heads)
-    return softmax_attention(q, k, v, softmax_scale(d_h, d_r))
+    return softmax_attention(q, k, v, attention_scale(d_h, d_r, base))
 
 
 # ----------------------------------------------------------------------------
@@ -222,7 +277,7 @@ def mla_decode_absorbed(q_nope, q_rope_raw, pos, rows, w_uk, w_uv, *, n_h, d_h, 
     """Full absorbed decode step for one sequence: returns dict with q_abs,
     ctx_lat, lse, o (and u when W^O is given)."""
     q_abs = absorb_query(q_nope, q_rope_raw, pos, w_uk, n_h=n_h, d_h=d_h, d_r=d_r, base=base)
-    ctx_lat, lse = latent_attention(q_abs, rows, d_c=d_c, scale=softmax_scale(d_h, d_r))
+    ctx_lat, lse = latent_attention(q_abs, rows, d_c=d_c, scale=attention_scale(d_h, d_r, base))
     o, u = out_project(ctx_lat, w_uv, n_h=n_h, d_h=d_h, w_o=w_o)
     return {"q_abs": q_abs, "ctx_lat": ctx_lat, "lse": lse, "o": o, "u": u}
 
@@ -264,6 +319,27 @@ def brute_force_decode(h_seq, q_nope, q_rope_raw, w: dict, *, n_h, d_h, d_c, d_r
     multiply-add at a time.  Returns (o as nested lists [n_h][d_h], lse list [n_h])."""
     S = len(h_seq)
     d = len(h_seq[0])
+    # Frequencies and score scale again, one pair at a time (a second reading
+    # of the same definitions as rope_theta / attention_scale): a pair that
+    # turns at least beta times over the original window keeps theta, at most
+    # alpha times gets theta / s, and in between the linear blend.
+    spec = _spec(base)
+    theta = []
+    for p in range(d_r // 2):
+        th = spec.base ** (-2.0 * p / d_r)
+        if spec.factor > 1.0:
+            turns = spec.original_ctx * th / (2.0 * math.pi)
+            if turns >= spec.beta:
+                frac = 1.0
+            elif turns <= spec.alpha:
+                frac = 0.0
+            else:
+                frac = (turns - spec.alpha) / (spec.beta - spec.alpha)
+            th = frac * th + (1.0 - frac) * th / spec.factor
+        theta.append(th)
+    scale = 1.0 / math.sqrt(d_h + d_r)
+    if spec.factor > 1.0:
+        scale *= (spec.mscale_coef * math.log(spec.factor) + 1.0) ** 2
     rows = []
     for t in range(S):
         c = [sum(float(w["w_dkv"][r][k]) * float(h_seq[t][k]) for k in range(d))
@@ -272,8 +348,7 @@ def brute_force_decode(h_seq, q_nope, q_rope_raw, w: dict, *, n_h, d_h, d_c, d_r
                   for r in range(d_r)]
         kr = [0.0] * d_r
         for p in range(d_r // 2):
-            th = base ** (-2.0 * p / d_r)
-            a = t * th
+            a = t * theta[p]
             kr[2 * p] = kr_raw[2 * p] * math.cos(a) - kr_raw[2 * p + 1] * math.sin(a)
             kr[2 * p + 1] = kr_raw[2 * p] * math.sin(a) + kr_raw[2 * p + 1] * math.cos(a)
         rows.append((c, kr))
@@ -282,7 +357,7 @@ def brute_force_decode(h_seq, q_nope, q_rope_raw, w: dict, *, n_h, d_h, d_c, d_r
     for i in range(n_h):
         qr = [0.0] * d_r
         for p in range(d_r // 2):
-            a = pos * base ** (-2.0 * p / d_r)
+            a = pos * theta[p]
             x0, x1 = float(q_rope_raw[i][2 * p]), float(q_rope_raw[i][2 * p + 1])
             qr[2 * p] = x0 * math.cos(a) - x1 * math.sin(a)
             qr[2 * p + 1] = x0 * math.sin(a) + x1 * math.cos(a)
@@ -295,7 +370,7 @@ def brute_force_decode(h_seq, q_nope, q_rope_raw, w: dict, *, n_h, d_h, d_c, d_r
                   for r in range(d_h)]
             dot = sum(float(q_nope[i][r]) * kc[r] for r in range(d_h))
             dot += sum(qr[r] * kr[r] for r in range(d_r))
-            scores.append(dot / math.sqrt(d_h + d_r))
+            scores.append(dot * scale)
             vals.append(vc)
         mx = max(scores)
         e = [math.exp(s - mx) for s in scores]

@@ -39,6 +39,28 @@ def config_of(wl) -> M.mla_config:
                         dtype=M.MLA_BF16 if wl.dtype == "bf16" else M.MLA_FP32)
 
 
+def rope_arg(wl):
+    """The oracle's `base` argument for a workload: a plain base, or a RopeSpec
+    carrying its YaRN scaling."""
+    if wl.rope_scaling is None:
+        return wl.rope_base
+    s, orig, alpha, beta, coef = wl.rope_scaling
+    return O.RopeSpec(base=wl.rope_base, factor=s, original_ctx=orig, alpha=alpha, beta=beta,
+                      mscale_coef=coef)
+
+
+def create_handle(wl) -> int:
+    """mla_create for the workload, with its RoPE scaling applied."""
+    handle = M.mla_create(config_of(wl))
+    if wl.rope_scaling is not None:
+        try:
+            M.mla_set_rope_scaling(handle, *wl.rope_scaling)
+        except Exception:
+            M.mla_destroy(handle)
+            raise
+    return handle
+
+
 def torch_dtype(wl):
     return torch.bfloat16 if wl.dtype == "bf16" else torch.float32
 
@@ -101,8 +123,7 @@ class DeviceCache:
 
 def run_decode_step(wl, num_parts=0, with_wo=False, dev="cuda", keep=False, fill_rows=None):
     """One decode step for every sequence of the workload.  Returns host arrays."""
-    cfg = config_of(wl)
-    handle = M.mla_create(cfg)
+    handle = create_handle(wl)
     try:
         wnp = draw_weights(wl, with_wo=with_wo)
         w = {k: to_dev(v, wl, dev) for k, v in wnp.items()}
@@ -170,11 +191,12 @@ def oracle_step(wl, seqs, with_wo=False, explicit_heads=None, fill_rows=None):
     ctx = ctx_lengths(wl)
     qn, qr = queries(wl)
     res = {k: {} for k in ("q_abs", "ctx_lat", "lse", "o", "u", "cache_new_rows", "o_explicit")}
-    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base)
+    base = rope_arg(wl)
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=base)
     for b in seqs:
         n = int(ctx[b])
         hb = hidden_states(wl, b, n) if fill_rows is None else fill_rows(b, n)
-        rows = O.cache_rows(hb, w["w_dkv"], w["w_kr"], np.arange(n), wl.rope_base)
+        rows = O.cache_rows(hb, w["w_dkv"], w["w_kr"], np.arange(n), base)
         r = O.mla_decode_absorbed(qn[b], qr[b], max(n - 1, 0), rows, w["w_uk"], w["w_uv"],
                                   w_o=w.get("w_o"), **kw)
         for k in ("q_abs", "ctx_lat", "lse", "o", "u"):

@@ -57,6 +57,24 @@ def _combine_bad_lse(parts):
     ctx, lse = _ORIG_COMBINE(parts)
     return ctx, lse + 1e-6
 
+_ORIG_THETA = O.rope_theta
+
+
+def _yarn_ramp_inverted(d_r, base):
+    # slows the fast pairs and keeps the slow ones (the ramp read backwards)
+    spec = O._spec(base)
+    plain = _ORIG_THETA(d_r, spec.base)
+    if spec.factor <= 1.0:
+        return plain
+    scaled = _ORIG_THETA(d_r, spec)
+    return plain * plain / np.where(scaled == 0, 1.0, scaled) / spec.factor
+
+
+def _temperature_not_squared(base):
+    spec = O._spec(base)
+    return 1.0 if spec.factor <= 1.0 else spec.mscale_coef * math.log(spec.factor) + 1.0
+
+
 MUTATIONS = [
     ("scale_without_rope_width", "softmax_scale", lambda d_h, d_r: 1.0 / math.sqrt(d_h),
      [P.test_two_token_softmax_closed_form]),
@@ -68,6 +86,11 @@ MUTATIONS = [
      [lambda: P.test_brute_force_tiny_workload(0)]),
     ("combine_lse_off", "combine_partials", _combine_bad_lse,
      [lambda: P.test_split_combine_is_exact((0, 10, 11, 40, 64))]),
+    ("yarn_ramp_inverted", "rope_theta", _yarn_ramp_inverted,
+     [P.test_yarn_keeps_fast_pairs_and_slows_slow_pairs_by_s,
+      lambda: P.test_yarn_absorbed_explicit_and_brute_force_agree(0.0707)]),
+    ("yarn_temperature_not_squared", "attention_temperature", _temperature_not_squared,
+     [lambda: P.test_yarn_absorbed_explicit_and_brute_force_agree(0.1)]),
 ]
 
 

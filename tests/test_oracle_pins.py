@@ -309,3 +309,85 @@ def test_cache_rows_by_hand():
     want = [raw[0] * math.cos(a0) - raw[1] * math.sin(a0), raw[0] * math.sin(a0) + raw[1] * math.cos(a0),
             raw[2] * math.cos(a1) - raw[3] * math.sin(a1), raw[2] * math.sin(a1) + raw[3] * math.cos(a1)]
     assert np.allclose(row[d_c:], want, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# YaRN long-context scaling of the rotary part ("DeepSeek-V2" §3.2.4; the
+# "DeepSeek-V3" note's context extension): s = 40, alpha = 1, beta = 32 over a
+# 4K window, sqrt(t) = c ln s + 1
+# --------------------------------------------------------------------------
+
+V2_YARN = O.RopeSpec(base=10000.0, factor=40.0, original_ctx=4096, alpha=1.0, beta=32.0,
+                     mscale_coef=0.0707)
+
+
+def test_yarn_with_factor_one_is_plain_rope():
+    spec = O.RopeSpec(base=10000.0, factor=1.0)
+    assert np.array_equal(O.rope_theta(64, spec), O.rope_theta(64, 10000.0))
+    assert O.attention_temperature(spec) == 1.0
+    x = np.random.default_rng(3).standard_normal((5, 64))
+    assert np.array_equal(O.rope(x, 777, spec), O.rope(x, 777, 10000.0))
+
+
+def test_yarn_keeps_fast_pairs_and_slows_slow_pairs_by_s():
+    d_r = 64
+    plain = O.rope_theta(d_r, 10000.0)
+    ratio = O.rope_theta(d_r, V2_YARN) / plain
+    # turns of each pair over the original 4096-token window
+    turns = 4096 * plain / (2 * math.pi)
+    assert turns[0] > 32 and turns[-1] < 1                      # both regimes occur at d_r = 64
+    assert np.all(ratio[turns >= 32] == 1.0)                    # fast pairs unchanged
+    assert np.allclose(ratio[turns <= 1], 1 / 40.0, rtol=1e-15) # slow pairs slowed by s
+    mid = (turns > 1) & (turns < 32)
+    assert mid.any() and np.all((ratio[mid] > 1 / 40.0) & (ratio[mid] < 1.0))
+    assert np.all(np.diff(ratio) <= 1e-15)                      # never faster for slower pairs
+
+
+def test_yarn_rope_keeps_norm_and_relative_position():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((20, 64))
+    pos = rng.integers(0, 163840, size=20)
+    y = O.rope(x, pos, V2_YARN)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    ref = O.rope(q, 131071, V2_YARN) @ O.rope(k, 5, V2_YARN)
+    got = O.rope(q, 131071 - 5, V2_YARN) @ O.rope(k, 0, V2_YARN)
+    assert abs(got - ref) <= 1e-9 * max(1.0, abs(ref))
+
+
+def test_yarn_temperature_acts_as_a_query_scale():
+    # Every score is multiplied by t, so the step equals a plain-temperature
+    # step (same frequencies) on the query scaled by t.
+    wl, w, rows, qn, qr = _tiny_inputs(seed=5)
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r)
+    spec = O.RopeSpec(base=wl.rope_base, factor=40.0, original_ctx=16, alpha=1.0, beta=32.0,
+                      mscale_coef=0.0707)
+    t = O.attention_temperature(spec)
+    assert t > 1.0
+    assert O.attention_temperature(O.RopeSpec(factor=40.0, mscale_coef=0.1)) > t
+    res = O.mla_decode_absorbed(qn, qr, 22, rows, w["w_uk"], w["w_uv"], base=spec, **kw)
+    q_abs = O.absorb_query(qn, qr, 22, w["w_uk"], n_h=wl.n_h, d_h=wl.d_h, d_r=wl.d_r, base=spec)
+    ctx, lse = O.latent_attention(q_abs * t, rows, d_c=wl.d_c, scale=O.softmax_scale(wl.d_h, wl.d_r))
+    assert _rel(res["ctx_lat"], ctx) <= 1e-13
+    assert np.allclose(res["lse"], lse, rtol=1e-13)
+
+
+@pytest.mark.parametrize("coef", [0.0707, 0.1])
+def test_yarn_absorbed_explicit_and_brute_force_agree(coef):
+    wl = TINY
+    w = draw_weights(wl)
+    b, ctx = 1, wl.ctx[1]
+    h = hidden_states(wl, b, ctx)
+    qn, qr = queries(wl)
+    spec = O.RopeSpec(base=wl.rope_base, factor=40.0, original_ctx=16, alpha=1.0, beta=32.0,
+                      mscale_coef=coef)
+    assert not np.array_equal(O.rope_theta(wl.d_r, spec), O.rope_theta(wl.d_r, wl.rope_base))
+    kw = dict(n_h=wl.n_h, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, base=spec)
+    rows = O.cache_rows(h, w["w_dkv"], w["w_kr"], np.arange(ctx), spec)
+    res = O.mla_decode_absorbed(qn[b], qr[b], ctx - 1, rows, w["w_uk"], w["w_uv"], **kw)
+    o_ex, lse_ex = O.mla_decode_explicit(qn[b], qr[b], ctx - 1, rows, w["w_uk"], w["w_uv"], **kw)
+    bf_o, bf_lse = O.brute_force_decode(h.tolist(), qn[b].tolist(), qr[b].tolist(),
+                                        {k: v.tolist() for k, v in w.items()}, **kw)
+    assert _rel(res["o"], bf_o) <= 1e-12
+    assert _rel(o_ex, bf_o) <= 1e-12
+    assert np.allclose(res["lse"], bf_lse, rtol=1e-12)

@@ -46,6 +46,10 @@ class Workload:
     d_cq: int | None = None         # query compression width d'_c, None = no query compression
     page_size: int = 0              # 0 = contiguous cache, else tokens per block
     rope_base: float = 10000.0
+    # YaRN long-context scaling of the rotary part, passed through unchanged to
+    # the library and the oracle: (factor s, original window, alpha, beta,
+    # coefficient c of sqrt(t) = c ln s + 1); None = plain RoPE.
+    rope_scaling: tuple | None = None
     note: str = field(default="", compare=False)
 
     @property
