@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch size (small cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-query-proj", action="store_true",
+                    help="skip the separate timing of the query projection")
     return ap.parse_args()
 
 
@@ -82,6 +84,21 @@ def algorithmic_bytes(wl, ctx_sum, with_wo=False):
     if with_wo:
         w += wl.d_model * wl.n_h * wl.d_h
     return ctx_sum * wl.D * esz + w * esz
+
+
+def query_proj_bytes(wl, B):
+    """Bytes mla_query_proj must move at least: its weights once (W^DQ, W^UQ,
+    W^QR, or W^Q, W^QR without query compression), the hidden states read,
+    c^Q written and read back by the two up-projections, q^C and q^R written."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    nq = wl.n_h * (wl.d_h + wl.d_r)
+    if wl.d_cq:
+        w = wl.d_cq * wl.d_model + nq * wl.d_cq
+        act = B * wl.d_model + 3 * B * wl.d_cq + B * nq
+    else:
+        w = nq * wl.d_model
+        act = B * wl.d_model + B * nq
+    return (w + act) * esz
 
 
 def algorithmic_flops(wl, ctx_sum):
@@ -399,6 +416,39 @@ def run_ours(args):
     per_call = {n: float(np.mean([ev[j].elapsed_time(ev[j + 1]) for ev in call_ev])) * 1e3
                 for j, n in enumerate(names)}
 
+    # ---- the query projection from the hidden state (upstream of the step):
+    # its weights fit in L2, so a buffer larger than L2 is written before every
+    # call and the events bracket the call alone.
+    qproj = None
+    if not args.no_query_proj:
+        if wl.d_cq:
+            w_dq = randn(wl.d_cq, d, std=d ** -0.5)
+            w_uq = randn(H * wl.d_h, wl.d_cq, std=wl.d_cq ** -0.5)
+            w_qr = randn(H * wl.d_r, wl.d_cq, std=wl.d_cq ** -0.5)
+            c_q = torch.empty((B, wl.d_cq), dtype=bf, device=dev)
+        else:
+            w_dq, c_q = None, None
+            w_uq = randn(H * wl.d_h, d, std=d ** -0.5)
+            w_qr = randn(H * wl.d_r, d, std=d ** -0.5)
+        qn_out = torch.empty_like(q_nope)
+        qr_out = torch.empty_like(q_rope)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        q_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for i in range(3 + args.steps):
+            flush.fill_(i & 0xFF)
+            if i >= 3:
+                q_ev[i - 3][0].record(stream)
+            M.mla_query_proj(handle, h_new, B, w_dq, wl.d_cq or 0, w_uq, w_qr, c_q, qn_out, qr_out, sh)
+            if i >= 3:
+                q_ev[i - 3][1].record(stream)
+        torch.cuda.synchronize()
+        st = M.mla_get_device_status(handle, sh)
+        if st != M.MLA_OK:
+            raise M.MlaError(st, "device status after the query projection")
+        q_us = float(np.mean([ev[0].elapsed_time(ev[1]) for ev in q_ev])) * 1e3
+        del flush
+        qproj = {"us": q_us, "bytes": query_proj_bytes(wl, B)}
+
     # ---- end to end: host buffers in pinned memory, copies inside the timed region
     hp = {k: v.cpu().pin_memory() for k, v in
           (("h_new", h_new), ("q_nope", q_nope), ("q_rope", q_rope), ("pos", pos), ("ctx", ctx_d))}
@@ -479,6 +529,12 @@ def run_ours(args):
         "clocks": clk,
         "cpu_baseline": cpu,
     }
+    if qproj is not None:
+        gbs = qproj["bytes"] / (qproj["us"] * 1e-6) / 1e9
+        line["query_proj"] = {
+            "us": qproj["us"], "algorithmic_bytes": qproj["bytes"], "achieved_gbs": gbs,
+            "frac": gbs / hbm_peak, "bound": "hbm",
+            "note": "mla_query_proj alone, L2 flushed before each call; not part of the step"}
     print(json.dumps(line), flush=True)
 
 

@@ -29,6 +29,7 @@ EXPORTED = (
     "mla_status_string", "mla_config_validate", "mla_create", "mla_destroy",
     "mla_cache_append", "mla_absorb_q", "mla_decode_workspace_size",
     "mla_default_num_parts", "mla_decode_attn", "mla_combine_splits", "mla_out_proj",
+    "mla_query_proj",
     "mla_get_device_status", "mla_plan_pieces", "mla_decode_attn_combine_noalloc",
     "mla_noalloc_scratch_bytes", "mla_set_rope_scaling",
 )
@@ -71,6 +72,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_decode_attn": (i, [vp, vp, vp, ll, vp, i, vp, i, i, vp, sz, vp]),
         "mla_combine_splits": (i, [vp, vp, sz, i, i, vp, vp, vp]),
         "mla_out_proj": (i, [vp, vp, vp, vp, vp, vp, i, vp]),
+        "mla_query_proj": (i, [vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp]),
         "mla_get_device_status": (i, [vp, vp]),
         "mla_plan_pieces": (ll, [vp, i, i, vp]),
         "mla_decode_attn_combine_noalloc": (i, [vp, vp, vp, ll, vp, i, vp, i, i, vp, vp, vp]),
@@ -176,6 +178,12 @@ def mla_combine_splits(handle, workspace, ws_bytes, B, num_parts, ctx_lat, lse=N
     _check(load().mla_combine_splits(handle, _ptr(workspace), ws_bytes, B, num_parts,
                                      _ptr(ctx_lat), _ptr(lse), _stream(stream)),
            "mla_combine_splits")
+
+
+def mla_query_proj(handle, x, B, w_dq, d_cq, w_uq, w_qr, c_q, q_nope, q_rope, stream=None):
+    _check(load().mla_query_proj(handle, _ptr(x), B, _ptr(w_dq), d_cq, _ptr(w_uq), _ptr(w_qr),
+                                 _ptr(c_q), _ptr(q_nope), _ptr(q_rope), _stream(stream)),
+           "mla_query_proj")
 
 
 def mla_out_proj(handle, ctx_lat, w_uv, w_o, o, u, B, stream=None):

@@ -264,6 +264,40 @@ int mla_out_proj(mla_handle *h, const void *ctx_lat, const void *w_uv, const voi
   return MLA_OK;
 }
 
+namespace {
+// y[N, M] = x[N, K] w[M, K]^T on the handle's GEMM path, CUDA cores when the
+// tensor-core kernel lacks the shape (or for fp32).
+cudaError_t linear(const mla_handle *h, const void *x, const void *w, void *y, int M, int K, int N,
+                   cudaStream_t s) {
+  cudaError_t e = cudaErrorNotSupported;
+  if (h->gemm_kind == kGemmTc) e = launch_linear_tc(x, w, y, M, K, N, s);
+  if (e == cudaErrorNotSupported) e = launch_linear_simt(x, w, y, M, K, N, h->cfg.dtype == MLA_FP32, s);
+  return e;
+}
+}  // namespace
+
+int mla_query_proj(mla_handle *h, const void *x, int B, const void *w_dq, int d_cq, const void *w_uq,
+                   const void *w_qr, void *c_q, void *q_nope, void *q_rope, mla_stream_t stream) {
+  if (!h || B < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!x || !w_uq || !w_qr || !q_nope || !q_rope) return MLA_ERR_INVALID_ARG;
+  if (w_dq && (!c_q || d_cq <= 0)) return MLA_ERR_INVALID_ARG;
+  const mla_config &c = h->cfg;
+  cudaStream_t s = (cudaStream_t)stream;
+  const void *src = x;
+  int K = c.d_model;
+  cudaError_t e = cudaSuccess;
+  if (w_dq) {
+    e = linear(h, x, w_dq, c_q, d_cq, c.d_model, B, s);
+    src = c_q;
+    K = d_cq;
+  }
+  if (e == cudaSuccess) e = linear(h, src, w_uq, q_nope, c.n_h * c.d_h, K, B, s);
+  if (e == cudaSuccess) e = linear(h, src, w_qr, q_rope, c.n_h * c.d_r, K, B, s);
+  if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
 int mla_get_device_status(mla_handle *h, mla_stream_t stream) {
   if (!h) return MLA_ERR_INVALID_ARG;
   unsigned v = 0;

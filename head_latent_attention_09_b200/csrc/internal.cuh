@@ -173,6 +173,9 @@ cudaError_t launch_outproj_simt(const mla_config &cfg, const void *ctx_lat, cons
                                 void *o, int B, cudaStream_t s);
 cudaError_t launch_wo_simt(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
                            cudaStream_t s);
+// y[N, M] = x[N, K] w[M, K]^T (row-major, the config's dtype).
+cudaError_t launch_linear_simt(const void *x, const void *w, void *y, int M, int K, int N, bool fp32,
+                               cudaStream_t s);
 
 // tcgen05 paths (bf16 only); return cudaErrorNotSupported for shapes they lack.
 cudaError_t launch_append_tc(const mla_config &cfg, const void *h, int B, int T,
@@ -187,6 +190,7 @@ cudaError_t launch_outproj_tc(const mla_config &cfg, const void *ctx_lat, const 
                               void *o, int B, cudaStream_t s);
 cudaError_t launch_wo_tc(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
                          cudaStream_t s);
+cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, cudaStream_t s);
 cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s);
 cudaError_t launch_attn_tc_smallh(const AttnArgs &a, int P, cudaStream_t s);
 

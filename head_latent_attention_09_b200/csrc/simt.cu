@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(256) outproj_simt_kernel(const T *ctx, const T
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) wo_simt_kernel(const T *o, const T *w_o, T *u, int K, int d) {
+__global__ void __launch_bounds__(256) linear_simt_kernel(const T *o, const T *w_o, T *u, int K, int d) {
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.y * (blockDim.x >> 5) + warp;
@@ -511,17 +511,22 @@ cudaError_t launch_outproj_simt(const mla_config &cfg, const void *ctx_lat, cons
   return cudaGetLastError();
 }
 
+cudaError_t launch_linear_simt(const void *x, const void *w, void *y, int M, int K, int N, bool fp32,
+                               cudaStream_t s) {
+  // y[N, M] = x[N, K] w[M, K]^T: one warp per output element.
+  if (M <= 0 || N <= 0 || K <= 0 || (M + 7) / 8 > 65535) return cudaErrorNotSupported;
+  dim3 grid(N, (M + 7) / 8);
+  if (fp32)
+    linear_simt_kernel<float><<<grid, 256, 0, s>>>((const float *)x, (const float *)w, (float *)y, K, M);
+  else
+    linear_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w,
+                                                       (__nv_bfloat16 *)y, K, M);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_wo_simt(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
                            cudaStream_t s) {
-  const int K = cfg.n_h * cfg.d_h;
-  dim3 grid(B, (cfg.d_model + 7) / 8);
-  if (cfg.dtype == MLA_FP32)
-    wo_simt_kernel<float><<<grid, 256, 0, s>>>((const float *)o, (const float *)w_o, (float *)u, K,
-                                               cfg.d_model);
-  else
-    wo_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)w_o, (__nv_bfloat16 *)u, K, cfg.d_model);
-  return cudaGetLastError();
+  return launch_linear_simt(o, w_o, u, cfg.d_model, cfg.n_h * cfg.d_h, B, cfg.dtype == MLA_FP32, s);
 }
 
 }  // namespace mla

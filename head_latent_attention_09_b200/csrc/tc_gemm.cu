@@ -551,28 +551,32 @@ cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const vo
   return dispatch_bn<false>(B, ma, ma, mb, g, c.d_h / 128, c.n_h, s, bn);
 }
 
-cudaError_t launch_wo_tc(const mla_config &c, const void *o, const void *w_o, void *u, int B, cudaStream_t s) {
-  const int K = c.n_h * c.d_h;
-  if (!aligned16(o) || !aligned16(w_o) || K % 64 != 0) return cudaErrorNotSupported;
-  const int bn = pick_bn(B);
+cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, cudaStream_t s) {
+  // y[N, M] = x[N, K] w[M, K]^T, bf16 in and out, fp32 accumulation.
+  if (!aligned16(x) || !aligned16(w) || K % 64 != 0 || M <= 0 || N <= 0) return cudaErrorNotSupported;
+  const int bn = pick_bn(N);
   CUtensorMap ma, mb;
-  const uint64_t da[2] = {(uint64_t)K, (uint64_t)c.d_model};
+  const uint64_t da[2] = {(uint64_t)K, (uint64_t)M};
   const uint64_t sa[1] = {(uint64_t)K * 2};
   const uint32_t ba[2] = {64, 128};
-  const uint64_t db[2] = {(uint64_t)K, (uint64_t)B};
+  const uint64_t db[2] = {(uint64_t)K, (uint64_t)N};
   const uint64_t sb[1] = {(uint64_t)K * 2};
   const uint32_t bb[2] = {64, (uint32_t)bn};
-  if (!encode_map_bf16(&ma, w_o, 2, da, sa, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mb, o, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_map_bf16(&ma, w, 2, da, sa, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mb, x, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiWo;
   g.num_k_chunks = K / kKChunk;
-  g.M_valid = c.d_model;
-  g.N = B;
-  g.out = (__nv_bfloat16 *)u;
-  g.out_ld = c.d_model;
-  return dispatch_bn<false>(B, ma, ma, mb, g, (c.d_model + 127) / 128, 1, s, bn);
+  g.M_valid = M;
+  g.N = N;
+  g.out = (__nv_bfloat16 *)y;
+  g.out_ld = M;
+  return dispatch_bn<false>(N, ma, ma, mb, g, (M + 127) / 128, 1, s, bn);
+}
+
+cudaError_t launch_wo_tc(const mla_config &c, const void *o, const void *w_o, void *u, int B, cudaStream_t s) {
+  return launch_linear_tc(o, w_o, u, c.d_model, c.n_h * c.d_h, B, s);
 }
 
 cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, const int *start_pos,

@@ -19,6 +19,8 @@
  *   mla_decode_attn     split-KV softmax over the latent rows -> partials
  *   mla_combine_splits  log-sum-exp merge of the partials -> ctx_lat
  *   mla_out_proj        o_i = W^UV_i ctx_lat_i  (and optionally u = W^O o)
+ * and, ahead of mla_absorb_q when the caller starts from the hidden state,
+ *   mla_query_proj      q^C, q^R (unrotated) from h, with or without W^DQ
  *
  * Conventions for every call
  *   - Tensor pointers are DEVICE memory owned by the caller, row-major and
@@ -138,6 +140,24 @@ int mla_set_rope_scaling(mla_handle *handle, double factor, int original_ctx, do
 int mla_cache_append(mla_handle *handle, const void *h, int B, int T, const int *start_pos,
                      const void *w_dkv, const void *w_kr, void *cache, long long cache_len,
                      const int *block_table, int max_blocks_per_seq, mla_stream_t stream);
+
+/* Query projection of the current token, before absorption (V2 §2.1.2 query
+ * compression, c^Q_t = W^DQ h_t, q^C_t = W^UQ c^Q_t; §2.1.3 q^R_t = W^QR c^Q_t,
+ * rotated later by mla_absorb_q; Appendix B: V2-Lite has no query compression,
+ * q^C_t = W^Q h_t and q^R_t = W^QR h_t):
+ *   x      [B, d_model] hidden state of each sequence's new token
+ *   w_dq   [d_cq, d_model] (W^DQ), or NULL for the uncompressed form
+ *   d_cq   query compression width d_c' (ignored when w_dq is NULL)
+ *   w_uq   [n_h*d_h, d_cq] (W^UQ), or W^Q [n_h*d_h, d_model] when w_dq is NULL
+ *   w_qr   [n_h*d_r, d_cq], or [n_h*d_r, d_model] when w_dq is NULL
+ *   c_q    [B, d_cq] (out) the compressed query, or NULL when w_dq is NULL
+ *   q_nope [B, n_h, d_h] (out), q_rope [B, n_h, d_r] (out, not yet rotated):
+ *          the inputs mla_absorb_q takes.
+ * No normalisation is applied to c^Q.  Every product accumulates in fp32; c_q
+ * is stored in cfg.dtype and the up-projections read that stored value. */
+int mla_query_proj(mla_handle *handle, const void *x, int B, const void *w_dq, int d_cq,
+                   const void *w_uq, const void *w_qr, void *c_q, void *q_nope, void *q_rope,
+                   mla_stream_t stream);
 
 /* Query absorption (V2 Appendix C; V3 note q_{t,i} = [q^C_{t,i} ; q^R_{t,i}]):
  *   q_abs[b,i,:d_c]  = W^UK_i^T q_nope[b,i,:]        (W^UK_i = rows i*d_h.. of W^UK)

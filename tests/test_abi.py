@@ -76,6 +76,8 @@ def test_create_without_device_fails_cleanly(lib):
     assert lib.mla_get_device_status(None, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_absorb_q(None, None, None, None, None, None, 1, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_set_rope_scaling(None, 40.0, 4096, 1.0, 32.0, 0.0707) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_query_proj(None, None, 1, None, 0, None, None, None, None, None,
+                              None) == M.MLA_ERR_INVALID_ARG
 
 
 def python_plan(ctx, P):
