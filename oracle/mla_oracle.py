@@ -41,6 +41,16 @@ Readings of points the pages leave open (each is listed in the design doc):
   between), and sqrt(t) scaling both the query and the key, i.e. every score
   (content and rotary part) multiplied by t = (c ln s + 1)^2; c is a
   parameter, 0.0707 by default.  s = 1 is plain RoPE.
+* FP8 latent cache ("DeepSeek-V2" §3.2.3 quantises the deployed KV cache to
+  about 6 bits per element without giving the format; the "DeepSeek-V3" note's
+  FP8 section quantises activations tile-wise, per token and per 128 channels,
+  with the group's absolute maximum setting the scale).  Reading: each cached
+  row is cut into 128-channel groups, over c^KV and separately over k^R; a
+  group's scale is sigma = amax / 448 and its elements are stored as OCP FP8
+  E4M3 codes of x / sigma (round to nearest even, saturating at 448), both
+  divisions in float32, which is also where the GPU takes these decisions.  A
+  group of zeros has sigma = 0 and zero codes.  The stored value is
+  code * sigma.
 
 Parity pins: every function below is pinned by tests/test_oracle_pins.py
 (closed forms, invariants, brute force, the pages' printed cache sizes).
@@ -150,6 +160,86 @@ def kv_cache_elements_per_token(kind: str, *, n_h: int, d_h: int, layers: int = 
     if kind == "MLA":
         return (d_c + d_r) * layers
     raise ValueError(kind)
+
+
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) latent cache: per-token, per-128-channel-group scales
+# ----------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+FP8_GROUP = 128
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each OCP FP8 E4M3 code (float64): sign bit, four exponent bits
+    with bias 7, three mantissa bits; exponent field 0 holds the subnormals
+    m * 2^-9; S.1111.111 is NaN and there are no infinities."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(F64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2((e - 7).astype(F64)))
+    mag = np.where((e == 15) & (c & 7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """E4M3 code of each value (uint8): round to nearest, ties to even, finite
+    values beyond 448 saturate to +-448.  ``v`` is taken as float32."""
+    x = np.asarray(v, dtype=np.float32).astype(F64)
+    sign = np.signbit(x)
+    a = np.abs(x)
+    # spacing of representable magnitudes around a: 2^(e-3) in the binade
+    # [2^e, 2^(e+1)) for e >= -6, and 2^-9 below 2^-6 (subnormals)
+    e = np.frexp(np.where(a > 0, a, 1.0))[1] - 1
+    e = np.maximum(e, -6)
+    quantum = np.exp2((e - 3).astype(F64))
+    mag = np.rint(a / quantum) * quantum            # exact scaling; rint is half-to-even
+    mag = np.minimum(mag, E4M3_MAX)
+    sub = mag < 2.0 ** -6
+    ef = np.frexp(np.where(sub, 1.0, mag))[1] - 1   # binade of a normal result
+    mant = np.where(sub, mag / 2.0 ** -9, mag / np.exp2(ef.astype(F64)) * 8.0 - 8.0)
+    efield = np.where(sub, 0, ef + 7)
+    code = (sign.astype(np.int64) << 7) | (efield.astype(np.int64) << 3) | np.rint(mant).astype(np.int64)
+    return code.astype(np.uint8)
+
+
+def fp8_groups(d_c: int, d_r: int):
+    """Channel ranges [a, b) of a cached row's scale groups: 128-wide groups
+    over c^KV, then over k^R (the last group of each part may be narrower)."""
+    g = [(a, min(a + FP8_GROUP, d_c)) for a in range(0, d_c, FP8_GROUP)]
+    g += [(d_c + a, d_c + min(a + FP8_GROUP, d_r)) for a in range(0, d_r, FP8_GROUP)]
+    return g
+
+
+def quantize_rows_fp8(rows, d_c: int, d_r: int):
+    """Quantise cached rows [n, d_c + d_r]: per row and group, sigma = amax / 448
+    and codes E4M3(x / sigma), with x, the maximum and both divisions in float32.
+    Returns (codes uint8 [n, d_c + d_r], scales float32 [n, groups])."""
+    x = np.asarray(rows, dtype=np.float32)
+    x = x.reshape(-1, d_c + d_r)
+    groups = fp8_groups(d_c, d_r)
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    scales = np.zeros((x.shape[0], len(groups)), dtype=np.float32)
+    for gi, (a, b) in enumerate(groups):
+        blk = x[:, a:b]
+        amax = np.max(np.abs(blk), axis=1)
+        sigma = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+        nz = sigma > 0
+        q = blk[nz] / sigma[nz][:, None]
+        codes[nz, a:b] = e4m3_encode(q.astype(np.float32))
+        scales[:, gi] = sigma
+    return codes, scales
+
+
+def dequantize_rows_fp8(codes, scales, d_c: int, d_r: int) -> np.ndarray:
+    """Stored values of FP8 rows: code * sigma of the element's group (float64)."""
+    c = np.asarray(codes, dtype=np.uint8).reshape(-1, d_c + d_r)
+    sc = np.asarray(scales, dtype=np.float32).reshape(c.shape[0], -1).astype(F64)
+    out = e4m3_decode(c)
+    for gi, (a, b) in enumerate(fp8_groups(d_c, d_r)):
+        out[:, a:b] *= sc[:, gi:gi + 1]
+    return out
 
 
 # ----------------------------------------------------------------------------

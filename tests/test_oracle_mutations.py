@@ -75,6 +75,36 @@ def _temperature_not_squared(base):
     return 1.0 if spec.factor <= 1.0 else spec.mscale_coef * math.log(spec.factor) + 1.0
 
 
+_ORIG_ENCODE = O.e4m3_encode
+
+
+def _e4m3_truncating(v):
+    # rounds magnitudes toward zero instead of to nearest even
+    x = np.asarray(v, np.float32).astype(np.float64)
+    a = np.abs(x)
+    e = np.maximum(np.frexp(np.where(a > 0, a, 1.0))[1] - 1, -6)
+    q = np.exp2((e - 3).astype(np.float64))
+    return _ORIG_ENCODE((np.sign(x) * np.floor(a / q) * q).astype(np.float32))
+
+
+def _groups_across_parts(d_c, d_r):
+    # 128-channel groups over the whole row, mixing c^KV and k^R
+    D = d_c + d_r
+    return [(a, min(a + 128, D)) for a in range(0, D, 128)]
+
+
+def _quantize_with_e5m2_max(rows, d_c, d_r):
+    # scale from the other FP8 format's largest value
+    x = np.asarray(rows, np.float32).reshape(-1, d_c + d_r)
+    codes, sc = np.zeros(x.shape, np.uint8), np.zeros((x.shape[0], len(O.fp8_groups(d_c, d_r))), np.float32)
+    for gi, (a, b) in enumerate(O.fp8_groups(d_c, d_r)):
+        sig = (np.abs(x[:, a:b]).max(axis=1) / np.float32(57344.0)).astype(np.float32)
+        nz = sig > 0
+        codes[nz, a:b] = O.e4m3_encode(x[nz, a:b] / sig[nz][:, None])
+        sc[:, gi] = sig
+    return codes, sc
+
+
 MUTATIONS = [
     ("scale_without_rope_width", "softmax_scale", lambda d_h, d_r: 1.0 / math.sqrt(d_h),
      [P.test_two_token_softmax_closed_form]),
@@ -91,6 +121,12 @@ MUTATIONS = [
       lambda: P.test_yarn_absorbed_explicit_and_brute_force_agree(0.0707)]),
     ("yarn_temperature_not_squared", "attention_temperature", _temperature_not_squared,
      [lambda: P.test_yarn_absorbed_explicit_and_brute_force_agree(0.1)]),
+    ("e4m3_truncates", "e4m3_encode", _e4m3_truncating,
+     [P.test_e4m3_encode_matches_library_rounding, P.test_e4m3_encode_brute_force_nearest]),
+    ("fp8_groups_mix_parts", "fp8_groups", _groups_across_parts,
+     [P.test_fp8_groups_of_the_cached_row]),
+    ("fp8_scale_from_e5m2_max", "quantize_rows_fp8", _quantize_with_e5m2_max,
+     [P.test_fp8_quantize_rows_invariants]),
 ]
 
 

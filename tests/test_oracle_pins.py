@@ -391,3 +391,119 @@ def test_yarn_absorbed_explicit_and_brute_force_agree(coef):
     assert _rel(res["o"], bf_o) <= 1e-12
     assert _rel(o_ex, bf_o) <= 1e-12
     assert np.allclose(res["lse"], bf_lse, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) latent cache
+# --------------------------------------------------------------------------
+
+def _torch_e4m3():
+    torch = pytest.importorskip("torch")
+    return torch, torch.float8_e4m3fn
+
+
+def test_e4m3_decode_matches_library_for_every_code():
+    torch, f8 = _torch_e4m3()
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(f8).float().numpy().astype(np.float64)
+    mine = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    assert np.isnan(mine).sum() == 2                      # S.1111.111 only; no infinities
+    fin = ~np.isnan(ref)
+    assert np.array_equal(mine[fin], ref[fin])
+
+
+def test_e4m3_format_values():
+    # the format's defining values: largest finite 448 = 0.1111.110, 1 = 0.0111.000,
+    # smallest normal 2^-6 = 0.0001.000, smallest subnormal 2^-9 = 0.0000.001
+    enc = lambda x: int(O.e4m3_encode(np.float32(x)))
+    assert enc(448.0) == 0x7E and enc(-448.0) == 0xFE
+    assert enc(1.0) == 0x38 and enc(-2.0) == 0xC0
+    assert enc(2.0 ** -6) == 0x08 and enc(2.0 ** -9) == 0x01
+    assert enc(0.0) == 0x00 and enc(2.0 ** -11) == 0x00   # below half the smallest subnormal
+    # finite values past the largest code saturate
+    assert all(enc(x) == 0x7E for x in (449.0, 463.9, 464.0, 1e4, 3e38))
+
+
+def test_e4m3_encode_matches_library_rounding():
+    torch, f8 = _torch_e4m3()
+    rng = np.random.default_rng(7)
+    finite = O.e4m3_decode(np.arange(256, dtype=np.uint8))
+    finite = finite[~np.isnan(finite)]
+    pos = np.unique(finite[finite > 0])
+    mids = (pos[:-1] + pos[1:]) / 2                        # ties: must go to the even code
+    near = np.concatenate([np.nextafter(mids.astype(np.float32), np.float32(0)),
+                           np.nextafter(mids.astype(np.float32), np.float32(1e9))])
+    v = np.concatenate([finite, mids, -mids, near, rng.uniform(-448, 448, 20000),
+                        rng.uniform(-0.03, 0.03, 20000), rng.standard_normal(20000)]).astype(np.float32)
+    ref = torch.from_numpy(v.copy()).to(f8).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(v), ref)
+
+
+def test_e4m3_encode_brute_force_nearest():
+    # exhaustive nearest-code search over the finite codes, ties to the even mantissa
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = O.e4m3_decode(codes)
+    rng = np.random.default_rng(3)
+    xs = np.concatenate([rng.uniform(-460, 460, 300), rng.uniform(-0.02, 0.02, 300)]).astype(np.float32)
+    for x in xs:
+        xv = float(x)
+        if abs(xv) >= 448.0:
+            want = 0x7E | (0x80 if xv < 0 else 0)
+        else:
+            d = [abs(xv - float(v)) for v in vals]
+            best = min(d)
+            cand = [int(codes[i]) for i in range(len(codes)) if d[i] == best]
+            if len(cand) > 1:
+                cand = [c for c in cand if c & 1 == 0] or cand
+                # +0 and -0 tie at zero: the sign of x decides
+                cand = [c for c in cand if (c & 0x80) == (0x80 if np.signbit(x) else 0)] or cand
+            want = cand[0]
+        assert int(O.e4m3_encode(x)) == want, (xv, hex(int(O.e4m3_encode(x))), hex(want))
+
+
+def test_fp8_groups_of_the_cached_row():
+    # V2 shapes: four 128-channel groups over c^KV and one over the 64-wide k^R
+    assert O.fp8_groups(512, 64) == [(0, 128), (128, 256), (256, 384), (384, 512), (512, 576)]
+    assert O.fp8_groups(128, 16) == [(0, 128), (128, 144)]
+    assert O.fp8_groups(200, 16) == [(0, 128), (128, 200), (200, 216)]
+
+
+def test_fp8_quantize_rows_invariants():
+    rng = np.random.default_rng(11)
+    d_c, d_r = 512, 64
+    rows = rng.standard_normal((40, d_c + d_r)).astype(np.float32)
+    rows[3, :128] = 0.0                                      # an all-zero group
+    rows[5, 200] = 300.0                                     # an outlier confined to its group
+    rows[7, 512:] *= 1e-3                                    # a small rotary group
+    codes, sc = O.quantize_rows_fp8(rows, d_c, d_r)
+    assert codes.dtype == np.uint8 and codes.shape == rows.shape and sc.shape == (40, 5)
+    deq = O.dequantize_rows_fp8(codes, sc, d_c, d_r)
+    for gi, (a, b) in enumerate(O.fp8_groups(d_c, d_r)):
+        blk = rows[:, a:b].astype(np.float64)
+        amax = np.abs(blk).max(axis=1)
+        # scale = amax / 448 in float32
+        assert np.array_equal(sc[:, gi], (np.abs(rows[:, a:b]).max(axis=1) / np.float32(448)).astype(np.float32))
+        # the group's largest element is stored as +-448 sigma, i.e. amax itself
+        k = np.abs(blk).argmax(axis=1)
+        got = np.abs(deq[np.arange(40), a + k])
+        assert np.allclose(got, amax, rtol=2 ** -22, atol=0)
+        # error bound from the format's spacing: half a step, 2^-4 relative for
+        # normals, 2^-10 sigma for subnormals
+        err = np.abs(deq[:, a:b] - blk)
+        bound = 2.0 ** -4 * np.abs(blk) + 2.0 ** -10 * sc[:, gi:gi + 1].astype(np.float64)
+        assert np.all(err <= bound * (1 + 1e-6))
+    assert np.all(codes[3, :128] == 0) and sc[3, 0] == 0.0
+    # the outlier's group alone carries a large scale
+    assert sc[5, 1] > 100 * np.median(sc[:, 1]) and sc[5, 0] < 2 * np.median(sc[:, 0])
+
+
+def test_fp8_quantize_is_scale_invariant_under_powers_of_two():
+    # multiplying a row by 2^k is exact in float32: same codes, scales times 2^k
+    rng = np.random.default_rng(5)
+    rows = rng.standard_normal((16, 144)).astype(np.float32)
+    c0, s0 = O.quantize_rows_fp8(rows, 128, 16)
+    for k in (-20, -3, 5, 30):
+        ck, sk = O.quantize_rows_fp8(rows * np.float32(2.0 ** k), 128, 16)
+        assert np.array_equal(ck, c0)
+        assert np.array_equal(sk, (s0 * np.float32(2.0 ** k)).astype(np.float32))
