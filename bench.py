@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-query-proj", action="store_true",
                     help="skip the separate timing of the query projection")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the separate timing of attention over an FP8 cache")
     return ap.parse_args()
 
 
@@ -277,6 +279,81 @@ def run_reference(args):
 # GPU arm
 # ----------------------------------------------------------------------------
 
+FP8_WORKLOAD = "v2lite_b4_ctx128k"
+
+
+def measure_fp8(M, dev, steps, seed):
+    """Attention over the same latent cache stored in bf16 and in FP8 (E4M3
+    codes + one float32 scale per token and 128-channel group), on the
+    V2-Lite 128K workload (16 heads, 4 x 131072 tokens: 604 MB in bf16,
+    312 MB in FP8, both larger than L2).  The FP8 cache is quantised from the
+    bf16 one by the library.  Returns the mean CUDA-event time of each
+    attention call (split plan included) and the bytes each one must read."""
+    import torch
+    from workloads import WORKLOADS
+    wl = WORKLOADS[FP8_WORKLOAD]
+    B, H, D, d = wl.B, wl.n_h, wl.D, wl.d_model
+    ctx = np.asarray(wl.ctx, dtype=np.int64)
+    cap = int(ctx.max())
+    cfg = M.mla_config(n_h=H, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, d_model=d, page_size=0,
+                       rope_base=wl.rope_base, dtype=M.MLA_BF16)
+    handle = M.mla_create(cfg)
+    try:
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        bf = torch.bfloat16
+
+        def randn(*shape, std=1.0):
+            return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(bf)
+
+        w_dkv = randn(wl.d_c, d, std=d ** -0.5)
+        w_kr = randn(wl.d_r, d, std=d ** -0.5)
+        cache = torch.empty((B, cap, D), dtype=bf, device=dev)
+        chunk = 4096
+        for b in range(B):
+            for t0 in range(0, int(ctx[b]), chunk):
+                t1 = min(int(ctx[b]), t0 + chunk)
+                sp = torch.tensor([t0], dtype=torch.int32, device=dev)
+                M.mla_cache_append(handle, randn(t1 - t0, d), 1, t1 - t0, sp, w_dkv, w_kr,
+                                   cache.data_ptr() + 2 * b * cap * D, cap)
+        G = M.mla_fp8_scale_groups(handle)
+        codes = torch.empty((B, cap, D), dtype=torch.uint8, device=dev)
+        scales = torch.empty((B, cap, G), dtype=torch.float32, device=dev)
+        M.mla_quantize_rows_fp8(handle, cache, B * cap, codes, scales)
+        q_abs = randn(B, H, D, std=0.5)
+        ctx_d = torch.from_numpy(ctx.astype(np.int32)).to(dev)
+        P = M.mla_default_num_parts(handle)
+        ws_bytes = M.mla_decode_workspace_size(handle, B, P)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        stream = torch.cuda.current_stream()
+        sh = stream.cuda_stream
+
+        def timed(call):
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+            for e in ev:
+                e[0].record(stream)
+                call()
+                e[1].record(stream)
+            torch.cuda.synchronize()
+            return float(np.mean([e[0].elapsed_time(e[1]) for e in ev])) * 1e3
+
+        us_bf16 = timed(lambda: M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, ctx_d, B, P,
+                                                  ws, ws_bytes, sh))
+        us_fp8 = timed(lambda: M.mla_decode_attn_fp8(handle, q_abs, codes, scales, cap, None, 0,
+                                                     ctx_d, B, P, ws, ws_bytes, sh))
+        st = M.mla_get_device_status(handle, sh)
+        if st != M.MLA_OK:
+            raise M.MlaError(st, "device status after the FP8 timing")
+    finally:
+        M.mla_destroy(handle)
+    tokens = int(ctx.sum())
+    return {"workload": FP8_WORKLOAD, "tokens": tokens, "bf16_us": us_bf16, "fp8_us": us_fp8,
+            "bf16_bytes": tokens * D * 2, "fp8_bytes": tokens * (D + 4 * G)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -481,6 +558,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
+    # ---- attention over an FP8 cache (a separate workload, rank 0 only)
+    fp8 = None
+    if not args.no_fp8 and rank == 0:
+        fp8 = measure_fp8(M, dev, args.steps, rank_seed(rank) + 17)
+
     # ---- reduce over ranks: max time
     ms, attn_ms, e2e_ms = reduce_max_over_ranks([ms, attn_ms, e2e_ms], world, dev)
     if world > 1:
@@ -529,6 +611,17 @@ def run_ours(args):
         "clocks": clk,
         "cpu_baseline": cpu,
     }
+    if fp8 is not None:
+        fp8_gbs = fp8["fp8_bytes"] / (fp8["fp8_us"] * 1e-6) / 1e9
+        bf16_gbs = fp8["bf16_bytes"] / (fp8["bf16_us"] * 1e-6) / 1e9
+        line["fp8_kv"] = {
+            "workload": fp8["workload"], "tokens": fp8["tokens"],
+            "fp8_attn_us": fp8["fp8_us"], "bf16_attn_us": fp8["bf16_us"],
+            "speedup": fp8["bf16_us"] / fp8["fp8_us"],
+            "fp8_algorithmic_bytes": fp8["fp8_bytes"], "fp8_achieved_gbs": fp8_gbs,
+            "fp8_frac": fp8_gbs / hbm_peak, "bf16_achieved_gbs": bf16_gbs,
+            "bf16_frac": bf16_gbs / hbm_peak, "bound": "hbm",
+            "note": "mla_decode_attn_fp8 vs mla_decode_attn on the same cache; not part of the step"}
     if qproj is not None:
         gbs = qproj["bytes"] / (qproj["us"] * 1e-6) / 1e9
         line["query_proj"] = {

@@ -32,6 +32,8 @@ EXPORTED = (
     "mla_query_proj",
     "mla_get_device_status", "mla_plan_pieces", "mla_decode_attn_combine_noalloc",
     "mla_noalloc_scratch_bytes", "mla_set_rope_scaling",
+    "mla_fp8_scale_groups", "mla_cache_append_fp8_workspace_size", "mla_cache_append_fp8",
+    "mla_quantize_rows_fp8", "mla_decode_attn_fp8",
 )
 
 
@@ -79,6 +81,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_noalloc_scratch_bytes": (sz, []),
         "mla_set_rope_scaling": (i, [vp, ctypes.c_double, i, ctypes.c_double, ctypes.c_double,
                                      ctypes.c_double]),
+        "mla_fp8_scale_groups": (i, [vp]),
+        "mla_cache_append_fp8_workspace_size": (sz, [vp, i, i]),
+        "mla_cache_append_fp8": (i, [vp, vp, i, i, vp, vp, vp, vp, vp, ll, vp, i, vp, sz, vp]),
+        "mla_quantize_rows_fp8": (i, [vp, vp, ll, vp, vp, vp]),
+        "mla_decode_attn_fp8": (i, [vp, vp, vp, vp, ll, vp, i, vp, i, i, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -165,6 +172,35 @@ def mla_decode_workspace_size(handle, B, num_parts=0) -> int:
 
 def mla_default_num_parts(handle) -> int:
     return load().mla_default_num_parts(handle)
+
+
+def mla_fp8_scale_groups(handle):
+    return load().mla_fp8_scale_groups(handle)
+
+
+def mla_cache_append_fp8_workspace_size(handle, B, T):
+    return load().mla_cache_append_fp8_workspace_size(handle, B, T)
+
+
+def mla_cache_append_fp8(handle, h, B, T, start_pos, w_dkv, w_kr, cache, kv_scale, cache_len,
+                         block_table, max_blocks_per_seq, workspace, ws_bytes, stream=None):
+    _check(load().mla_cache_append_fp8(handle, _ptr(h), B, T, _ptr(start_pos), _ptr(w_dkv),
+                                       _ptr(w_kr), _ptr(cache), _ptr(kv_scale), cache_len,
+                                       _ptr(block_table), max_blocks_per_seq, _ptr(workspace),
+                                       ws_bytes, _stream(stream)), "mla_cache_append_fp8")
+
+
+def mla_quantize_rows_fp8(handle, rows, n_rows, codes, kv_scale, stream=None):
+    _check(load().mla_quantize_rows_fp8(handle, _ptr(rows), n_rows, _ptr(codes), _ptr(kv_scale),
+                                        _stream(stream)), "mla_quantize_rows_fp8")
+
+
+def mla_decode_attn_fp8(handle, q_abs, cache, kv_scale, cache_len, block_table, max_blocks_per_seq,
+                        ctx_len, B, num_parts, workspace, ws_bytes, stream=None):
+    _check(load().mla_decode_attn_fp8(handle, _ptr(q_abs), _ptr(cache), _ptr(kv_scale), cache_len,
+                                      _ptr(block_table), max_blocks_per_seq, _ptr(ctx_len), B,
+                                      num_parts, _ptr(workspace), ws_bytes, _stream(stream)),
+           "mla_decode_attn_fp8")
 
 
 def mla_decode_attn(handle, q_abs, cache, cache_len, block_table, max_blocks_per_seq, ctx_len, B,

@@ -192,9 +192,12 @@ size_t mla_decode_workspace_size(const mla_handle *h, int B, int num_parts) {
   return ws_layout(h->cfg, B, P).total;
 }
 
-int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long long cache_len,
-                    const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
-                    int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
+namespace {
+// Decode attention over a cache in cfg.dtype (kv_scale NULL) or of FP8 codes
+// with their group scales.
+int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float *kv_scale,
+                long long cache_len, const int *block_table, int max_blocks_per_seq, const int *ctx_len,
+                int B, int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
   if (!h || B < 0 || num_parts < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if (!q_abs || !cache || !ctx_len) return MLA_ERR_INVALID_ARG;
@@ -220,15 +223,82 @@ int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long lo
   a.d_c = c.d_c;
   a.d_r = c.d_r;
   a.scale_log2 = (float)(1.4426950408889634 * h->score_mult / sqrt((double)(c.d_h + c.d_r)));
+  a.kv_scale = kv_scale;
+  a.n_groups = fp8_num_groups(c.d_c, c.d_r);
   a.ws = (char *)workspace;
   a.L = L;
   a.status = h->d_status;
   e = cudaErrorNotSupported;
-  if (h->attn_kind == kAttnTcPair && aligned16(q_abs) && aligned16(cache))
+  if (h->attn_kind == kAttnTcPair && !kv_scale && aligned16(q_abs) && aligned16(cache))
     e = launch_attn_tc_pair(a, P, s);
   else if (h->attn_kind == kAttnTcSmallH && aligned16(q_abs) && aligned16(cache))
     e = launch_attn_tc_smallh(a, P, s);
   if (e == cudaErrorNotSupported) e = launch_attn_simt(a, P, c.dtype == MLA_FP32, s);
+  if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+}  // namespace
+
+int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long long cache_len,
+                    const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
+                    int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
+  return decode_attn(h, q_abs, cache, nullptr, cache_len, block_table, max_blocks_per_seq, ctx_len, B,
+                     num_parts, workspace, ws_bytes, stream);
+}
+
+int mla_decode_attn_fp8(mla_handle *h, const void *q_abs, const void *cache, const float *kv_scale,
+                        long long cache_len, const int *block_table, int max_blocks_per_seq,
+                        const int *ctx_len, int B, int num_parts, void *workspace, size_t ws_bytes,
+                        mla_stream_t stream) {
+  if (!kv_scale && h && B > 0) return MLA_ERR_INVALID_ARG;
+  return decode_attn(h, q_abs, cache, kv_scale, cache_len, block_table, max_blocks_per_seq, ctx_len, B,
+                     num_parts, workspace, ws_bytes, stream);
+}
+
+int mla_fp8_scale_groups(const mla_handle *h) { return h ? fp8_num_groups(h->cfg.d_c, h->cfg.d_r) : 0; }
+
+size_t mla_cache_append_fp8_workspace_size(const mla_handle *h, int B, int T) {
+  if (!h || B < 0 || T < 0) return 0;
+  const size_t n = (size_t)B * (size_t)T * (size_t)(h->cfg.d_c + h->cfg.d_r) * sizeof(float);
+  return align_up(n > 0 ? n : 1, 256);
+}
+
+int mla_cache_append_fp8(mla_handle *h, const void *x, int B, int T, const int *start_pos,
+                         const void *w_dkv, const void *w_kr, void *cache, float *kv_scale,
+                         long long cache_len, const int *block_table, int max_blocks_per_seq,
+                         void *workspace, size_t ws_bytes, mla_stream_t stream) {
+  if (!h || B < 0 || T < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MLA_OK;
+  if (!x || !start_pos || !w_dkv || !w_kr || !cache || !kv_scale) return MLA_ERR_INVALID_ARG;
+  const mla_config &c = h->cfg;
+  if (c.page_size > 0 && (!block_table || max_blocks_per_seq <= 0)) return MLA_ERR_INVALID_ARG;
+  if (c.page_size == 0 && block_table) return MLA_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < mla_cache_append_fp8_workspace_size(h, B, T))
+    return MLA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  float *rows = (float *)workspace;
+  cudaError_t e = cudaErrorNotSupported;
+  if (h->gemm_kind == kGemmTc)
+    e = launch_append_tc(c, x, B, T, start_pos, w_dkv, w_kr, nullptr, 0, nullptr, 0, h->d_theta,
+                         h->d_status, s, rows);
+  if (e == cudaErrorNotSupported)
+    e = launch_append_simt(c, x, B, T, start_pos, w_dkv, w_kr, nullptr, 0, nullptr, 0, h->d_theta,
+                           h->d_status, s, rows);
+  if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return from_cuda(e);
+  e = launch_quantize_fp8(c, rows, true, (long long)B * T, T, start_pos, (uint8_t *)cache, kv_scale,
+                          cache_len, block_table, max_blocks_per_seq, h->d_status, s);
+  if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+int mla_quantize_rows_fp8(mla_handle *h, const void *rows, long long n_rows, void *codes, float *kv_scale,
+                          mla_stream_t stream) {
+  if (!h || n_rows < 0) return MLA_ERR_INVALID_ARG;
+  if (n_rows == 0) return MLA_OK;
+  if (!rows || !codes || !kv_scale) return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_quantize_fp8(h->cfg, rows, false, n_rows, 1, nullptr, (uint8_t *)codes,
+                                            kv_scale, 0, nullptr, 0, h->d_status, (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
   return from_cuda(e);
 }

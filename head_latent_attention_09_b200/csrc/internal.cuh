@@ -14,6 +14,12 @@ namespace mla {
 // tiles, and the paged fast paths require page_size == kTile.
 constexpr int kTile = 64;
 
+// FP8 latent cache: channels per scale group (over c^KV, then over k^R).
+constexpr int kFp8Group = 128;
+__host__ __device__ inline int fp8_num_groups(int d_c, int d_r) {
+  return (d_c + kFp8Group - 1) / kFp8Group + (d_r + kFp8Group - 1) / kFp8Group;
+}
+
 // Bits of the device status word.
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBounds = 2u;
@@ -146,6 +152,10 @@ struct AttnArgs {
   int B;
   int n_h, d_c, d_r;
   float scale_log2;  // log2(e) / sqrt(d_h + d_r)
+  // FP8 cache: the rows are E4M3 codes and kv_scale [rows, n_groups] holds
+  // each row's group scales; NULL for a cache in cfg.dtype
+  const float *kv_scale;
+  int n_groups;
   char *ws;
   WsLayout L;
   unsigned *status;
@@ -165,7 +175,15 @@ cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int 
                                const int *start_pos, const void *w_dkv, const void *w_kr,
                                void *cache, long long cache_len, const int *block_table,
                                int max_blocks, const double *theta, unsigned *status,
-                               cudaStream_t s);
+                               cudaStream_t s, float *rows_out = nullptr);
+// FP8 E4M3 quantisation of n_rows rows [n_rows, d_c + d_r] (cfg.dtype, or
+// float32 when src_f32): per row and 128-channel group, sigma = amax / 448 and
+// codes E4M3(x / sigma).  With start_pos, row r is token r % T of sequence
+// r / T and goes to its cache row (bounds flagged); without, to row r.
+cudaError_t launch_quantize_fp8(const mla_config &cfg, const void *src, bool src_f32, long long n_rows,
+                                int T, const int *start_pos, uint8_t *codes, float *scales,
+                                long long cache_len, const int *block_table, int max_blocks,
+                                unsigned *status, cudaStream_t s);
 cudaError_t launch_absorb_simt(const mla_config &cfg, const void *q_nope, const void *q_rope,
                                const int *pos, const void *w_uk, void *q_abs, int B,
                                const double *theta, cudaStream_t s);
@@ -178,11 +196,13 @@ cudaError_t launch_linear_simt(const void *x, const void *w, void *y, int M, int
                                cudaStream_t s);
 
 // tcgen05 paths (bf16 only); return cudaErrorNotSupported for shapes they lack.
+// With rows_out set, the rotated rows go to rows_out [B*T, d_c + d_r] in
+// float32 instead of to the cache (the cache arguments are then unused).
 cudaError_t launch_append_tc(const mla_config &cfg, const void *h, int B, int T,
                              const int *start_pos, const void *w_dkv, const void *w_kr,
                              void *cache, long long cache_len, const int *block_table,
                              int max_blocks, const double *theta, unsigned *status,
-                             cudaStream_t s);
+                             cudaStream_t s, float *rows_out = nullptr);
 cudaError_t launch_absorb_tc(const mla_config &cfg, const void *q_nope, const void *q_rope,
                              const int *pos, const void *w_uk, void *q_abs, int B,
                              const double *theta, cudaStream_t s);

@@ -360,5 +360,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 // rejects the map.
 bool encode_map_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                      const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz);
+// The same for a byte tensor (FP8 codes).
+bool encode_map_u8(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                   const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz);
 
 }  // namespace mla

@@ -2,6 +2,7 @@
 // (any shape, fp32 or bf16) versions of append / absorb / attention /
 // output projection.  The fp32 configuration runs entirely here; bf16 shapes
 // with a tensor-core kernel use those instead (see api.cu).
+#include <cuda_fp8.h>
 #include <math_constants.h>
 
 #include "internal.cuh"
@@ -119,7 +120,18 @@ constexpr int kSimtMaxC = 512;      // d_c
 constexpr int kQPerLane = kSimtMaxD / 32;
 constexpr int kOPerLane = kSimtMaxC / 32;
 
-template <typename T>
+__device__ __forceinline__ float e4m3_value(uint8_t c) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3)));
+}
+
+// Group of channel f of a cached row (see fp8_group_range).
+__device__ __forceinline__ int fp8_group_of(int f, int d_c) {
+  return f < d_c ? f / kFp8Group : (d_c + kFp8Group - 1) / kFp8Group + (f - d_c) / kFp8Group;
+}
+
+// T: element type of the query; F8: the cache holds E4M3 codes with group
+// scales (else elements of type T).
+template <typename T, bool F8>
 __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
   const WsHeader *hd = reinterpret_cast<const WsHeader *>(a.ws);
   const long long P = hd->P, Ttot = hd->Ttot;
@@ -134,6 +146,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
   float *opart = reinterpret_cast<float *>(a.ws + a.L.opart_off);
   float *lse = reinterpret_cast<float *>(a.ws + a.L.lse_off);
   const T *cache = reinterpret_cast<const T *>(a.cache);
+  const uint8_t *cache8 = reinterpret_cast<const uint8_t *>(a.cache);
   const T *qg = reinterpret_cast<const T *>(a.q_abs);
 
   const long long t0 = plan_begin(w, P, Ttot), t1 = plan_begin(w + 1, P, Ttot);
@@ -173,13 +186,19 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
         if (lane == 0) atomicOr(a.status, kStatusBounds);
         continue;
       }
-      const T *r = cache + row * D;
-      float part = 0.f;
+      float val[kQPerLane];
 #pragma unroll
       for (int j = 0; j < kQPerLane; ++j) {
         const int f = lane + 32 * j;
-        if (f < D) part += q[j] * to_f(r[f]);
+        val[j] = 0.f;
+        if (f < D) {
+          if (F8) val[j] = e4m3_value(cache8[row * D + f]) * a.kv_scale[row * a.n_groups + fp8_group_of(f, a.d_c)];
+          else val[j] = to_f(cache[row * D + f]);
+        }
       }
+      float part = 0.f;
+#pragma unroll
+      for (int j = 0; j < kQPerLane; ++j) part += q[j] * val[j];
       const float s = warp_sum(part) * a.scale_log2;   // score in log2 units
       const float m_new = fmaxf(m, s);
       const float corr = exp2f(m - m_new);
@@ -188,7 +207,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
 #pragma unroll
       for (int j = 0; j < kOPerLane; ++j) {
         const int f = lane + 32 * j;
-        if (f < a.d_c) o[j] = o[j] * corr + pr * to_f(r[f]);
+        if (f < a.d_c) o[j] = o[j] * corr + pr * val[j];
       }
       m = m_new;
     }
@@ -244,7 +263,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) append_simt_kernel(
     const T *h, int T_new, int d, int d_c, int d_r, const int *start_pos, const T *w_dkv,
     const T *w_kr, T *cache, long long cache_len, const int *block_table, int max_blocks,
-    int page_size, const double *theta, unsigned *status) {
+    int page_size, const double *theta, unsigned *status, float *rows_out) {
   extern __shared__ float sh[];
   const long long tok = blockIdx.x;
   const int b = (int)(tok / T_new), t = (int)(tok % T_new);
@@ -273,6 +292,11 @@ __global__ void __launch_bounds__(256) append_simt_kernel(
     a0 = r0;
     a1 = r1;
   }
+  if (rows_out) {
+    rows_out[tok * D + f0] = a0;
+    rows_out[tok * D + f0 + 1] = a1;
+    return;
+  }
   const long long row = cache_row(b, p, cache_len, block_table, max_blocks, page_size);
   if (row < 0) {
     atomicOr(status, kStatusBounds);
@@ -280,6 +304,63 @@ __global__ void __launch_bounds__(256) append_simt_kernel(
   }
   cache[row * D + f0] = from_f<T>(a0);
   cache[row * D + f0 + 1] = from_f<T>(a1);
+}
+
+// ---------------------------------------------------------------------------
+// FP8 E4M3 quantisation of cached rows: one warp per row; per 128-channel
+// group (over c^KV, then over k^R) sigma = amax / 448 and the codes of
+// x / sigma, both divisions rounded to nearest in float32, the conversion
+// rounding to nearest even and saturating at 448.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ void fp8_group_range(int g, int d_c, int d_r, int &a, int &e) {
+  const int gc = (d_c + kFp8Group - 1) / kFp8Group;
+  if (g < gc) {
+    a = g * kFp8Group;
+    e = min(a + kFp8Group, d_c);
+  } else {
+    a = d_c + (g - gc) * kFp8Group;
+    e = min(a + kFp8Group, d_c + d_r);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_fp8_kernel(
+    const T *src, long long n_rows, int d_c, int d_r, int T_new, const int *start_pos,
+    uint8_t *codes, float *scales, long long cache_len, const int *block_table, int max_blocks,
+    int page_size, unsigned *status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (r >= n_rows) return;
+  long long dst = r;
+  if (start_pos) {
+    const int b = (int)(r / T_new), t = (int)(r % T_new);
+    dst = cache_row(b, (long long)start_pos[b] + t, cache_len, block_table, max_blocks, page_size);
+    if (dst < 0) {
+      if (lane == 0) atomicOr(status, kStatusBounds);
+      return;
+    }
+  }
+  const int D = d_c + d_r, G = fp8_num_groups(d_c, d_r);
+  const T *x = src + r * D;
+  uint8_t *out = codes + dst * D;
+  for (int g = 0; g < G; ++g) {
+    int a, e;
+    fp8_group_range(g, d_c, d_r, a, e);
+    float amax = 0.f;
+    for (int f = a + lane; f < e; f += 32) amax = fmaxf(amax, fabsf(to_f(x[f])));
+    amax = warp_max(amax);
+    const float sigma = __fdiv_rn(amax, 448.f);
+    for (int f = a + lane; f < e; f += 32)
+      out[f] = sigma > 0.f ? (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(to_f(x[f]), sigma), __NV_SATFINITE, __NV_E4M3)
+                           : (uint8_t)0;
+    if (lane == 0) scales[dst * G + g] = sigma;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -358,8 +439,11 @@ cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s
   if (a.d_c + a.d_r > kSimtMaxD || a.d_c > kSimtMaxC) return cudaErrorNotSupported;
   const int warps = a.n_h < 8 ? a.n_h : 8;
   dim3 grid(P, (a.n_h + warps - 1) / warps);
-  if (fp32) attn_simt_kernel<float><<<grid, warps * 32, 0, s>>>(a);
-  else attn_simt_kernel<__nv_bfloat16><<<grid, warps * 32, 0, s>>>(a);
+  const bool f8 = a.kv_scale != nullptr;
+  if (fp32 && f8) attn_simt_kernel<float, true><<<grid, warps * 32, 0, s>>>(a);
+  else if (fp32) attn_simt_kernel<float, false><<<grid, warps * 32, 0, s>>>(a);
+  else if (f8) attn_simt_kernel<__nv_bfloat16, true><<<grid, warps * 32, 0, s>>>(a);
+  else attn_simt_kernel<__nv_bfloat16, false><<<grid, warps * 32, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -463,7 +547,7 @@ cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int 
                                const int *start_pos, const void *w_dkv, const void *w_kr,
                                void *cache, long long cache_len, const int *block_table,
                                int max_blocks, const double *theta, unsigned *status,
-                               cudaStream_t s) {
+                               cudaStream_t s, float *rows_out) {
   const int D = cfg.d_c + cfg.d_r;
   dim3 grid((unsigned)((long long)B * T), (D / 2 + 7) / 8);
   const size_t smem = sizeof(float) * cfg.d_model;
@@ -472,12 +556,30 @@ cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int 
     append_simt_kernel<float><<<grid, 256, smem, s>>>(
         (const float *)h, T, cfg.d_model, cfg.d_c, cfg.d_r, start_pos, (const float *)w_dkv,
         (const float *)w_kr, (float *)cache, cache_len, block_table, max_blocks, cfg.page_size,
-        theta, status);
+        theta, status, rows_out);
   else
     append_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
         (const __nv_bfloat16 *)h, T, cfg.d_model, cfg.d_c, cfg.d_r, start_pos,
         (const __nv_bfloat16 *)w_dkv, (const __nv_bfloat16 *)w_kr, (__nv_bfloat16 *)cache,
-        cache_len, block_table, max_blocks, cfg.page_size, theta, status);
+        cache_len, block_table, max_blocks, cfg.page_size, theta, status, rows_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_fp8(const mla_config &cfg, const void *src, bool src_f32, long long n_rows,
+                                int T, const int *start_pos, uint8_t *codes, float *scales,
+                                long long cache_len, const int *block_table, int max_blocks,
+                                unsigned *status, cudaStream_t s) {
+  if (n_rows <= 0) return cudaSuccess;
+  const long long blocks = (n_rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return cudaErrorNotSupported;
+  if (src_f32 || cfg.dtype == MLA_FP32)
+    quantize_fp8_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(
+        (const float *)src, n_rows, cfg.d_c, cfg.d_r, T, start_pos, codes, scales, cache_len,
+        block_table, max_blocks, cfg.page_size, status);
+  else
+    quantize_fp8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+        (const __nv_bfloat16 *)src, n_rows, cfg.d_c, cfg.d_r, T, start_pos, codes, scales, cache_len,
+        block_table, max_blocks, cfg.page_size, status);
   return cudaGetLastError();
 }
 

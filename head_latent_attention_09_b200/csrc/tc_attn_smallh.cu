@@ -15,6 +15,14 @@
 //
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 tensor-memory
 // allocation and MMA issue, warps 2-5 softmax / rescale / epilogue.
+//
+// FP8 cache (E4M3 codes, a float32 scale per token and 128-channel group):
+// the producer stages each 64 x 64 chunk of codes (4 KB) by TMA, and four
+// more warps (6-9) widen it into the bf16 ring slot the MMAs read, applying
+// the group scale on the way (code * sigma rounded to bf16).  HBM then
+// carries 576 B + 20 B of scales per token instead of 1152 B; the products,
+// the softmax and the epilogue are those of the bf16 cache.
+#include <cuda_fp8.h>
 #include <math_constants.h>
 
 #include "ptx.cuh"
@@ -22,31 +30,48 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kChunk = 8192;               // [64 rows x 128 B]
+constexpr int kChunk8 = 4096;              // FP8 staging: [64 rows x 64 B]
 constexpr int kTileTok = 64;
 constexpr float kRescale = 8.0f;
+constexpr int kGroups8 = 5;                // scale groups of a 576-wide row
 
-template <int H>
+template <int H, bool F8>
 struct Cfg {
-  static constexpr int kNS = H <= 16 ? 24 : 18;             // ring chunk slots
+  static constexpr int kThreads = F8 ? 320 : 192;
+  // Ring chunk slots.  A tile holds its nine slots until its P.V is done,
+  // which is issued after the next tile's S: at least two tiles' worth.
+  static constexpr int kNS = F8 ? 18 : (H <= 16 ? 24 : 18);
+  static constexpr int kNSt = F8 ? (H <= 16 ? 12 : 8) : 0;  // FP8 staging chunks
   static constexpr int kQ = 9 * H * 128;                    // H rows x 576
   static constexpr int kPT = H * 128;                       // P^T: H rows x 64 tokens
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = (kQ + 1023) / 1024 * 1024;
-  static constexpr int kOffP = kOffRing + kNS * kChunk;
+  static constexpr int kOffStage = kOffRing + kNS * kChunk;
+  static constexpr int kOffP = kOffStage + kNSt * kChunk8;
   static constexpr int kOffRed = kOffP + 2 * ((kPT + 1023) / 1024 * 1024);  // float [2][4][H] max, [4][H] sum
   static constexpr int kOffBar = kOffRed + 12 * H * 4;
   // barriers
   static constexpr int bFull = 0, bEmpty = kNS, bQFull = 2 * kNS, bQEmpty = bQFull + 1, bSFull = bQEmpty + 1,
                        bPFull = bSFull + 2, bPFree = bPFull + 2, bODone = bPFree + 2, bOFree = bODone + 2,
-                       bXchg = bOFree + 1, bLsum = bXchg + 2, kNumBars = bLsum + 1;
+                       bXchg = bOFree + 1, bLsum = bXchg + 2, bStFull = bLsum + 1, bStEmpty = bStFull + kNSt,
+                       kNumBars = bStEmpty + kNSt;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;
   static constexpr uint32_t kTmemCols = 10 * H <= 256 ? 256 : 512;  // S^T 2 x H, O^T 8 x H
   static constexpr uint32_t kColO = 2 * H;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
+
+// Two E4M3 codes (low byte first) times sigma, as a bf16 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two, float sigma) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  float2 f = __half22float2(__half2(hr));
+  f.x *= sigma;
+  f.y *= sigma;
+  const __nv_bfloat162 b = __float22bfloat162_rn(f);
+  return *reinterpret_cast<const uint32_t *>(&b);
+}
 
 struct Piece {
   int b;
@@ -119,17 +144,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
   return ok;
 }
 
-template <int H>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int H, bool F8>
+__global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
     attn_smallh_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapKV,
                        const AttnArgs a, const long long kv_rows) {
-  using C = Cfg<H>;
+  using C = Cfg<H, F8>;
   constexpr int NS = C::kNS;
+  constexpr int NSt = C::kNSt;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + C::kOffQ;
   uint8_t *sRing = sm + C::kOffRing;
   uint8_t *sP = sm + C::kOffP;
+  uint8_t *sStage = sm + C::kOffStage;
   constexpr int kPStride = (C::kPT + 1023) / 1024 * 1024;
   float *red_m = reinterpret_cast<float *>(sm + C::kOffRed);  // [2][4][H]
   float *red_s = red_m + 8 * H;                                // [4][H]
@@ -143,8 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      ptx::mbar_init(bar + C::bFull + s, 1);
+      ptx::mbar_init(bar + C::bFull + s, F8 ? 4 : 1);   // FP8: the four converter warps
       ptx::mbar_init(bar + C::bEmpty + s, 1);
+    }
+    for (int s = 0; s < NSt; ++s) {
+      ptx::mbar_init(bar + C::bStFull + s, 1);
+      ptx::mbar_init(bar + C::bStEmpty + s, 4);
     }
     ptx::mbar_init(bar + C::bQFull, 1);
     ptx::mbar_init(bar + C::bQEmpty, 1);
@@ -200,7 +231,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (r >= 0) y = (int)r;
           else if (lane == 0) atomicOr(a.status, kStatusBounds);
         }
-        for (int c = 0; c < 9; ++c) {
+        for (int c = 0; c < 9 && F8; ++c) {
+          // FP8: stage the 64 x 64 chunk of codes for the converter warps
+          const int s = sc % NSt;
+          if (sc >= NSt && !warp_wait(bar + C::bStEmpty + s, ((sc / NSt) - 1) & 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t *dst = sStage + s * kChunk8;
+          if (manual) {
+            for (int u = lane; u < 64 * 4; u += 32) {
+              const int row = u >> 2, cc = u & 3;
+              const int t = tok0 + row;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (t < pc.ctx) {
+                const long long r = kv_row(a, pc.b, t);
+                if (r >= 0)
+                  v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(a.cache) + r * 576 +
+                                                       64 * c + 16 * cc);
+                else
+                  atomicOr(a.status, kStatusBounds);
+              }
+              *reinterpret_cast<uint4 *>(dst + row * 64 + 16 * cc) = v;
+            }
+            ptx::fence_proxy_async_smem();   // later TMA writes to this slot come after these
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar + C::bStFull + s);
+          } else if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(bar + C::bStFull + s, kChunk8);
+            ptx::tma_load_2d(dst, &mapKV, bar + C::bStFull + s, 64 * c, y);
+          }
+          ++sc;
+        }
+        for (int c = 0; c < 9 && !F8; ++c) {
           const int s = sc % NS;
           if (sc >= NS && !warp_wait(bar + C::bEmpty + s, ((sc / NS) - 1) & 1, a.status, abort_flag)) {
             ok = false;
@@ -300,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && have_prev) pv(prev);
     }
-  } else {
+  } else if (warp < 6) {
     // --------------------------------------- softmax, rescale and epilogue
     // M = 64 accumulators live in lanes 0-15 of each 32-lane quarter: this
     // thread's token (S^T row) or latent column within a block (O^T row) is
@@ -473,6 +536,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ptx::mbar_arrive(bar + C::bOFree);
       ++npc;
     }
+  } else if (F8) {
+    // ------------------------------------------- FP8 converters (warps 6-9)
+    // Thread ct handles rows ct/4 and ct/4 + 32 of every chunk, 16 codes
+    // (unit ct%4 of the row's 64) each: 32 bytes of bf16, i.e. two 16-byte
+    // units of the 128-byte-swizzled ring row.
+    const int ct = (warp - 6) * 32 + lane;
+    const int r0 = ct >> 2, u = ct & 3;
+    Walk w;
+    walk_init(w, a, share);
+    Piece pc;
+    int sc = 0;
+    bool ok = true;
+    while (ok && walk_next(w, a, share, pc)) {
+      for (int k = 0; k < pc.ntiles && ok; ++k) {
+        const int tok0 = pc.tok_begin + kTileTok * k;
+        float sig[2][kGroups8];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int t = tok0 + r0 + 32 * rr;
+          const long long r = t < pc.ctx ? kv_row(a, pc.b, t) : -1;
+#pragma unroll
+          for (int g = 0; g < kGroups8; ++g) sig[rr][g] = r >= 0 ? a.kv_scale[r * kGroups8 + g] : 0.f;
+        }
+        for (int c = 0; c < 9; ++c) {
+          const int st = sc % NSt, s = sc % NS;
+          if (!warp_wait(bar + C::bStFull + st, (sc / NSt) & 1, a.status, abort_flag)) { ok = false; break; }
+          if (sc >= NS && !warp_wait(bar + C::bEmpty + s, ((sc / NS) - 1) & 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int g = c >> 1;   // chunks 0-7: c^KV groups 0-3; chunk 8: the k^R group
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int row = r0 + 32 * rr;
+            // select the group's scale without indexing the array at run time
+            float sg = sig[rr][0];
+#pragma unroll
+            for (int gg = 1; gg < kGroups8; ++gg) sg = g == gg ? sig[rr][gg] : sg;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(sStage + st * kChunk8 + row * 64 + 16 * u);
+            uint4 lo, hi;
+            lo.x = e4m3x2_to_bf16x2(raw.x, sg);
+            lo.y = e4m3x2_to_bf16x2(raw.x >> 16, sg);
+            lo.z = e4m3x2_to_bf16x2(raw.y, sg);
+            lo.w = e4m3x2_to_bf16x2(raw.y >> 16, sg);
+            hi.x = e4m3x2_to_bf16x2(raw.z, sg);
+            hi.y = e4m3x2_to_bf16x2(raw.z >> 16, sg);
+            hi.z = e4m3x2_to_bf16x2(raw.w, sg);
+            hi.w = e4m3x2_to_bf16x2(raw.w >> 16, sg);
+            uint8_t *dst = sRing + s * kChunk + row * 128;
+            *reinterpret_cast<uint4 *>(dst + (((2 * u) ^ (row & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4 *>(dst + (((2 * u + 1) ^ (row & 7)) << 4)) = hi;
+          }
+          ptx::fence_proxy_async_smem();   // the MMAs read the slot through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            ptx::mbar_arrive(bar + C::bFull + s);
+            ptx::mbar_arrive(bar + C::bStEmpty + st);
+          }
+          ++sc;
+        }
+      }
+    }
   }
 
   ptx::tc_fence_before();
@@ -484,26 +609,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int H>
+template <int H, bool F8>
 cudaError_t launch_h(const AttnArgs &a, int P, cudaStream_t s) {
-  using C = Cfg<H>;
+  using C = Cfg<H, F8>;
   const long long rows = a.page_size ? a.cache_len * kTile : (long long)a.B * a.cache_len;
   if (rows <= 0 || rows >= (1ll << 31) - 256) return cudaErrorNotSupported;
   CUtensorMap mq, mkv;
   const uint64_t dq[2] = {576, (uint64_t)a.B * H};
   const uint64_t dkv[2] = {576, (uint64_t)rows};
   const uint64_t st[1] = {576 * 2};
+  const uint64_t st8[1] = {576};
   const uint32_t bq[2] = {64, (uint32_t)H}, bkv[2] = {64, 64};
-  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mkv, a.cache, 2, dkv, st, bkv, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorNotSupported;
+  if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, bq, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorNotSupported;
+  const bool kv_ok = F8 ? encode_map_u8(&mkv, a.cache, 2, dkv, st8, bkv, CU_TENSOR_MAP_SWIZZLE_NONE)
+                        : encode_map_bf16(&mkv, a.cache, 2, dkv, st, bkv, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!kv_ok) return cudaErrorNotSupported;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_smallh_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(attn_smallh_kernel<H, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  return launch_pdl(attn_smallh_kernel<H>, dim3(P), dim3(kThreads), C::kSmem, s, 1, mq, mkv, a, rows);
+  return launch_pdl(attn_smallh_kernel<H, F8>, dim3(P), dim3(C::kThreads), C::kSmem, s, 1, mq, mkv, a, rows);
 }
 
 }  // namespace
@@ -511,8 +639,14 @@ cudaError_t launch_h(const AttnArgs &a, int P, cudaStream_t s) {
 cudaError_t launch_attn_tc_smallh(const AttnArgs &a, int P, cudaStream_t s) {
   if (a.d_c != 512 || a.d_r != 64) return cudaErrorNotSupported;
   if (a.page_size != 0 && a.page_size != kTile) return cudaErrorNotSupported;
-  if (a.n_h == 16) return launch_h<16>(a, P, s);
-  if (a.n_h == 32) return launch_h<32>(a, P, s);
+  if (a.kv_scale) {
+    if (a.n_groups != kGroups8) return cudaErrorNotSupported;
+    if (a.n_h == 16) return launch_h<16, true>(a, P, s);
+    if (a.n_h == 32) return launch_h<32, true>(a, P, s);
+    return cudaErrorNotSupported;
+  }
+  if (a.n_h == 16) return launch_h<16, false>(a, P, s);
+  if (a.n_h == 32) return launch_h<32, false>(a, P, s);
   return cudaErrorNotSupported;
 }
 

@@ -39,8 +39,9 @@ static EncodeTiledFn resolve_encode() {
 
 bool tma_available() { return resolve_encode() != nullptr; }
 
-bool encode_map_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                     const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz) {
+static bool encode_map(CUtensorMap *map, CUtensorMapDataType type, const void *base, int rank,
+                       const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                       CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = resolve_encode();
   if (!fn) return false;
   cuuint64_t d[5], st[4];
@@ -51,10 +52,20 @@ bool encode_map_bf16(CUtensorMap *map, const void *base, int rank, const uint64_
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), d, st,
-                  bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = fn(map, type, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_map_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                     const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides, box, swz);
+}
+
+bool encode_map_u8(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                   const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides, box, swz);
 }
 
 namespace {
@@ -94,6 +105,9 @@ struct GemmParams {
   const int *block_table;
   int max_blocks;
   int page_size;
+  // append: when set, token n's row goes to out_f32[n * (d_c + d_r) ..] in
+  // float32 (for a later FP8 quantisation) instead of to the cache
+  float *out_f32;
   unsigned *status;
 };
 
@@ -250,8 +264,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (n < g.N) {
           const int b = n / g.T, t = n % g.T;
           p = g.start_pos[b] + t;
-          row = dest_row(b, p, g);
-          if (row < 0) atomicOr(g.status, kStatusBounds);
+          if (g.out_f32) {
+            row = n;
+          } else {
+            row = dest_row(b, p, g);
+            if (row < 0) atomicOr(g.status, kStatusBounds);
+          }
         }
         s_row[j] = row;
         s_pos[j] = p;
@@ -306,7 +324,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mm_ok || n >= g.N) continue;
             if (g.mode == kEpiAppend) {
               const long long row = s_row[c0 + j];
-              if (row >= 0) g.out[row * (long long)(g.d_c + g.d_r) + mm] = __float2bfloat16_rn(v);
+              if (row >= 0) {
+                if (g.out_f32) g.out_f32[row * (long long)(g.d_c + g.d_r) + mm] = v;
+                else g.out[row * (long long)(g.d_c + g.d_r) + mm] = __float2bfloat16_rn(v);
+              }
             } else {
               g.out[(long long)n * g.out_ld + (long long)z * g.out_z + mm] = __float2bfloat16_rn(v);
             }
@@ -386,7 +407,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (m >= g.M_valid) continue;
           if (g.mode == kEpiAppend) {
             const long long row = s_row[c];
-            if (row >= 0) g.out[row * (long long)(g.d_c + g.d_r) + m] = __float2bfloat16_rn(v[e]);
+            if (row >= 0) {
+              if (g.out_f32) g.out_f32[row * (long long)(g.d_c + g.d_r) + m] = v[e];
+              else g.out[row * (long long)(g.d_c + g.d_r) + m] = __float2bfloat16_rn(v[e]);
+            }
           } else {
             g.out[(long long)n * g.out_ld + (long long)z * g.out_z + m] = __float2bfloat16_rn(v[e]);
           }
@@ -582,7 +606,7 @@ cudaError_t launch_wo_tc(const mla_config &c, const void *o, const void *w_o, vo
 cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, const int *start_pos,
                              const void *w_dkv, const void *w_kr, void *cache, long long cache_len,
                              const int *block_table, int max_blocks, const double *theta,
-                             unsigned *status, cudaStream_t s) {
+                             unsigned *status, cudaStream_t s, float *rows_out) {
   if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr)) return cudaErrorNotSupported;
   const long long N = (long long)B * T;
   if (N > 65535LL * 256) return cudaErrorNotSupported;
@@ -617,6 +641,7 @@ cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, c
   g.block_table = block_table;
   g.max_blocks = max_blocks;
   g.page_size = c.page_size;
+  g.out_f32 = rows_out;
   g.status = status;
   const int mtiles = c.d_c / 128 + (c.d_r + 127) / 128;
   return dispatch_bn<false>((int)N, m0, m1, mb, g, mtiles, 1, s, bn);

@@ -243,6 +243,63 @@ int mla_decode_attn_combine_noalloc(mla_handle *handle, const void *q_abs, const
 /* Size in bytes of the scratch array mla_decode_attn_combine_noalloc uses. */
 size_t mla_noalloc_scratch_bytes(void);
 
+/* ---------------------------------------------------------------------------
+ * FP8 latent cache ("DeepSeek-V2" §3.2.3: the deployed KV cache is quantised
+ * to about 6 bits per element, format not given; "DeepSeek-V3" note, FP8
+ * section: activations are quantised tile-wise, per token and per 128
+ * channels, scaled by the group's absolute maximum).
+ *
+ * Format.  A token's row of D = d_c + d_r elements [c^KV | k^R] is stored as
+ * D one-byte OCP FP8 E4M3 codes, in the same row layout as the cfg.dtype
+ * cache (contiguous [B, cache_len, D] or paged [cache_len, page_size, D]).
+ * The row is cut into scale groups of 128 channels over c^KV, then over k^R
+ * (the last group of each part may be narrower); G = mla_fp8_scale_groups()
+ * (5 at d_c = 512, d_r = 64).  kv_scale is float32 [rows, G] with the same
+ * row indexing as the codes.  For a group with absolute maximum a (float32):
+ * sigma = a / 448 and code = E4M3(x / sigma), both divisions rounded to
+ * nearest in float32, the conversion rounding to nearest even and saturating
+ * at 448; a group of zeros has sigma = 0 and zero codes.  The stored value is
+ * code * sigma.
+ * ------------------------------------------------------------------------- */
+
+/* G, the number of scale groups per row (0 for a NULL handle). */
+int mla_fp8_scale_groups(const mla_handle *handle);
+
+/* Bytes of workspace mla_cache_append_fp8 needs for B sequences of T new
+ * tokens (float32 rows before quantisation); 0 on invalid arguments. */
+size_t mla_cache_append_fp8_workspace_size(const mla_handle *handle, int B, int T);
+
+/* mla_cache_append into an FP8 cache: the rows [c^KV ; RoPE(k^R)] are formed
+ * in float32 exactly as mla_cache_append forms them, then quantised.
+ *   cache       uint8 codes, layout as for mla_cache_append
+ *   kv_scale    float32 [rows, G]
+ *   workspace   >= mla_cache_append_fp8_workspace_size(handle, B, T) bytes of
+ *               device memory, 256-byte aligned; overwritten.
+ * Other arguments and errors as for mla_cache_append; MLA_ERR_WORKSPACE for a
+ * missing, misaligned or short workspace. */
+int mla_cache_append_fp8(mla_handle *handle, const void *h, int B, int T, const int *start_pos,
+                         const void *w_dkv, const void *w_kr, void *cache, float *kv_scale,
+                         long long cache_len, const int *block_table, int max_blocks_per_seq,
+                         void *workspace, size_t ws_bytes, mla_stream_t stream);
+
+/* Quantise n_rows rows [n_rows, D] (cfg.dtype; e.g. rows of an existing
+ * cache) into codes [n_rows, D] (uint8) and kv_scale [n_rows, G], row i to
+ * row i.  Rows are independent, so a contiguous cache converts in one call
+ * and a paged pool by passing the whole pool as rows. */
+int mla_quantize_rows_fp8(mla_handle *handle, const void *rows, long long n_rows, void *codes,
+                          float *kv_scale, mla_stream_t stream);
+
+/* mla_decode_attn over an FP8 cache (codes and kv_scale as above).  The
+ * partials, the workspace and mla_combine_splits are those of
+ * mla_decode_attn.  16 or 32 heads at d_c = 512, d_r = 64 run on the tensor
+ * cores (the codes are widened to bf16 in shared memory, code * sigma rounded
+ * to bf16); every other shape, 128 heads included, on the CUDA-core kernel,
+ * which is functional but not fast.  kv_scale NULL is MLA_ERR_INVALID_ARG. */
+int mla_decode_attn_fp8(mla_handle *handle, const void *q_abs, const void *cache, const float *kv_scale,
+                        long long cache_len, const int *block_table, int max_blocks_per_seq,
+                        const int *ctx_len, int B, int num_parts, void *workspace, size_t ws_bytes,
+                        mla_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

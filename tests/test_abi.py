@@ -25,7 +25,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -78,6 +78,13 @@ def test_create_without_device_fails_cleanly(lib):
     assert lib.mla_set_rope_scaling(None, 40.0, 4096, 1.0, 32.0, 0.0707) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_query_proj(None, None, 1, None, 0, None, None, None, None, None,
                               None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_fp8_scale_groups(None) == 0
+    assert lib.mla_cache_append_fp8_workspace_size(None, 4, 1) == 0
+    assert lib.mla_cache_append_fp8(None, None, 1, 1, None, None, None, None, None, 0, None, 0,
+                                    None, 0, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_quantize_rows_fp8(None, None, 1, None, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode_attn_fp8(None, None, None, None, 0, None, 0, None, 1, 0, None, 0,
+                                   None) == M.MLA_ERR_INVALID_ARG
 
 
 def python_plan(ctx, P):
