@@ -36,13 +36,25 @@ constexpr int kTileTok = 64;
 constexpr float kRescale = 8.0f;
 constexpr int kGroups8 = 5;                // scale groups of a 576-wide row
 
+#ifndef MLA_F8_CONV_WARPS
+#define MLA_F8_CONV_WARPS 4
+#endif
+#ifndef MLA_F8_RING
+#define MLA_F8_RING 21
+#endif
+#ifndef MLA_F8_STAGE16
+#define MLA_F8_STAGE16 6
+#endif
+
 template <int H, bool F8>
 struct Cfg {
-  static constexpr int kThreads = F8 ? 320 : 192;
+  static constexpr int kConvWarps = F8 ? MLA_F8_CONV_WARPS : 0;   // FP8 converter warps (4 or 8)
+  static constexpr int kThreads = 192 + 32 * kConvWarps;
   // Ring chunk slots.  A tile holds its nine slots until its P.V is done,
   // which is issued after the next tile's S: at least two tiles' worth.
-  static constexpr int kNS = F8 ? 18 : (H <= 16 ? 24 : 18);
-  static constexpr int kNSt = F8 ? (H <= 16 ? 12 : 8) : 0;  // FP8 staging chunks
+  static constexpr int kNS = F8 ? (H <= 16 ? MLA_F8_RING : 18) : (H <= 16 ? 24 : 18);
+  static constexpr int kNSt = F8 ? (H <= 16 ? MLA_F8_STAGE16 : 8) : 0;  // FP8 staging chunks
+  static_assert(!F8 || kNS >= 18, "the ring must hold two tiles");
   static constexpr int kQ = 9 * H * 128;                    // H rows x 576
   static constexpr int kPT = H * 128;                       // P^T: H rows x 64 tokens
   static constexpr int kOffQ = 0;
@@ -150,7 +162,7 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
                        const AttnArgs a, const long long kv_rows) {
   using C = Cfg<H, F8>;
   constexpr int NS = C::kNS;
-  constexpr int NSt = C::kNSt;
+  constexpr int NSt = C::kNSt > 0 ? C::kNSt : 1;   // (1: never used without FP8)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + C::kOffQ;
@@ -170,12 +182,12 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      ptx::mbar_init(bar + C::bFull + s, F8 ? 4 : 1);   // FP8: the four converter warps
+      ptx::mbar_init(bar + C::bFull + s, F8 ? C::kConvWarps : 1);   // FP8: every converter warp
       ptx::mbar_init(bar + C::bEmpty + s, 1);
     }
     for (int s = 0; s < NSt; ++s) {
       ptx::mbar_init(bar + C::bStFull + s, 1);
-      ptx::mbar_init(bar + C::bStEmpty + s, 4);
+      ptx::mbar_init(bar + C::bStEmpty + s, C::kConvWarps);
     }
     ptx::mbar_init(bar + C::bQFull, 1);
     ptx::mbar_init(bar + C::bQEmpty, 1);
@@ -537,10 +549,12 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       ++npc;
     }
   } else if (F8) {
-    // ------------------------------------------- FP8 converters (warps 6-9)
-    // Thread ct handles rows ct/4 and ct/4 + 32 of every chunk, 16 codes
-    // (unit ct%4 of the row's 64) each: 32 bytes of bf16, i.e. two 16-byte
-    // units of the 128-byte-swizzled ring row.
+    // ------------------------------------------ FP8 converters (warps 6 ..)
+    // A chunk is 64 rows x 4 units of 16 codes.  Thread ct handles unit ct%4
+    // of rows ct/4, ct/4 + RS, ... (RS = rows covered by all converters at
+    // once): 16 codes become 32 bytes of bf16, two 16-byte units of the
+    // 128-byte-swizzled ring row.
+    constexpr int RS = (C::kConvWarps > 0 ? C::kConvWarps : 4) * 8, NR = 64 / RS;
     const int ct = (warp - 6) * 32 + lane;
     const int r0 = ct >> 2, u = ct & 3;
     Walk w;
@@ -551,10 +565,10 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
     while (ok && walk_next(w, a, share, pc)) {
       for (int k = 0; k < pc.ntiles && ok; ++k) {
         const int tok0 = pc.tok_begin + kTileTok * k;
-        float sig[2][kGroups8];
+        float sig[NR][kGroups8];
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int t = tok0 + r0 + 32 * rr;
+        for (int rr = 0; rr < NR; ++rr) {
+          const int t = tok0 + r0 + RS * rr;
           const long long r = t < pc.ctx ? kv_row(a, pc.b, t) : -1;
 #pragma unroll
           for (int g = 0; g < kGroups8; ++g) sig[rr][g] = r >= 0 ? a.kv_scale[r * kGroups8 + g] : 0.f;
@@ -568,8 +582,8 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
           }
           const int g = c >> 1;   // chunks 0-7: c^KV groups 0-3; chunk 8: the k^R group
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int row = r0 + 32 * rr;
+          for (int rr = 0; rr < NR; ++rr) {
+            const int row = r0 + RS * rr;
             // select the group's scale without indexing the array at run time
             float sg = sig[rr][0];
 #pragma unroll
