@@ -15,8 +15,6 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; 
 
 bool dtype_ok(int dt) { return dt == MLA_BF16 || dt == MLA_FP32; }
 
-size_t elt(const mla_config &c) { return c.dtype == MLA_FP32 ? 4 : 2; }
-
 // Attention kernel for a configuration.  The tensor-core kernels exist for the
 // DeepSeek-V2 attention shapes in bf16; everything else runs the generic
 // CUDA-core kernel.
