@@ -556,7 +556,73 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
+    e2e_serial_ms = e0.elapsed_time(e1) / args.steps
+
+    # The same steps with the transfers overlapped: every step still copies its
+    # own inputs from pinned host memory and reads its result back, but the
+    # host-to-device copies run on one stream and the device-to-host reads on
+    # another, into double buffers, so step i's copies overlap the compute of
+    # steps i-1 and i+1.
+    def e2e_pipelined_ms():
+        copy_s = torch.cuda.Stream(device=dev)
+        d2h_s = torch.cuda.Stream(device=dev)
+        ins = [{k: torch.empty_like(v, device=dev) for k, v in hp.items()} for _ in range(2)]
+        outs = [torch.empty_like(o) for _ in range(2)]
+        o_hosts = [torch.empty(o.shape, dtype=bf).pin_memory() for _ in range(2)]
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]         # step using ins[k], outs[k] computed
+        out_free = [torch.cuda.Event() for _ in range(2)]     # device-to-host read of outs[k] done
+        for k in range(2):
+            done[k].record(stream)
+            out_free[k].record(d2h_s)
+
+        def one(i):
+            k = i & 1
+            copy_s.wait_event(done[k])
+            with torch.cuda.stream(copy_s):
+                for name in hp:
+                    ins[k][name].copy_(hp[name], non_blocking=True)
+            in_ready[k].record(copy_s)
+            stream.wait_event(in_ready[k])
+            stream.wait_event(out_free[k])
+            d = ins[k]
+            # no event between the five calls, so that each kernel's set-up
+            # still overlaps the previous one's tail
+            M.mla_cache_append(handle, d["h_new"], B, 1, d["pos"], w_dkv, w_kr, cache, cap, None, 0, sh)
+            M.mla_absorb_q(handle, d["q_nope"], d["q_rope"], d["pos"], w_uk, q_abs, B, sh)
+            M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, d["ctx"], B, P, ws, ws_bytes, sh)
+            M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
+            M.mla_out_proj(handle, ctx_lat, w_uv, None, outs[k], None, B, sh)
+            done[k].record(stream)
+            d2h_s.wait_event(done[k])
+            with torch.cuda.stream(d2h_s):
+                o_hosts[k].copy_(outs[k], non_blocking=True)
+            out_free[k].record(d2h_s)
+
+        for i in range(3):
+            one(i)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(copy_s)
+        for i in range(args.steps):
+            one(i)
+        stream.wait_stream(copy_s)
+        stream.wait_stream(d2h_s)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / args.steps
+
+    if world > 1:
+        dist.barrier()
+    e2e_mode = "pipelined: inputs and results double-buffered, copies on their own streams"
+    try:
+        e2e_ms = e2e_pipelined_ms()
+    except Exception as exc:  # keep the serial figure rather than lose the line
+        e2e_ms = e2e_serial_ms
+        e2e_mode = f"serial (pipelined run failed: {type(exc).__name__}: {exc})"
+    st = M.mla_get_device_status(handle, sh)
+    if st != M.MLA_OK:
+        raise M.MlaError(st, "device status after the end-to-end runs")
 
     # ---- attention over an FP8 cache (a separate workload, rank 0 only)
     fp8 = None
@@ -564,7 +630,8 @@ def run_ours(args):
         fp8 = measure_fp8(M, dev, args.steps, rank_seed(rank) + 17)
 
     # ---- reduce over ranks: max time
-    ms, attn_ms, e2e_ms = reduce_max_over_ranks([ms, attn_ms, e2e_ms], world, dev)
+    ms, attn_ms, e2e_ms, e2e_serial_ms = reduce_max_over_ranks([ms, attn_ms, e2e_ms, e2e_serial_ms],
+                                                               world, dev)
     if world > 1:
         dist.barrier()
     M.mla_destroy(handle)
@@ -604,7 +671,9 @@ def run_ours(args):
                      "frac_of_8TBps": attn_gbs / 8000.0,
                      "tensor_tflops": attn_flops / (attn_ms * 1e-3) / 1e12},
         "e2e": {"value": whole_job_gbs(step_bytes, world, e2e_ms), "unit": "GB/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "mode": e2e_mode, "serial_ms_per_step": e2e_serial_ms,
+                "serial_value": whole_job_gbs(step_bytes, world, e2e_serial_ms)},
         "gpu_launches": 6 * args.steps,
         "per_call_us": per_call,
         "per_call_note": "separate pass after the timed region, events between all calls",
