@@ -162,7 +162,9 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
                        const AttnArgs a, const long long kv_rows) {
   using C = Cfg<H, F8>;
   constexpr int NS = C::kNS;
-  constexpr int NSt = C::kNSt > 0 ? C::kNSt : 1;   // (1: never used without FP8)
+  // Staging chunks as a divisor for the FP8 code paths; without FP8 those
+  // paths never run and there are no staging barriers (C::kNSt = 0).
+  constexpr int NSt = C::kNSt > 0 ? C::kNSt : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + C::kOffQ;
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       ptx::mbar_init(bar + C::bFull + s, F8 ? C::kConvWarps : 1);   // FP8: every converter warp
       ptx::mbar_init(bar + C::bEmpty + s, 1);
     }
-    for (int s = 0; s < NSt; ++s) {
+    for (int s = 0; s < C::kNSt; ++s) {
       ptx::mbar_init(bar + C::bStFull + s, 1);
       ptx::mbar_init(bar + C::bStEmpty + s, C::kConvWarps);
     }
