@@ -33,7 +33,7 @@ EXPORTED = (
     "mla_get_device_status", "mla_plan_pieces", "mla_decode_attn_combine_noalloc",
     "mla_noalloc_scratch_bytes", "mla_set_rope_scaling",
     "mla_fp8_scale_groups", "mla_cache_append_fp8_workspace_size", "mla_cache_append_fp8",
-    "mla_quantize_rows_fp8", "mla_decode_attn_fp8",
+    "mla_quantize_rows_fp8", "mla_decode_attn_fp8", "mla_selftest_wait_timeout",
 )
 
 
@@ -86,6 +86,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_cache_append_fp8": (i, [vp, vp, i, i, vp, vp, vp, vp, vp, ll, vp, i, vp, sz, vp]),
         "mla_quantize_rows_fp8": (i, [vp, vp, ll, vp, vp, vp]),
         "mla_decode_attn_fp8": (i, [vp, vp, vp, vp, ll, vp, i, vp, i, i, vp, sz, vp]),
+        "mla_selftest_wait_timeout": (i, [vp, ll, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -201,6 +202,11 @@ def mla_decode_attn_fp8(handle, q_abs, cache, kv_scale, cache_len, block_table, 
                                       _ptr(block_table), max_blocks_per_seq, _ptr(ctx_len), B,
                                       num_parts, _ptr(workspace), ws_bytes, _stream(stream)),
            "mla_decode_attn_fp8")
+
+
+def mla_selftest_wait_timeout(handle, limit_ns, stream=None):
+    _check(load().mla_selftest_wait_timeout(handle, limit_ns, _stream(stream)),
+           "mla_selftest_wait_timeout")
 
 
 def mla_decode_attn(handle, q_abs, cache, cache_len, block_table, max_blocks_per_seq, ctx_len, B,

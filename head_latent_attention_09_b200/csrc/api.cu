@@ -366,6 +366,12 @@ int mla_query_proj(mla_handle *h, const void *x, int B, const void *w_dq, int d_
   return MLA_OK;
 }
 
+int mla_selftest_wait_timeout(mla_handle *h, long long limit_ns, mla_stream_t stream) {
+  if (!h || limit_ns < 1000 || limit_ns > 1000000000LL) return MLA_ERR_INVALID_ARG;
+  return from_cuda(launch_wait_timeout_selftest(h->d_status, (unsigned long long)limit_ns,
+                                                (cudaStream_t)stream));
+}
+
 int mla_get_device_status(mla_handle *h, mla_stream_t stream) {
   if (!h) return MLA_ERR_INVALID_ARG;
   unsigned v = 0;

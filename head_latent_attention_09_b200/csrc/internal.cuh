@@ -214,6 +214,10 @@ cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K
 cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s);
 cudaError_t launch_attn_tc_smallh(const AttnArgs &a, int P, cudaStream_t s);
 
+// One bounded wait on a barrier that nothing completes, giving up after
+// limit_ns: sets the status word's time-out bit (self-test of that path).
+cudaError_t launch_wait_timeout_selftest(unsigned *status, unsigned long long limit_ns, cudaStream_t s);
+
 // Resolve the driver entry point for tensor-map encoding (no libcuda link).
 bool tma_available();
 

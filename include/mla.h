@@ -205,6 +205,14 @@ int mla_combine_splits(mla_handle *handle, const void *workspace, size_t ws_byte
 int mla_out_proj(mla_handle *handle, const void *ctx_lat, const void *w_uv, const void *w_o,
                  void *o, void *u, int B, mla_stream_t stream);
 
+/* Self-test of the device-side time-out path: launches one wait on a barrier
+ * that nothing completes, which gives up after limit_ns nanoseconds (1e3 ..
+ * 1e9) and sets the time-out bit in the handle's status word, exactly as a
+ * wait in the decode kernels does past its 2 s limit.  The next
+ * mla_get_device_status then returns MLA_ERR_TIMEOUT; the context stays
+ * usable.  MLA_ERR_INVALID_ARG for a NULL handle or a limit out of range. */
+int mla_selftest_wait_timeout(mla_handle *handle, long long limit_ns, mla_stream_t stream);
+
 /* Synchronise `stream`, read and clear the handle's device status word.
  * Returns MLA_OK, MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_BOUNDS or MLA_ERR_CUDA. */
 int mla_get_device_status(mla_handle *handle, mla_stream_t stream);

@@ -78,6 +78,7 @@ def test_create_without_device_fails_cleanly(lib):
     assert lib.mla_set_rope_scaling(None, 40.0, 4096, 1.0, 32.0, 0.0707) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_query_proj(None, None, 1, None, 0, None, None, None, None, None,
                               None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_selftest_wait_timeout(None, 5000000, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_fp8_scale_groups(None) == 0
     assert lib.mla_cache_append_fp8_workspace_size(None, 4, 1) == 0
     assert lib.mla_cache_append_fp8(None, None, 1, 1, None, None, None, None, None, 0, None, 0,
