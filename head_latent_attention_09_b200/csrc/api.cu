@@ -5,6 +5,8 @@
 
 #include <cmath>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.cuh"
 
 using namespace mla;
@@ -12,6 +14,16 @@ using namespace mla;
 namespace {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// An NVTX range around an entry point, named after it, so that profilers can
+// attribute the kernels each call launches (e.g. ncu --nvtx).  Without an
+// attached tool the push and pop are no-ops.
+struct Range {
+  explicit Range(const char *name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range &) = delete;
+  Range &operator=(const Range &) = delete;
+};
 
 bool dtype_ok(int dt) { return dt == MLA_BF16 || dt == MLA_FP32; }
 
@@ -149,6 +161,7 @@ int mla_set_rope_scaling(mla_handle *h, double factor, int original_ctx, double 
 int mla_cache_append(mla_handle *h, const void *x, int B, int T, const int *start_pos,
                      const void *w_dkv, const void *w_kr, void *cache, long long cache_len,
                      const int *block_table, int max_blocks_per_seq, mla_stream_t stream) {
+  Range range("mla_cache_append");
   if (!h || B < 0 || T < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0 || T == 0) return MLA_OK;
   if (!x || !start_pos || !w_dkv || !w_kr || !cache) return MLA_ERR_INVALID_ARG;
@@ -169,6 +182,7 @@ int mla_cache_append(mla_handle *h, const void *x, int B, int T, const int *star
 
 int mla_absorb_q(mla_handle *h, const void *q_nope, const void *q_rope, const int *pos,
                  const void *w_uk, void *q_abs, int B, mla_stream_t stream) {
+  Range range("mla_absorb_q");
   if (!h || B < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if (!q_nope || !q_rope || !pos || !w_uk || !q_abs) return MLA_ERR_INVALID_ARG;
@@ -240,6 +254,7 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
 int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long long cache_len,
                     const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
                     int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
+  Range range("mla_decode_attn");
   return decode_attn(h, q_abs, cache, nullptr, cache_len, block_table, max_blocks_per_seq, ctx_len, B,
                      num_parts, workspace, ws_bytes, stream);
 }
@@ -248,6 +263,7 @@ int mla_decode_attn_fp8(mla_handle *h, const void *q_abs, const void *cache, con
                         long long cache_len, const int *block_table, int max_blocks_per_seq,
                         const int *ctx_len, int B, int num_parts, void *workspace, size_t ws_bytes,
                         mla_stream_t stream) {
+  Range range("mla_decode_attn_fp8");
   if (!kv_scale && h && B > 0) return MLA_ERR_INVALID_ARG;
   return decode_attn(h, q_abs, cache, kv_scale, cache_len, block_table, max_blocks_per_seq, ctx_len, B,
                      num_parts, workspace, ws_bytes, stream);
@@ -265,6 +281,7 @@ int mla_cache_append_fp8(mla_handle *h, const void *x, int B, int T, const int *
                          const void *w_dkv, const void *w_kr, void *cache, float *kv_scale,
                          long long cache_len, const int *block_table, int max_blocks_per_seq,
                          void *workspace, size_t ws_bytes, mla_stream_t stream) {
+  Range range("mla_cache_append_fp8");
   if (!h || B < 0 || T < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0 || T == 0) return MLA_OK;
   if (!x || !start_pos || !w_dkv || !w_kr || !cache || !kv_scale) return MLA_ERR_INVALID_ARG;
@@ -292,6 +309,7 @@ int mla_cache_append_fp8(mla_handle *h, const void *x, int B, int T, const int *
 
 int mla_quantize_rows_fp8(mla_handle *h, const void *rows, long long n_rows, void *codes, float *kv_scale,
                           mla_stream_t stream) {
+  Range range("mla_quantize_rows_fp8");
   if (!h || n_rows < 0) return MLA_ERR_INVALID_ARG;
   if (n_rows == 0) return MLA_OK;
   if (!rows || !codes || !kv_scale) return MLA_ERR_INVALID_ARG;
@@ -303,6 +321,7 @@ int mla_quantize_rows_fp8(mla_handle *h, const void *rows, long long n_rows, voi
 
 int mla_combine_splits(mla_handle *h, const void *workspace, size_t ws_bytes, int B, int num_parts,
                        void *ctx_lat, float *lse, mla_stream_t stream) {
+  Range range("mla_combine_splits");
   if (!h || B < 0 || num_parts < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if (!ctx_lat) return MLA_ERR_INVALID_ARG;
@@ -315,6 +334,7 @@ int mla_combine_splits(mla_handle *h, const void *workspace, size_t ws_bytes, in
 
 int mla_out_proj(mla_handle *h, const void *ctx_lat, const void *w_uv, const void *w_o, void *o,
                  void *u, int B, mla_stream_t stream) {
+  Range range("mla_out_proj");
   if (!h || B < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if (!ctx_lat || !w_uv || !o || (w_o && !u)) return MLA_ERR_INVALID_ARG;
@@ -346,6 +366,7 @@ cudaError_t linear(const mla_handle *h, const void *x, const void *w, void *y, i
 
 int mla_query_proj(mla_handle *h, const void *x, int B, const void *w_dq, int d_cq, const void *w_uq,
                    const void *w_qr, void *c_q, void *q_nope, void *q_rope, mla_stream_t stream) {
+  Range range("mla_query_proj");
   if (!h || B < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if (!x || !w_uq || !w_qr || !q_nope || !q_rope) return MLA_ERR_INVALID_ARG;
