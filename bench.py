@@ -282,6 +282,12 @@ def run_reference(args):
 FP8_WORKLOAD = "v2lite_b4_ctx128k"
 
 
+def fp8_cache_bytes(tokens, D, groups):
+    """Bytes an FP8 cache holds for `tokens` rows: D one-byte codes and
+    `groups` float32 scales per row."""
+    return tokens * (D + 4 * groups)
+
+
 def measure_fp8(M, dev, steps, seed):
     """Attention over the same latent cache stored in bf16 and in FP8 (E4M3
     codes + one float32 scale per token and 128-channel group), on the
@@ -351,7 +357,7 @@ def measure_fp8(M, dev, steps, seed):
         M.mla_destroy(handle)
     tokens = int(ctx.sum())
     return {"workload": FP8_WORKLOAD, "tokens": tokens, "bf16_us": us_bf16, "fp8_us": us_fp8,
-            "bf16_bytes": tokens * D * 2, "fp8_bytes": tokens * (D + 4 * G)}
+            "bf16_bytes": tokens * D * 2, "fp8_bytes": fp8_cache_bytes(tokens, D, G)}
 
 
 def run_ours(args):
