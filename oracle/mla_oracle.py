@@ -21,7 +21,7 @@ the pages, written out directly:
   directly from h_t), Appendix C (W^UK can be absorbed into the query side and
   W^UV into the output side by associativity).
 
-Readings of points the pages leave open (each is listed in the design doc):
+Readings of points the pages leave open:
 
 * RoPE follows the RoFormer form the pages cite (Su et al.): consecutive pairs
   (x_{2k}, x_{2k+1}) rotated by angle p * theta_k, theta_k = base^(-2k/d_h^R),
@@ -40,7 +40,10 @@ Readings of points the pages leave open (each is listed in the design doc):
   frequency, one that turns fewer than alpha times is slowed by s, linear in
   between), and sqrt(t) scaling both the query and the key, i.e. every score
   (content and rotary part) multiplied by t = (c ln s + 1)^2; c is a
-  parameter, 0.0707 by default.  s = 1 is plain RoPE.
+  parameter, 0.0707 by default.  s = 1 is plain RoPE.  (YaRN itself writes
+  its logit temperature the same way: the square root of the factor on the
+  logits is 0.1 ln s + 1, applied as a scale on both q and k, so the logits
+  carry its square.)
 * FP8 latent cache ("DeepSeek-V2" §3.2.3 quantises the deployed KV cache to
   about 6 bits per element without giving the format; the "DeepSeek-V3" note's
   FP8 section quantises activations tile-wise, per token and per 128 channels,

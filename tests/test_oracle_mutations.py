@@ -70,6 +70,23 @@ def _yarn_ramp_inverted(d_r, base):
     return plain * plain / np.where(scaled == 0, 1.0, scaled) / spec.factor
 
 
+def _yarn_ramp_linear_in_pair_index(d_r, base):
+    # blends linearly in the pair index between the (fractional) indices where
+    # a pair turns beta and alpha times, instead of linearly in the turns
+    spec = O._spec(base)
+    plain = _ORIG_THETA(d_r, spec.base)
+    if spec.factor <= 1.0:
+        return plain
+    k = np.arange(d_r // 2, dtype=np.float64)
+
+    def index_at(turns):
+        return -(d_r / 2.0) * math.log(2 * math.pi * turns / spec.original_ctx) / math.log(spec.base)
+
+    k_fast, k_slow = index_at(spec.beta), index_at(spec.alpha)
+    gamma = np.clip((k_slow - k) / (k_slow - k_fast), 0.0, 1.0)
+    return (1.0 - gamma) * plain / spec.factor + gamma * plain
+
+
 def _temperature_not_squared(base):
     spec = O._spec(base)
     return 1.0 if spec.factor <= 1.0 else spec.mscale_coef * math.log(spec.factor) + 1.0
@@ -120,7 +137,11 @@ MUTATIONS = [
      [P.test_yarn_keeps_fast_pairs_and_slows_slow_pairs_by_s,
       lambda: P.test_yarn_absorbed_explicit_and_brute_force_agree(0.0707)]),
     ("yarn_temperature_not_squared", "attention_temperature", _temperature_not_squared,
-     [lambda: P.test_yarn_absorbed_explicit_and_brute_force_agree(0.1)]),
+     [P.test_yarn_temperature_matches_page_values,
+      lambda: P.test_yarn_two_token_softmax_closed_form("v2"),
+      lambda: P.test_yarn_two_token_softmax_closed_form("v3")]),
+    ("yarn_ramp_linear_in_pair_index", "rope_theta", _yarn_ramp_linear_in_pair_index,
+     [P.test_yarn_interior_ramp_hand_values]),
     ("e4m3_truncates", "e4m3_encode", _e4m3_truncating,
      [P.test_e4m3_encode_matches_library_rounding, P.test_e4m3_encode_brute_force_nearest]),
     ("fp8_groups_mix_parts", "fp8_groups", _groups_across_parts,

@@ -372,6 +372,56 @@ def test_yarn_temperature_acts_as_a_query_scale():
     assert np.allclose(res["lse"], lse, rtol=1e-13)
 
 
+def test_yarn_temperature_matches_page_values():
+    # sqrt(t) = c ln s + 1 with the pages' s and c, squared by hand
+    # (tests/golden/yarn_scaling.txt): t multiplies every score.
+    g = _golden("yarn_scaling.txt")
+    for coef, want in ((g["v2_coef"], g["v2_t"]), (g["v3_coef"], g["v3_t"])):
+        spec = O.RopeSpec(base=10000.0, factor=g["yarn_s"], original_ctx=int(g["yarn_window"]),
+                          alpha=g["yarn_alpha"], beta=g["yarn_beta"], mscale_coef=coef)
+        assert abs(O.attention_temperature(spec) - want) <= 1e-14 * want
+    assert abs(g["v2_sqrt_t"] ** 2 - g["v2_t"]) <= 1e-14 and abs(g["v3_sqrt_t"] ** 2 - g["v3_t"]) <= 1e-14
+
+
+@pytest.mark.parametrize("which", ["v2", "v3"])
+def test_yarn_two_token_softmax_closed_form(which):
+    # Two cached tokens whose content keys give raw scores differing by delta,
+    # no rotary signal: the decode step must weight them p0 / p1 =
+    # exp(t delta / sqrt(d_h + d_h^R)) with the hand-computed t of the pages'
+    # sqrt(t) = c ln s + 1.
+    g = _golden("yarn_scaling.txt")
+    spec = O.RopeSpec(base=10000.0, factor=g["yarn_s"], original_ctx=int(g["yarn_window"]),
+                      alpha=g["yarn_alpha"], beta=g["yarn_beta"], mscale_coef=g[which + "_coef"])
+    t = g[which + "_t"]
+    n_h, d_h, d_c, d_r = 1, 2, 2, 2
+    w_uk = np.eye(2)                       # k^C = c
+    w_uv = np.eye(2)                       # o = ctx_lat
+    rows = np.array([[1.0, 0.0, 0.0, 0.0], [0.0, 1.0, 0.0, 0.0]])
+    qn = np.array([[1.3, -0.4]])           # raw scores 1.3 and -0.4
+    qr = np.zeros((1, 2))
+    res = O.mla_decode_absorbed(qn, qr, 1, rows, w_uk, w_uv, n_h=n_h, d_h=d_h, d_c=d_c, d_r=d_r,
+                                base=spec)
+    delta = 1.3 - (-0.4)
+    k = t * delta / math.sqrt(d_h + d_r)
+    p0 = 1.0 / (1.0 + math.exp(-k))
+    assert np.allclose(res["o"][0], [p0, 1.0 - p0], rtol=0, atol=1e-14)
+    lse = t * 1.3 / math.sqrt(d_h + d_r) + math.log(1.0 + math.exp(-k))
+    assert abs(res["lse"][0] - lse) <= 1e-13
+
+
+def test_yarn_interior_ramp_hand_values():
+    # Frequencies of pairs that turn between alpha and beta times over the
+    # trained window: YaRN's ramp is linear in the number of turns, values
+    # worked out by hand in tests/golden/yarn_scaling.txt.
+    g = _golden("yarn_scaling.txt")
+    spec = O.RopeSpec(base=10000.0, factor=g["yarn_s"], original_ctx=int(g["yarn_window"]),
+                      alpha=g["yarn_alpha"], beta=g["yarn_beta"], mscale_coef=g["v2_coef"])
+    theta = O.rope_theta(64, spec)
+    for k in (12, 16, 20):
+        want = g[f"yarn_theta_k{k}"]
+        assert abs(theta[k] - want) <= 1e-13 * want, (k, theta[k], want)
+
+
 @pytest.mark.parametrize("coef", [0.0707, 0.1])
 def test_yarn_absorbed_explicit_and_brute_force_agree(coef):
     wl = TINY
