@@ -34,6 +34,7 @@ EXPORTED = (
     "mla_noalloc_scratch_bytes", "mla_set_rope_scaling",
     "mla_fp8_scale_groups", "mla_cache_append_fp8_workspace_size", "mla_cache_append_fp8",
     "mla_quantize_rows_fp8", "mla_decode_attn_fp8", "mla_selftest_wait_timeout",
+    "mla_set_strict",
 )
 
 
@@ -87,6 +88,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_quantize_rows_fp8": (i, [vp, vp, ll, vp, vp, vp]),
         "mla_decode_attn_fp8": (i, [vp, vp, vp, vp, ll, vp, i, vp, i, i, vp, sz, vp]),
         "mla_selftest_wait_timeout": (i, [vp, ll, vp]),
+        "mla_set_strict": (i, [vp, i]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -153,6 +155,10 @@ def mla_destroy(handle: int) -> None:
 def mla_set_rope_scaling(handle, factor, original_ctx, alpha, beta, mscale_coef) -> None:
     _check(load().mla_set_rope_scaling(handle, float(factor), int(original_ctx), float(alpha),
                                        float(beta), float(mscale_coef)), "mla_set_rope_scaling")
+
+
+def mla_set_strict(handle, strict) -> None:
+    _check(load().mla_set_strict(handle, int(bool(strict))), "mla_set_strict")
 
 
 def mla_cache_append(handle, h, B, T, start_pos, w_dkv, w_kr, cache, cache_len,

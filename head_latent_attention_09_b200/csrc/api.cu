@@ -57,6 +57,12 @@ int default_parts(const mla_handle *h) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Strict mode: a tensor-core kernel that exists for the configuration but
+// could not take the call's arguments is not replaced by a CUDA-core kernel.
+bool strict_refuses(const mla_handle *h, bool tc_exists, cudaError_t e) {
+  return h->strict && tc_exists && e == cudaErrorNotSupported;
+}
+
 }  // namespace
 
 extern "C" {
@@ -103,6 +109,10 @@ int mla_create(const mla_config *cfg, mla_handle **out) {
   h->gemm_kind = choose_gemm(*cfg);
   h->score_mult = 1.0;
   if ((h->attn_kind != kAttnSimt || h->gemm_kind != kGemmSimt) && !tma_available()) {
+    free(h);
+    return MLA_ERR_CUDA;
+  }
+  if (noalloc_scratch_lookup(&h->noalloc_scratch) != MLA_OK) {
     free(h);
     return MLA_ERR_CUDA;
   }
@@ -158,6 +168,12 @@ int mla_set_rope_scaling(mla_handle *h, double factor, int original_ctx, double 
   return MLA_OK;
 }
 
+int mla_set_strict(mla_handle *h, int strict) {
+  if (!h) return MLA_ERR_INVALID_ARG;
+  h->strict = strict ? 1 : 0;
+  return MLA_OK;
+}
+
 int mla_cache_append(mla_handle *h, const void *x, int B, int T, const int *start_pos,
                      const void *w_dkv, const void *w_kr, void *cache, long long cache_len,
                      const int *block_table, int max_blocks_per_seq, mla_stream_t stream) {
@@ -173,6 +189,7 @@ int mla_cache_append(mla_handle *h, const void *x, int B, int T, const int *star
   if (h->gemm_kind == kGemmTc)
     e = launch_append_tc(c, x, B, T, start_pos, w_dkv, w_kr, cache, cache_len, block_table,
                          max_blocks_per_seq, h->d_theta, h->d_status, s);
+  if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported)
     e = launch_append_simt(c, x, B, T, start_pos, w_dkv, w_kr, cache, cache_len, block_table,
                            max_blocks_per_seq, h->d_theta, h->d_status, s);
@@ -190,6 +207,7 @@ int mla_absorb_q(mla_handle *h, const void *q_nope, const void *q_rope, const in
   cudaError_t e = cudaErrorNotSupported;
   if (h->gemm_kind == kGemmTc)
     e = launch_absorb_tc(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, s);
+  if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported)
     e = launch_absorb_simt(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, s);
   if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
@@ -220,7 +238,11 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
   const WsLayout L = ws_layout(c, B, P);
   if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_plan(ctx_len, B, P, (char *)workspace, L, h->d_status, s);
+  // Tokens one sequence can address: the contiguous cache's capacity, or the
+  // pages of its block-table row.
+  const long long cap = c.page_size > 0 ? (long long)max_blocks_per_seq * c.page_size : cache_len;
+  const long long cap_i = cap < 0x7fffffffLL ? cap : 0x7fffffffLL;
+  cudaError_t e = launch_plan(ctx_len, B, P, cap_i, (char *)workspace, L, h->d_status, s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   AttnArgs a;
   a.q_abs = q_abs;
@@ -229,7 +251,6 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
   a.block_table = block_table;
   a.max_blocks = max_blocks_per_seq;
   a.page_size = c.page_size;
-  a.ctx_len = ctx_len;
   a.B = B;
   a.n_h = c.n_h;
   a.d_c = c.d_c;
@@ -245,6 +266,8 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
     e = launch_attn_tc_pair(a, P, s);
   else if (h->attn_kind == kAttnTcSmallH && aligned16(q_abs) && aligned16(cache))
     e = launch_attn_tc_smallh(a, P, s);
+  const bool tc_exists = (h->attn_kind == kAttnTcPair && !kv_scale) || h->attn_kind == kAttnTcSmallH;
+  if (strict_refuses(h, tc_exists, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported) e = launch_attn_simt(a, P, c.dtype == MLA_FP32, s);
   if (e == cudaErrorNotSupported) return MLA_ERR_UNSUPPORTED;
   return from_cuda(e);
@@ -296,6 +319,7 @@ int mla_cache_append_fp8(mla_handle *h, const void *x, int B, int T, const int *
   if (h->gemm_kind == kGemmTc)
     e = launch_append_tc(c, x, B, T, start_pos, w_dkv, w_kr, nullptr, 0, nullptr, 0, h->d_theta,
                          h->d_status, s, rows);
+  if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported)
     e = launch_append_simt(c, x, B, T, start_pos, w_dkv, w_kr, nullptr, 0, nullptr, 0, h->d_theta,
                            h->d_status, s, rows);
@@ -341,11 +365,13 @@ int mla_out_proj(mla_handle *h, const void *ctx_lat, const void *w_uv, const voi
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaErrorNotSupported;
   if (h->gemm_kind == kGemmTc) e = launch_outproj_tc(h->cfg, ctx_lat, w_uv, o, B, s);
+  if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported) e = launch_outproj_simt(h->cfg, ctx_lat, w_uv, o, B, s);
   if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
   if (w_o) {
     e = cudaErrorNotSupported;
     if (h->gemm_kind == kGemmTc) e = launch_wo_tc(h->cfg, o, w_o, u, B, s);
+    if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
     if (e == cudaErrorNotSupported) e = launch_wo_simt(h->cfg, o, w_o, u, B, s);
     if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
   }
@@ -359,6 +385,7 @@ cudaError_t linear(const mla_handle *h, const void *x, const void *w, void *y, i
                    cudaStream_t s) {
   cudaError_t e = cudaErrorNotSupported;
   if (h->gemm_kind == kGemmTc) e = launch_linear_tc(x, w, y, M, K, N, s);
+  if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return e;   // reported as MLA_ERR_UNSUPPORTED
   if (e == cudaErrorNotSupported) e = launch_linear_simt(x, w, y, M, K, N, h->cfg.dtype == MLA_FP32, s);
   return e;
 }

@@ -6,9 +6,15 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "mla.h"
 
 namespace mla {
+
+// Devices a process may drive (per-device launch set-up is kept per index).
+constexpr int kMaxDevices = 64;
 
 // KV tokens per tile; the split plan and every attention kernel work in whole
 // tiles, and the paged fast paths require page_size == kTile.
@@ -84,6 +90,8 @@ struct mla_handle {
   double score_mult;   // YaRN temperature t multiplying every score (1 without scaling)
   int attn_kind;       // mla::AttnKind
   int gemm_kind;       // mla::GemmKind
+  int strict;          // 1: no CUDA-core substitute for a tensor-core kernel (mla_set_strict)
+  void *noalloc_scratch;  // device address of the allocation-free entry point's array
 };
 
 namespace mla {
@@ -116,6 +124,7 @@ struct WsHeader {
 struct WsLayout {
   size_t tile_prefix_off;  // int64 [B+1]
   size_t piece_base_off;   // int64 [B+1]
+  size_t ctx_off;          // int32 [B]: each sequence's length as attended (clamped by the plan)
   size_t opart_off;        // float [max_pieces, n_h, d_c]
   size_t lse_off;          // float [max_pieces, n_h]
   size_t total;
@@ -132,6 +141,8 @@ inline WsLayout ws_layout(const mla_config &cfg, int B, int P) {
   off = align_up(off + sizeof(long long) * (size_t)(B + 1), 256);
   L.piece_base_off = off;
   off = align_up(off + sizeof(long long) * (size_t)(B + 1), 256);
+  L.ctx_off = off;
+  off = align_up(off + sizeof(int) * (size_t)(B > 0 ? B : 1), 256);
   L.opart_off = off;
   off = align_up(off + sizeof(float) * (size_t)L.max_pieces * cfg.n_h * cfg.d_c, 256);
   L.lse_off = off;
@@ -148,7 +159,6 @@ struct AttnArgs {
   const int *block_table;
   int max_blocks;
   int page_size;
-  const int *ctx_len;
   int B;
   int n_h, d_c, d_r;
   float scale_log2;  // log2(e) / sqrt(d_h + d_r)
@@ -164,8 +174,17 @@ struct AttnArgs {
 // ---------------------------------------------------------------------------
 // Launchers (return cudaGetLastError() of the launch).
 // ---------------------------------------------------------------------------
-cudaError_t launch_plan(const int *ctx_len, int B, int P, char *ws, const WsLayout &L,
+// The plan clamps every length to [0, cap] (cap: the tokens the cache can
+// address for one sequence), flags any length outside it in the status word,
+// and stores the clamped lengths in the workspace; every attention kernel reads
+// those instead of ctx_len, so that the plan's tiles and the kernels agree.
+cudaError_t launch_plan(const int *ctx_len, int B, int P, long long cap, char *ws, const WsLayout &L,
                         unsigned *status, cudaStream_t s);
+
+// The clamped length of sequence b, as the plan stored it.
+__device__ __forceinline__ int plan_ctx(const char *ws, const WsLayout &L, int b) {
+  return reinterpret_cast<const int *>(ws + L.ctx_off)[b];
+}
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s);
 cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
@@ -220,5 +239,27 @@ cudaError_t launch_wait_timeout_selftest(unsigned *status, unsigned long long li
 
 // Resolve the driver entry point for tensor-map encoding (no libcuda link).
 bool tma_available();
+
+// Device address, on the current device, of the fixed scratch array of the
+// allocation-free entry point (noalloc.cu).  MLA_OK or MLA_ERR_CUDA.
+int noalloc_scratch_lookup(void **out);
+
+// Once-per-device launch set-up (the dynamic shared-memory opt-in, which
+// applies per device): runs `fn` the first time it is called for the current
+// device and caches its result; concurrent callers wait for the first.
+template <typename Fn>
+cudaError_t once_per_device(std::atomic<int> (&state)[kMaxDevices], Fn fn) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
+  if (state[dev].load(std::memory_order_acquire) == 2) return cudaSuccess;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (state[dev].load(std::memory_order_relaxed) == 2) return cudaSuccess;
+  e = fn();
+  if (e == cudaSuccess) state[dev].store(2, std::memory_order_release);
+  return e;
+}
 
 }  // namespace mla

@@ -60,29 +60,35 @@ __device__ long long block_exclusive_scan(long long v, long long *smem, long lon
   return incl - v;
 }
 
-__global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, int P_req, char *ws,
-                                                    WsLayout L, unsigned *status) {
+__global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, int P_req, long long cap,
+                                                    char *ws, WsLayout L, unsigned *status) {
   pdl_trigger();
   pdl_wait();   // the workspace may still be read by the previous step's combine
   __shared__ long long scan[1024];
   long long *tile_prefix = reinterpret_cast<long long *>(ws + L.tile_prefix_off);
   long long *piece_base = reinterpret_cast<long long *>(ws + L.piece_base_off);
+  int *ctx_eff = reinterpret_cast<int *>(ws + L.ctx_off);
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (B + nt - 1) / nt;
   const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
 
   long long local = 0;
   for (int b = b0; b < b1; ++b) {
-    int c = ctx_len[b];
-    if (c < 0) { atomicOr(status, kStatusBounds); c = 0; }
+    // A length outside [0, cap] is flagged and clamped; the tiles below and
+    // every attention kernel use the clamped length.
+    long long c = ctx_len[b];
+    if (c < 0 || c > cap) {
+      atomicOr(status, kStatusBounds);
+      c = c < 0 ? 0 : cap;
+    }
+    ctx_eff[b] = (int)c;
     local += ceil_div_ll(c, kTile);
   }
   long long Ttot;
   long long run = block_exclusive_scan(local, scan, &Ttot);
   for (int b = b0; b < b1; ++b) {
     tile_prefix[b] = run;
-    int c = max(ctx_len[b], 0);
-    run += ceil_div_ll(c, kTile);
+    run += ceil_div_ll(ctx_eff[b], kTile);
   }
   if (tid == 0) tile_prefix[B] = Ttot;
   const long long P = Ttot < (long long)P_req ? Ttot : (long long)P_req;
@@ -90,7 +96,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, i
   long long local_pieces = 0;
   for (int b = b0; b < b1; ++b) {
     long long s = tile_prefix[b];
-    long long t = ceil_div_ll(max(ctx_len[b], 0), kTile);
+    long long t = ceil_div_ll(ctx_eff[b], kTile);
     if (t > 0) local_pieces += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
   long long n_pieces;
@@ -98,7 +104,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, i
   for (int b = b0; b < b1; ++b) {
     piece_base[b] = prun;
     long long s = tile_prefix[b];
-    long long t = ceil_div_ll(max(ctx_len[b], 0), kTile);
+    long long t = ceil_div_ll(ctx_eff[b], kTile);
     if (t > 0) prun += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
   if (tid == 0) {
@@ -161,11 +167,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
     const long long s1 = t1 < tp[b + 1] ? t1 : tp[b + 1];
     if (s0 >= s1) continue;
     const long long piece = pb[b] + (w - plan_share_of_tile(tp[b], P, Ttot));
-    int ctx = a.ctx_len[b];
-    if (a.page_size == 0 && ctx > a.cache_len) {
-      if (lane == 0) atomicOr(a.status, kStatusBounds);
-      ctx = (int)a.cache_len;
-    }
+    const int ctx = plan_ctx(a.ws, a.L, b);
     const long long p_begin = (s0 - tp[b]) * kTile;
     const long long p_end = min((long long)ctx, (s1 - tp[b]) * kTile);
 
@@ -430,9 +432,9 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const T *o, const T *w
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_plan(const int *ctx_len, int B, int P, char *ws, const WsLayout &L,
+cudaError_t launch_plan(const int *ctx_len, int B, int P, long long cap, char *ws, const WsLayout &L,
                         unsigned *status, cudaStream_t s) {
-  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_len, B, P, ws, L, status);
+  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_len, B, P, cap, ws, L, status);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s) {

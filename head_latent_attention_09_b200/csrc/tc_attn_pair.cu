@@ -56,6 +56,17 @@ constexpr int kQBytes = 9 * 8192;       // 64 heads x 576 bf16, nine 64-column c
 constexpr int kPBytes = 4 * 8192;       // 64 heads x 256 tokens bf16, four 64-token chunks
 constexpr float kRescale = 8.0f;        // rescale O only when the running max grows by > 2^8
 
+// L2 prefetch distance in pair tiles (0 = off) and the evict-first hint on a
+// row's last read (the column-split V staging).
+#ifndef MLA_PAIR_PREFETCH
+#define MLA_PAIR_PREFETCH 2
+#endif
+#ifndef MLA_PAIR_EVICT
+#define MLA_PAIR_EVICT 1
+#endif
+constexpr int kPrefetch = MLA_PAIR_PREFETCH;
+constexpr int kPrefetchRows = 32;       // rows per bulk prefetch (36 KB); 32 divides a 64-token page
+
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kOffQ + kQBytes;
 constexpr int kOffP = kOffRing + kSlots * kSlot;
@@ -133,8 +144,7 @@ __device__ __forceinline__ bool walk_next(Walk &w, const AttnArgs &a, int share,
     const long long s0 = w.t0 > w.tp[b] ? w.t0 : w.tp[b];
     const long long s1 = w.t1 < w.tp[b + 1] ? w.t1 : w.tp[b + 1];
     if (s0 >= s1) continue;
-    int ctx = a.ctx_len[b];
-    if (a.page_size == 0 && ctx > a.cache_len) ctx = (int)a.cache_len;
+    const int ctx = plan_ctx(a.ws, a.L, b);
     pc.b = b;
     pc.piece = w.pb[b] + (share - plan_share_of_tile(w.tp[b], w.P, w.Ttot));
     pc.tok_begin = (int)((s0 - w.tp[b]) * kTile);
@@ -277,6 +287,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     Walk w;
     walk_init(w, a, share);
+    // L2 prefetch of the rows kPrefetch tiles ahead of the tile whose K chunks
+    // are being loaded (tiles counted across the share's pieces): this CTA's
+    // token half of each tile, the peer prefetching the other.  HBM latency is
+    // then covered by the prefetch distance, which takes no shared memory, and
+    // the ring's TMA loads only wait for L2.  Lane 0 of warp 6 issues.
+    Walk pw;
+    walk_init(pw, a, share);
+    Piece ppc;
+    int pk = 0;
+    bool pvalid = kPrefetch > 0 && walk_next(pw, a, share, ppc);
+    const char *cache_bytes = reinterpret_cast<const char *>(a.cache);
+    auto prefetch_next = [&]() {
+      if (!pvalid) return;
+      if (pid == 1 && lane == 0) {
+        const int ts = ppc.tok_begin + kTileTok * pk + kHalfTok * (int)rank;
+        const int te = min(ts + kHalfTok, ppc.tok_end);
+        for (int t = ts; t < te; t += kPrefetchRows) {
+          const int n = min(kPrefetchRows, te - t);
+          const long long r = kv_row(a, ppc.b, t);   // a run of n rows never crosses a page
+          if (r >= 0) ptx::bulk_prefetch_l2(cache_bytes + r * 1152, (uint32_t)n * 1152u);
+        }
+      }
+      if (++pk >= ppc.ntiles) {
+        pk = 0;
+        pvalid = walk_next(pw, a, share, ppc);
+      }
+    };
+    for (int d = 0; d < kPrefetch; ++d) prefetch_next();
+#if MLA_PAIR_EVICT
+    const uint64_t last_read = ptx::l2_policy_evict_first();
+#endif
     Piece pc, vpc;            // vpc/vt0: the tile whose V sub-stages are pending
     int vt0 = 0;
     bool vpending = false;
@@ -344,8 +385,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int y = block_row(a, p, tok0, kv_rows);
             if (leader) ptx::mbar_arrive_expect_tx(bars.full(s), 2 * kSlot);
             const int feat0 = 256 * g + 128 * (int)rank;
+#if MLA_PAIR_EVICT
+            ptx::tma_load_2d_pair_hint(dst, &mapV, lf0 + 8 * s, feat0, y, last_read);
+            ptx::tma_load_2d_pair_hint(dst + 8192, &mapV, lf0 + 8 * s, feat0 + 64, y, last_read);
+#else
             ptx::tma_load_2d_pair(dst, &mapV, lf0 + 8 * s, feat0, y);
             ptx::tma_load_2d_pair(dst + 8192, &mapV, lf0 + 8 * s, feat0 + 64, y);
+#endif
           }
           ++sc;
         }
@@ -364,6 +410,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!__shfl_sync(0xffffffffu, qok ? 1 : 0, 0)) break;
       for (int k = 0; k < pc.ntiles && ok; ++k) {
+        prefetch_next();
         // K chunks of this tile: this CTA's 128 tokens x 64 columns each.
         const int t0 = pc.tok_begin + kTileTok * k;
         const int tr = t0 + kHalfTok * (int)rank;
@@ -650,12 +697,11 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
       !encode_map_bf16(&mk, a.cache, 2, dkv, st, boxk, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_map_bf16(&mv, a.cache, 2, dkv, st, boxv, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = once_per_device(configured, [] {
+    return cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  });
+  if (e != cudaSuccess) return e;
   return launch_pdl(attn_pair_kernel, dim3(2 * P), dim3(kThreads), kSmemAlloc, s, 1, mq, mk, mv, a, rows);
 }
 

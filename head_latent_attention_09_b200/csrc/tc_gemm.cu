@@ -448,16 +448,11 @@ cudaError_t launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUte
   const size_t smem = 1024 + region + smem_tail<BN>();
   if (smem > kSmemLimit) return cudaErrorNotSupported;
   auto kern = gemm_tc_kernel<BN, A_MN>;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = once_per_device(configured, [kern] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+  });
   if (e != cudaSuccess) return e;
-  static bool configured[64] = {};
-  if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
   const int groups = (mtiles + g.mt_per_cta - 1) / g.mt_per_cta;
   const dim3 grid(groups * g.ksplit, ntiles, nz);
   return launch_pdl(kern, grid, dim3(kGemmThreads), smem, s, g.ksplit, a0, a1, b, g);

@@ -100,8 +100,11 @@ const char *mla_status_string(int status);
 int mla_config_validate(const mla_config *cfg);
 
 /* Create a handle on the current CUDA device.  Allocates the status word and
- * the RoPE frequency table (theta_k in double precision).  On failure *out is
- * NULL.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+ * the RoPE frequency table (theta_k in double precision), and looks up the
+ * device address of the scratch array that mla_decode_attn_combine_noalloc
+ * uses (that lookup loads the part of the library's device image holding the
+ * array, which is when the array's memory is reserved on this device).  On
+ * failure *out is NULL.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 int mla_create(const mla_config *cfg, mla_handle **out);
 
 /* Release a handle (synchronises nothing; the caller must not have work in
@@ -127,6 +130,19 @@ void mla_destroy(mla_handle *handle);
  * current device), CUDA. */
 int mla_set_rope_scaling(mla_handle *handle, double factor, int original_ctx, double alpha,
                          double beta, double mscale_coef);
+
+/* Strict tensor-core mode (off by default).  A bf16 configuration of the
+ * DeepSeek-V2 attention shapes runs its append, absorption, attention, output
+ * projection and query projection on tcgen05 kernels; when one of those
+ * kernels cannot take a call's arguments (a pointer that is not 16-byte
+ * aligned, a cache of 2^31 rows or more, a tensor map the driver rejects) the
+ * call normally runs the CUDA-core kernel instead, with the same results.
+ * With strict mode on, such a call returns MLA_ERR_UNSUPPORTED before
+ * launching anything.  Calls for which the configuration has no tensor-core
+ * kernel at all (fp32, other shapes, the FP8 cache at 128 heads) are not
+ * affected.  Meant for tests and benchmarks that must run the tensor-core
+ * path.  Errors: INVALID_ARG (NULL handle). */
+int mla_set_strict(mla_handle *handle, int strict);
 
 /* Cache append (V3 note, MLA equations: c^KV_t = W^DKV h_t, k^R_t = RoPE(W^KR h_t);
  * V2 §2.1.3: the cached row is [c^KV_t ; k^R_t]).
@@ -183,7 +199,12 @@ int mla_default_num_parts(const mla_handle *handle);
  * heads) and yields, per (sequence, share) piece, the normalised partial
  * ctx_lat and its log-sum-exp, written into the workspace.
  *   q_abs   [B, n_h, d_c+d_r] absorbed queries
- *   ctx_len device int32 [B], ctx_len[b] tokens of sequence b are attended
+ *   ctx_len device int32 [B], ctx_len[b] tokens of sequence b are attended.
+ *           A length below 0 or above what the cache can address for one
+ *           sequence (cache_len for a contiguous cache, max_blocks_per_seq *
+ *           page_size for a paged one) sets MLA_ERR_DEVICE_BOUNDS in the status
+ *           word and is clamped to that range, for the split plan and for the
+ *           attention alike.
  *   workspace >= mla_decode_workspace_size(handle, B, num_parts) bytes, 256-byte
  *   aligned, device memory; its contents are overwritten. */
 int mla_decode_attn(mla_handle *handle, const void *q_abs, const void *cache, long long cache_len,
@@ -237,9 +258,12 @@ long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *p
  *   num_parts = 0 picks the default split count, lowered until the partials
  *   fit the array; an explicit num_parts (or a batch) whose partials do not
  *   fit is rejected with MLA_ERR_WORKSPACE before anything is launched.
- * No cudaMalloc/cudaFree or allocating library call is made.  The first call
- * on a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.
+ * No cudaMalloc/cudaFree or allocating library call is made.  The array's
+ * device address is looked up once, by mla_create on the handle's device
+ * (cudaGetSymbolAddress with that device current); that lookup is also what
+ * loads the array onto the device, so creating the handle is the step that
+ * reserves its memory, and this call itself allocates nothing.  The handle's
+ * device must be current.
  * All calls share the array and leave their partials in it; calls whose work
  * overlaps on the GPU (unordered streams) race on it.  The array needs no
  * zeroing: each call writes everything it reads. */

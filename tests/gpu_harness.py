@@ -49,15 +49,28 @@ def rope_arg(wl):
                       mscale_coef=coef)
 
 
-def create_handle(wl) -> int:
-    """mla_create for the workload, with its RoPE scaling applied."""
+def strict_on(handle, wl, strict=None):
+    """Strict tensor-core mode for bf16 workloads (strict=None): a call whose
+    tensor-core kernel cannot take its arguments then fails instead of
+    silently running the CUDA-core kernel, so a passing bf16 parity test shows
+    that the tensor-core path ran."""
+    if strict is None:
+        strict = wl.dtype == "bf16"
+    M.mla_set_strict(handle, 1 if strict else 0)
+    return handle
+
+
+def create_handle(wl, strict=None) -> int:
+    """mla_create for the workload, with its RoPE scaling applied and strict
+    tensor-core mode on for bf16 (see strict_on)."""
     handle = M.mla_create(config_of(wl))
-    if wl.rope_scaling is not None:
-        try:
+    try:
+        if wl.rope_scaling is not None:
             M.mla_set_rope_scaling(handle, *wl.rope_scaling)
-        except Exception:
-            M.mla_destroy(handle)
-            raise
+        strict_on(handle, wl, strict)
+    except Exception:
+        M.mla_destroy(handle)
+        raise
     return handle
 
 

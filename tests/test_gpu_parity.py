@@ -17,8 +17,8 @@ import torch
 
 import head_latent_attention_09_b200 as M
 from oracle import mla_oracle as O
-from tests.gpu_harness import (compare, config_of, oracle_step, run_decode_step, to_dev, to_host,
-                               torch_dtype)
+from tests.gpu_harness import (compare, config_of, oracle_step, run_decode_step, strict_on, to_dev,
+                               to_host, torch_dtype)
 from workloads import WORKLOADS, ctx_lengths, random_cache
 
 pytestmark = pytest.mark.gpu
@@ -122,6 +122,7 @@ def _attention_only(wl, ctx, parts, q_scale=0.5, cache_std=1.0, plant=None):
     cfg = config_of(wl)
     handle = M.mla_create(cfg)
     try:
+        strict_on(handle, wl)
         ctx = np.asarray(ctx)
         B, T = len(ctx), int(max(1, ctx.max()))
         w2 = wl.with_(B=B)
@@ -186,3 +187,129 @@ def test_attention_late_dominant_key(name):
     gc, gl, wc, wlse = _attention_only(wl, ctx, 7, plant=plant)
     compare(gc, wc, wl, "ctx_lat dominant", [0, 1])
     compare(gl, wlse, wl, "lse dominant", [0, 1])
+
+
+# ---------------------------------------------------------------------------
+# lengths the cache cannot hold, and strict tensor-core mode
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k", "tiny_fp32"])
+def test_length_past_the_cache_is_flagged_and_clamped(name):
+    """ctx_len = cache_len + 1 (contiguous cache): the call flags
+    MLA_ERR_DEVICE_BOUNDS and attends the cache_len tokens that exist, in the
+    split plan and in the attention kernel alike (each kernel kind)."""
+    wl = WORKLOADS[name]
+    T = 300
+    ctx = np.array([T + 1, 5, T, 0])
+    B = len(ctx)
+    handle = M.mla_create(config_of(wl))
+    try:
+        strict_on(handle, wl)
+        rows = random_cache(wl.with_(B=B), T, 1.0)
+        rng = np.random.default_rng(77)
+        q = rng.standard_normal((B, wl.n_h, wl.D)).astype(np.float32) * 0.5
+        from workloads import bf16_round
+        if wl.dtype == "bf16":
+            q = bf16_round(q)
+        cache, q_d = to_dev(rows, wl), to_dev(q, wl)
+        ctx_d = torch.from_numpy(ctx.astype(np.int32)).cuda()
+        for parts in (0, 3):
+            P = parts or M.mla_default_num_parts(handle)
+            ws_bytes = M.mla_decode_workspace_size(handle, B, P)
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+            out = torch.empty((B, wl.n_h, wl.d_c), dtype=torch_dtype(wl), device="cuda")
+            lse = torch.empty((B, wl.n_h), dtype=torch.float32, device="cuda")
+            M.mla_decode_attn(handle, q_d, cache, T, None, 0, ctx_d, B, P, ws, ws_bytes)
+            M.mla_combine_splits(handle, ws, ws_bytes, B, P, out, lse)
+            assert M.mla_get_device_status(handle) == M.MLA_ERR_DEVICE_BOUNDS
+            assert M.mla_get_device_status(handle) == M.MLA_OK       # read and cleared
+            got_c, got_l = to_host(out), to_host(lse)
+            scale = O.softmax_scale(wl.d_h, wl.d_r)
+            want_c, want_l = {}, {}
+            for b in range(3):
+                n = min(int(ctx[b]), T)
+                want_c[b], want_l[b] = O.latent_attention(q[b], rows[b, :n], d_c=wl.d_c, scale=scale)
+            compare(got_c, want_c, wl, f"ctx_lat clamped, parts={P}", [0, 1, 2])
+            compare(got_l, want_l, wl, f"lse clamped, parts={P}", [0, 1, 2])
+            assert np.all(got_c[3] == 0) and np.all(np.isneginf(got_l[3]))
+    finally:
+        M.mla_destroy(handle)
+
+
+def test_paged_length_past_the_block_table_is_flagged_and_clamped():
+    wl = WORKLOADS["v2lite_paged_ragged_b128"]
+    ps = wl.page_size
+    max_blk = 3
+    ctx = np.array([max_blk * ps + 10, 70])
+    B = len(ctx)
+    handle = M.mla_create(config_of(wl))
+    try:
+        strict_on(handle, wl)
+        n_pool = B * max_blk
+        pool_rows = random_cache(wl.with_(B=1), n_pool * ps, 1.0)[0]
+        perm = np.random.default_rng(5).permutation(n_pool).astype(np.int32)
+        table = perm.reshape(B, max_blk)
+        rng = np.random.default_rng(78)
+        from workloads import bf16_round
+        q = bf16_round(rng.standard_normal((B, wl.n_h, wl.D)).astype(np.float32) * 0.5)
+        pool = to_dev(pool_rows.reshape(n_pool, ps, wl.D), wl)
+        q_d = to_dev(q, wl)
+        tbl = torch.from_numpy(table).cuda()
+        ctx_d = torch.from_numpy(ctx.astype(np.int32)).cuda()
+        P = M.mla_default_num_parts(handle)
+        ws_bytes = M.mla_decode_workspace_size(handle, B, P)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        out = torch.empty((B, wl.n_h, wl.d_c), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B, wl.n_h), dtype=torch.float32, device="cuda")
+        M.mla_decode_attn(handle, q_d, pool, n_pool, tbl, max_blk, ctx_d, B, P, ws, ws_bytes)
+        M.mla_combine_splits(handle, ws, ws_bytes, B, P, out, lse)
+        assert M.mla_get_device_status(handle) == M.MLA_ERR_DEVICE_BOUNDS
+        got_c, got_l = to_host(out), to_host(lse)
+    finally:
+        M.mla_destroy(handle)
+    scale = O.softmax_scale(wl.d_h, wl.d_r)
+    flat = pool_rows.reshape(n_pool, ps, wl.D)
+    want_c, want_l = {}, {}
+    for b in range(B):
+        n = min(int(ctx[b]), max_blk * ps)
+        seq = np.concatenate([flat[table[b, j]] for j in range(max_blk)])[:n]
+        want_c[b], want_l[b] = O.latent_attention(q[b], seq, d_c=wl.d_c, scale=scale)
+    compare(got_c, want_c, wl, "ctx_lat clamped (paged)", [0, 1])
+    compare(got_l, want_l, wl, "lse clamped (paged)", [0, 1])
+
+
+def test_strict_mode_refuses_instead_of_substituting():
+    """With strict mode on, arguments the tensor-core kernels cannot take (a
+    pointer that is not 16-byte aligned) make the call fail before any launch
+    instead of running the CUDA-core kernel."""
+    wl = WORKLOADS["v2_b64_ctx8k"]
+    B = 2
+    handle = M.mla_create(config_of(wl))
+    try:
+        M.mla_set_strict(handle, 1)
+        bf = torch.bfloat16
+        buf = torch.zeros(B * wl.n_h * wl.D + 64, dtype=bf, device="cuda")
+        odd = buf.data_ptr() + 2                       # 2-byte aligned only
+        cache = torch.zeros((B, 64, wl.D), dtype=bf, device="cuda")
+        ctx_d = torch.full((B,), 64, dtype=torch.int32, device="cuda")
+        ws_bytes = M.mla_decode_workspace_size(handle, B, 0)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        with pytest.raises(M.MlaError) as err:
+            M.mla_decode_attn(handle, odd, cache, 64, None, 0, ctx_d, B, 0, ws, ws_bytes)
+        assert err.value.status == M.MLA_ERR_UNSUPPORTED
+        q_nope = torch.zeros((B, wl.n_h, wl.d_h), dtype=bf, device="cuda")
+        q_rope = torch.zeros((B, wl.n_h, wl.d_r), dtype=bf, device="cuda")
+        w_uk = torch.zeros((wl.n_h * wl.d_h, wl.d_c), dtype=bf, device="cuda")
+        pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+        q_abs = torch.empty((B, wl.n_h, wl.D), dtype=bf, device="cuda")
+        with pytest.raises(M.MlaError) as err:
+            M.mla_absorb_q(handle, odd, q_rope, pos, w_uk, q_abs, B)
+        assert err.value.status == M.MLA_ERR_UNSUPPORTED
+        o = torch.empty((B, wl.n_h, wl.d_h), dtype=bf, device="cuda")
+        with pytest.raises(M.MlaError) as err:
+            M.mla_out_proj(handle, odd, w_uk, None, o, None, B)
+        assert err.value.status == M.MLA_ERR_UNSUPPORTED
+        torch.cuda.synchronize()
+        assert M.mla_get_device_status(handle) == M.MLA_OK
+    finally:
+        M.mla_destroy(handle)

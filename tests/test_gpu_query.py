@@ -42,8 +42,8 @@ def _hidden(wl):
     return np.stack([hidden_states(wl, b, b + 1)[-1] for b in range(wl.B)])
 
 
-def _run(wl, x, qw):
-    handle = create_handle(wl)
+def _run(wl, x, qw, strict):
+    handle = create_handle(wl, strict=strict)
     try:
         dt = torch_dtype(wl)
         w = {k: to_dev(v, wl) for k, v in qw.items()}
@@ -75,10 +75,10 @@ def _close(got, want, rtol, atol, what):
     return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30))
 
 
-def _check(wl):
+def _check(wl, strict=None):
     qw = draw_query_weights(wl)
     x = _hidden(wl)
-    c_q, q_nope, q_rope = _run(wl, x, qw)
+    c_q, q_nope, q_rope = _run(wl, x, qw, strict)
     H, dh, dr = wl.n_h, wl.d_h, wl.d_r
     chain = [O.query_from_hidden(x[b], qw, H, dh, dr) for b in range(wl.B)]
     if wl.dtype == "fp32":
@@ -118,7 +118,8 @@ def _check(wl):
 ])
 def test_query_proj_matches_oracle(name, B, over):
     wl = WORKLOADS[name].with_(B=B, ctx=(1,) * B, **over)
-    _check(wl)
+    # the overridden shapes run (part of) the projection on CUDA cores by design
+    _check(wl, strict=False if over else None)
 
 
 def test_query_proj_empty_batch_and_bad_arguments():
