@@ -47,6 +47,13 @@ def parse():
                     help="skip the separate timing of the query projection")
     ap.add_argument("--no-fp8", action="store_true",
                     help="skip the separate timing of attention over an FP8 cache")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the separate timings of the other workloads (V2-Lite, ragged paged, 128K)")
+    ap.add_argument("--attn-samples", type=int, default=200,
+                    help="attention calls timed one by one for the median and p10/p90")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="only start the ranks, join the process group (gloo without a GPU) and "
+                         "report the ranks seen; no GPU work")
     return ap.parse_args()
 
 
@@ -360,6 +367,120 @@ def measure_fp8(M, dev, steps, seed):
             "bf16_bytes": tokens * D * 2, "fp8_bytes": fp8_cache_bytes(tokens, D, G)}
 
 
+EXTRA_WORKLOADS = ("v2lite_b32_ctx4k", "v2lite_paged_ragged_b128", "v2lite_b4_ctx128k")
+
+
+def measure_workload(M, wl, dev, steps, seed, hbm_peak, n_samples=100):
+    """The decode step (append, absorb, attention, combine, output projection)
+    and the attention call alone on another workload's shapes, with its own
+    cache filled through mla_cache_append from random hidden states.  A cache
+    smaller than twice L2 is kept in two copies used alternately, so that
+    every step reads its cache from HBM.  Returns times (µs), the algorithmic
+    bytes and the roofline fraction of the attention call."""
+    import torch
+    from workloads import block_table, ctx_lengths
+    B, H, D, d = wl.B, wl.n_h, wl.D, wl.d_model
+    ctx = ctx_lengths(wl)
+    cfg = M.mla_config(n_h=H, d_h=wl.d_h, d_c=wl.d_c, d_r=wl.d_r, d_model=d, page_size=wl.page_size,
+                       rope_base=wl.rope_base, dtype=M.MLA_BF16)
+    handle = M.mla_create(cfg)
+    try:
+        M.mla_set_strict(handle, 1)
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        bf = torch.bfloat16
+
+        def randn(*shape, std=1.0):
+            return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(bf)
+
+        w_dkv = randn(wl.d_c, d, std=d ** -0.5)
+        w_kr = randn(wl.d_r, d, std=d ** -0.5)
+        w_uk = randn(H * wl.d_h, wl.d_c, std=wl.d_c ** -0.5)
+        w_uv = randn(H * wl.d_h, wl.d_c, std=wl.d_c ** -0.5)
+        tokens = int(ctx.sum())
+        cache_bytes = tokens * D * 2
+        props = torch.cuda.get_device_properties(dev)
+        l2 = int(getattr(props, "L2_cache_size", 126 << 20) or (126 << 20))
+        copies = 2 if cache_bytes < 2 * l2 else 1
+        if wl.page_size:
+            table_np, pool = block_table(wl, ctx)
+            table = torch.from_numpy(table_np).to(dev)
+            max_blk, cap = table_np.shape[1], pool
+            caches = [torch.empty((pool, wl.page_size, D), dtype=bf, device=dev) for _ in range(copies)]
+        else:
+            table, max_blk = None, 0
+            cap = int(ctx.max())
+            caches = [torch.empty((B, cap, D), dtype=bf, device=dev) for _ in range(copies)]
+        chunk = 4096
+        for c in caches:
+            for b in range(B):
+                n = int(ctx[b]) - 1
+                for t0 in range(0, n, chunk):
+                    t1 = min(n, t0 + chunk)
+                    sp = torch.tensor([t0], dtype=torch.int32, device=dev)
+                    if wl.page_size:
+                        M.mla_cache_append(handle, randn(t1 - t0, d), 1, t1 - t0, sp, w_dkv, w_kr, c, cap,
+                                           table.data_ptr() + 4 * b * max_blk, max_blk)
+                    else:
+                        M.mla_cache_append(handle, randn(t1 - t0, d), 1, t1 - t0, sp, w_dkv, w_kr,
+                                           c.data_ptr() + 2 * b * cap * D, cap)
+        h_new = randn(B, 1, d)
+        q_nope = randn(B, H, wl.d_h)
+        q_rope = randn(B, H, wl.d_r)
+        pos = torch.from_numpy((ctx - 1).astype(np.int32)).to(dev)
+        ctx_d = torch.from_numpy(ctx.astype(np.int32)).to(dev)
+        q_abs = torch.empty((B, H, D), dtype=bf, device=dev)
+        ctx_lat = torch.empty((B, H, wl.d_c), dtype=bf, device=dev)
+        o = torch.empty((B, H, wl.d_h), dtype=bf, device=dev)
+        P = M.mla_default_num_parts(handle)
+        ws_bytes = M.mla_decode_workspace_size(handle, B, P)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        stream = torch.cuda.current_stream()
+        sh = stream.cuda_stream
+
+        def step(i):
+            c = caches[i % copies]
+            M.mla_cache_append(handle, h_new, B, 1, pos, w_dkv, w_kr, c, cap, table, max_blk, sh)
+            M.mla_absorb_q(handle, q_nope, q_rope, pos, w_uk, q_abs, B, sh)
+            M.mla_decode_attn(handle, q_abs, c, cap, table, max_blk, ctx_d, B, P, ws, ws_bytes, sh)
+            M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, None, sh)
+            M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        step_us = t0.elapsed_time(t1) * 1e3 / steps
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_samples)]
+        for i, e in enumerate(ev):
+            c = caches[i % copies]
+            e[0].record(stream)
+            M.mla_decode_attn(handle, q_abs, c, cap, table, max_blk, ctx_d, B, P, ws, ws_bytes, sh)
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        st = M.mla_get_device_status(handle, sh)
+        if st != M.MLA_OK:
+            raise M.MlaError(st, f"device status after the {wl.name} timing")
+        t = np.array([e[0].elapsed_time(e[1]) * 1e3 for e in ev])
+    finally:
+        M.mla_destroy(handle)
+    med = float(np.median(t))
+    gbs = cache_bytes / (med * 1e-6) / 1e9
+    w_bytes = ((wl.d_c + wl.d_r) * d + 2 * H * wl.d_h * wl.d_c) * 2
+    return {"B": B, "n_h": H, "tokens": tokens, "page_size": wl.page_size, "cache_bytes": cache_bytes,
+            "cache_copies": copies, "num_parts": P, "us_per_step": step_us,
+            "step_gbs": (cache_bytes + w_bytes) / (step_us * 1e-6) / 1e9,
+            "attn_median_us": med, "attn_p10_us": float(np.percentile(t, 10)),
+            "attn_p90_us": float(np.percentile(t, 90)), "attn_gbs": gbs, "attn_frac": gbs / hbm_peak,
+            "tokens_scanned_per_s": tokens / (med * 1e-6), "attn_us_at_70pct_of_8TBps": cache_bytes / 5.6e3,
+            "bound": "hbm"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -371,6 +492,8 @@ def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} rank(s) were started")
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
@@ -498,6 +621,21 @@ def run_ours(args):
     names = ["cache_append", "absorb_q", "decode_attn", "combine_splits", "out_proj"]
     per_call = {n: float(np.mean([ev[j].elapsed_time(ev[j + 1]) for ev in call_ev])) * 1e3
                 for j, n in enumerate(names)}
+
+    # ---- the attention call alone, timed one call at a time (the latent
+    # cache is larger than L2, so every call reads it from HBM): median and
+    # spread of the roofline kernel's time.
+    n_s = max(args.attn_samples, 1)
+    s_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_s)]
+    for i in range(n_s):
+        s_ev[i][0].record(stream)
+        M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, ctx_d, B, P, ws, ws_bytes, sh)
+        s_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    attn_samples_us = np.array([e[0].elapsed_time(e[1]) * 1e3 for e in s_ev])
+    st = M.mla_get_device_status(handle, sh)
+    if st != M.MLA_OK:
+        raise M.MlaError(st, "device status after the attention samples")
 
     # ---- the query projection from the hidden state (upstream of the step):
     # its weights fit in L2, so a buffer larger than L2 is written before every
@@ -635,6 +773,15 @@ def run_ours(args):
     if not args.no_fp8 and rank == 0:
         fp8 = measure_fp8(M, dev, args.steps, rank_seed(rank) + 17)
 
+    # ---- the other workloads (rank 0 only): V2-Lite, ragged paged, 128K
+    configs = None
+    if not args.no_configs and rank == 0 and not args.batch:
+        hbm_peak_, _, _ = peaks()
+        configs = {}
+        for name in EXTRA_WORKLOADS:
+            configs[name] = measure_workload(M, WORKLOADS[name], dev, args.steps, rank_seed(rank) + 29,
+                                             hbm_peak_, n_samples=min(n_s, 100))
+
     # ---- reduce over ranks: max time
     ms, attn_ms, e2e_ms, e2e_serial_ms = reduce_max_over_ranks([ms, attn_ms, e2e_ms, e2e_serial_ms],
                                                                world, dev)
@@ -680,6 +827,16 @@ def run_ours(args):
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "mode": e2e_mode, "serial_ms_per_step": e2e_serial_ms,
                 "serial_value": whole_job_gbs(step_bytes, world, e2e_serial_ms)},
+        "steps_per_s": world * 1e3 / ms,
+        "tokens_scanned_per_s": world * ctx_sum / (ms * 1e-3),
+        "attention_samples": {
+            "n": int(attn_samples_us.size), "median_us": float(np.median(attn_samples_us)),
+            "p10_us": float(np.percentile(attn_samples_us, 10)),
+            "p90_us": float(np.percentile(attn_samples_us, 90)),
+            "median_gbs": attn_bytes / (float(np.median(attn_samples_us)) * 1e-6) / 1e9,
+            "median_frac": attn_bytes / (float(np.median(attn_samples_us)) * 1e-6) / 1e9 / hbm_peak,
+            "tokens_scanned_per_s": ctx_sum / (float(np.median(attn_samples_us)) * 1e-6),
+            "note": "mla_decode_attn alone, one call per event pair, after the timed region"},
         "gpu_launches": 6 * args.steps,
         "per_call_us": per_call,
         "per_call_note": "separate pass after the timed region, events between all calls",
@@ -697,6 +854,8 @@ def run_ours(args):
             "fp8_frac": fp8_gbs / hbm_peak, "bf16_achieved_gbs": bf16_gbs,
             "bf16_frac": bf16_gbs / hbm_peak, "bound": "hbm",
             "note": "mla_decode_attn_fp8 vs mla_decode_attn on the same cache; not part of the step"}
+    if configs is not None:
+        line["configs"] = configs
     if qproj is not None:
         gbs = qproj["bytes"] / (qproj["us"] * 1e-6) / 1e9
         line["query_proj"] = {
@@ -706,9 +865,55 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+def rank_launch_command(args_gpus: int, argv, port: int):
+    """The command that runs this script as `args_gpus` ranks on one node, one
+    process per GPU (torch.distributed.run, rendezvous on 127.0.0.1), with the
+    same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={args_gpus}", "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_check(args):
+    """Join the process group the ranks were started with and report the
+    ranks seen (rank 0 prints one JSON line)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    backend = "nccl" if torch.cuda.is_available() and torch.cuda.device_count() >= world else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    ranks = [None] * world
+    dist.all_gather_object(ranks, rank)
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "world": world, "ranks": sorted(ranks),
+                          "backend": backend}), flush=True)
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # Started as a plain process: start the ranks ourselves, one per GPU.
+        import subprocess
+        cmd = rank_launch_command(args.gpus, sys.argv[1:], _free_port())
+        sys.exit(subprocess.call(cmd))
+    if args.launch_check:
+        launch_check(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -140,11 +140,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
       : "memory");
 }
 
-// Bulk prefetch of `bytes` (a multiple of 16) at a 16-byte-aligned global
-// address into L2; no shared memory, no completion to wait for.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 // L2 policy that marks lines for early eviction (the last read of a tile).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
@@ -291,13 +286,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
       "l"(m), "r"(leader_bar), "r"(x), "r"(y)
       : "memory");
 }
-// The same with an L2 cache policy (e.g. evict-first for a tile's last read).
-__device__ __forceinline__ void tma_load_2d_pair_hint(void *dst, const CUtensorMap *m, uint32_t leader_bar,
-                                                      int x, int y, uint64_t policy) {
+__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *m, uint32_t leader_bar, int x, int y,
+                                                 int z) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
           "r"(smem_u32(dst)),
-      "l"(m), "r"(leader_bar), "r"(x), "r"(y), "l"(policy)
+      "l"(m), "r"(leader_bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair_hint(void *dst, const CUtensorMap *m, uint32_t leader_bar, int x,
+                                                      int y, int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::
+          "r"(smem_u32(dst)),
+      "l"(m), "r"(leader_bar), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {

@@ -47,6 +47,14 @@ namespace mla {
 namespace {
 
 constexpr int kThreads = 224;
+// TMA producer warps 0 and 6.  A thread that issues cp.async.bulk.tensor
+// copies sustains about two copies per microsecond (about 31 GB/s of 16 KB
+// boxes, measured, from L2 or HBM alike), so two threads issue: each owns the
+// ring slots s with s % 2 == its index.  Warp 0 also loads Q.  (A third
+// producer warp measured slightly slower: it shares a sub-partition with a
+// softmax warp.)
+constexpr int kProducers = 2;
+__device__ __forceinline__ int producer_index(int warp) { return warp == 0 ? 0 : (warp == 6 ? 1 : -1); }
 constexpr int kTileTok = 256;           // tokens per pair tile (MMA N of S = Q K^T)
 constexpr int kHalfTok = 128;           // tokens of a tile each CTA stages for S
 constexpr int kSubTok = 64;             // tokens per O += P V sub-stage
@@ -56,16 +64,10 @@ constexpr int kQBytes = 9 * 8192;       // 64 heads x 576 bf16, nine 64-column c
 constexpr int kPBytes = 4 * 8192;       // 64 heads x 256 tokens bf16, four 64-token chunks
 constexpr float kRescale = 8.0f;        // rescale O only when the running max grows by > 2^8
 
-// L2 prefetch distance in pair tiles (0 = off) and the evict-first hint on a
-// row's last read (the column-split V staging).
-#ifndef MLA_PAIR_PREFETCH
-#define MLA_PAIR_PREFETCH 2
-#endif
+// The evict-first L2 hint on a row's last read (the column-split V staging).
 #ifndef MLA_PAIR_EVICT
 #define MLA_PAIR_EVICT 1
 #endif
-constexpr int kPrefetch = MLA_PAIR_PREFETCH;
-constexpr int kPrefetchRows = 32;       // rows per bulk prefetch (36 KB); 32 divides a 64-token page
 
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kOffQ + kQBytes;
@@ -216,7 +218,8 @@ __device__ __forceinline__ int tile_subs(const Piece &p, int t0) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                     const __grid_constant__ CUtensorMap mapV, const AttnArgs a, const long long kv_rows) {
+                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapV2,
+                     const AttnArgs a, const long long kv_rows) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + kOffQ;
@@ -265,56 +268,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // the query and the cache it wrote are read.
   pdl_wait();
 
-  if (warp == 0 || warp == 6) {
+  if (producer_index(warp) >= 0) {
     // -------------------------------------------------------------- producers
     // Fill the ring in the order the MMAs consume it: the nine K chunks of
     // tile i, then the V sub-stages of tile i-1 (tiles counted across the
-    // share's pieces).  Job j goes to slot j % kSlots; warp 0 owns the even
-    // slots and warp 6 the odd ones, so two warps keep TMA loads in flight at
-    // once (one issuing warp tops out near 40 GB/s per SM), while every slot
-    // still has one producer that visits its jobs in order: its empty barrier
-    // is never more than one phase behind the phase waited for (a parity wait
-    // cannot tell one phase behind from three).  Lane 0 issues TMA; the
+    // share's pieces).  Job j goes to slot j % kSlots, owned by producer
+    // (j % kSlots) % kProducers, so two threads keep TMA loads in flight at
+    // once, while every slot still has one producer that visits its jobs in
+    // order: its empty barrier is never more than one phase behind the phase
+    // waited for (a parity wait cannot tell one phase behind from three).  Lane 0 issues TMA; the
     // leader arms each slot with the bytes both CTAs' loads bring (the peer's
     // loads count on the leader's barrier directly).  Warp 0 also loads Q.
-    const int pid = warp == 0 ? 0 : 1;
+    const int pid = producer_index(warp);
     const uint32_t lq = ptx::leader_addr(bars.qfull());
     const uint32_t lf0 = ptx::leader_addr(bars.full(0));
     if (lane == 0) {
       ptx::tma_prefetch_desc(&mapQ);
       ptx::tma_prefetch_desc(&mapK);
       ptx::tma_prefetch_desc(&mapV);
+      ptx::tma_prefetch_desc(&mapV2);
     }
     Walk w;
     walk_init(w, a, share);
-    // L2 prefetch of the rows kPrefetch tiles ahead of the tile whose K chunks
-    // are being loaded (tiles counted across the share's pieces): this CTA's
-    // token half of each tile, the peer prefetching the other.  HBM latency is
-    // then covered by the prefetch distance, which takes no shared memory, and
-    // the ring's TMA loads only wait for L2.  Lane 0 of warp 6 issues.
-    Walk pw;
-    walk_init(pw, a, share);
-    Piece ppc;
-    int pk = 0;
-    bool pvalid = kPrefetch > 0 && walk_next(pw, a, share, ppc);
-    const char *cache_bytes = reinterpret_cast<const char *>(a.cache);
-    auto prefetch_next = [&]() {
-      if (!pvalid) return;
-      if (pid == 1 && lane == 0) {
-        const int ts = ppc.tok_begin + kTileTok * pk + kHalfTok * (int)rank;
-        const int te = min(ts + kHalfTok, ppc.tok_end);
-        for (int t = ts; t < te; t += kPrefetchRows) {
-          const int n = min(kPrefetchRows, te - t);
-          const long long r = kv_row(a, ppc.b, t);   // a run of n rows never crosses a page
-          if (r >= 0) ptx::bulk_prefetch_l2(cache_bytes + r * 1152, (uint32_t)n * 1152u);
-        }
-      }
-      if (++pk >= ppc.ntiles) {
-        pk = 0;
-        pvalid = walk_next(pw, a, share, ppc);
-      }
-    };
-    for (int d = 0; d < kPrefetch; ++d) prefetch_next();
 #if MLA_PAIR_EVICT
     const uint64_t last_read = ptx::l2_policy_evict_first();
 #endif
@@ -335,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ws_ = 0;
         ++wround;
       }
-      if ((s & 1) != pid) return -2;
+      if (s % kProducers != pid) return -2;
       bool got = true;
       if (lane == 0 && r > 0) got = ptx::mbar_wait(bars.empty(s), (r - 1) & 1, a.status, abort_flag);
       got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
@@ -385,12 +360,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int y = block_row(a, p, tok0, kv_rows);
             if (leader) ptx::mbar_arrive_expect_tx(bars.full(s), 2 * kSlot);
             const int feat0 = 256 * g + 128 * (int)rank;
+            // one 3D box: 64 rows x both 64-column chunks (chunk index feat0 / 64)
 #if MLA_PAIR_EVICT
-            ptx::tma_load_2d_pair_hint(dst, &mapV, lf0 + 8 * s, feat0, y, last_read);
-            ptx::tma_load_2d_pair_hint(dst + 8192, &mapV, lf0 + 8 * s, feat0 + 64, y, last_read);
+            ptx::tma_load_3d_pair_hint(dst, &mapV2, lf0 + 8 * s, 0, y, feat0 / 64, last_read);
 #else
-            ptx::tma_load_2d_pair(dst, &mapV, lf0 + 8 * s, feat0, y);
-            ptx::tma_load_2d_pair(dst + 8192, &mapV, lf0 + 8 * s, feat0 + 64, y);
+            ptx::tma_load_3d_pair(dst, &mapV2, lf0 + 8 * s, 0, y, feat0 / 64);
 #endif
           }
           ++sc;
@@ -410,7 +384,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!__shfl_sync(0xffffffffu, qok ? 1 : 0, 0)) break;
       for (int k = 0; k < pc.ntiles && ok; ++k) {
-        prefetch_next();
         // K chunks of this tile: this CTA's 128 tokens x 64 columns each.
         const int t0 = pc.tok_begin + kTileTok * k;
         const int tr = t0 + kHalfTok * (int)rank;
@@ -686,23 +659,29 @@ cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s) {
   if (a.page_size != 0 && a.page_size != kTile) return cudaErrorNotSupported;
   const long long rows = a.page_size ? a.cache_len * kTile : (long long)a.B * a.cache_len;
   if (rows <= 0 || rows >= (1ll << 31) - 256) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mv2;
   const uint64_t dq[2] = {576, (uint64_t)a.B * 128};
   const uint64_t dkv[2] = {576, (uint64_t)rows};
   const uint64_t st[1] = {576 * 2};
   const uint32_t boxq[2] = {64, 64};
   const uint32_t boxk[2] = {64, kHalfTok};
   const uint32_t boxv[2] = {64, kSubTok};
+  // The cache viewed as [9 chunks][rows][64 columns]: one box of 64 rows x 2
+  // chunks lands as two 8 KB row-major chunks, the V sub-stage layout.
+  const uint64_t dkv3[3] = {64, (uint64_t)rows, 9};
+  const uint64_t st3[2] = {576 * 2, 64 * 2};
+  const uint32_t boxv3[3] = {64, kSubTok, 2};
   if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, boxq, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_map_bf16(&mk, a.cache, 2, dkv, st, boxk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mv, a.cache, 2, dkv, st, boxv, CU_TENSOR_MAP_SWIZZLE_128B))
+      !encode_map_bf16(&mv, a.cache, 2, dkv, st, boxv, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_bf16(&mv2, a.cache, 3, dkv3, st3, boxv3, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t e = once_per_device(configured, [] {
     return cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_pair_kernel, dim3(2 * P), dim3(kThreads), kSmemAlloc, s, 1, mq, mk, mv, a, rows);
+  return launch_pdl(attn_pair_kernel, dim3(2 * P), dim3(kThreads), kSmemAlloc, s, 1, mq, mk, mv, mv2, a, rows);
 }
 
 }  // namespace mla

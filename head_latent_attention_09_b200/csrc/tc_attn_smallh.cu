@@ -36,12 +36,6 @@ constexpr int kTileTok = 64;
 constexpr float kRescale = 8.0f;
 constexpr int kGroups8 = 5;                // scale groups of a 576-wide row
 
-// L2 prefetch distance in 64-token tiles (0 = off).
-#ifndef MLA_SMALLH_PREFETCH
-#define MLA_SMALLH_PREFETCH 4
-#endif
-constexpr int kPrefetch = MLA_SMALLH_PREFETCH;
-
 #ifndef MLA_F8_CONV_WARPS
 #define MLA_F8_CONV_WARPS 4
 #endif
@@ -234,39 +228,6 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       ptx::tma_prefetch_desc(&mapQ);
       ptx::tma_prefetch_desc(&mapKV);
     }
-    // L2 prefetch of the tile kPrefetch tiles ahead of the one being staged
-    // (tiles counted across the share's pieces), so that HBM latency is
-    // covered without more shared memory; the ring's loads then hit L2.
-    Walk pw;
-    walk_init(pw, a, share);
-    Piece ppc;
-    int pk = 0;
-    bool pvalid = kPrefetch > 0 && walk_next(pw, a, share, ppc);
-    const char *cache_bytes = reinterpret_cast<const char *>(a.cache);
-    constexpr int kRowBytes = F8 ? 576 : 1152;
-    auto prefetch_next = [&]() {
-      if (!pvalid) return;
-      if (lane == 0) {
-        const int t0 = ppc.tok_begin + kTileTok * pk;
-        const int n = min(kTileTok, ppc.tok_end - t0);
-        const long long r = n > 0 ? kv_row(a, ppc.b, t0) : -1;   // 64 rows: one page at most
-        if (r >= 0) {
-          ptx::bulk_prefetch_l2(cache_bytes + r * kRowBytes, (uint32_t)(n * kRowBytes));
-          if (F8) {
-            // the tile's scales: the 16-byte-aligned span inside [first, last) byte
-            const uintptr_t lo = reinterpret_cast<uintptr_t>(a.kv_scale + r * kGroups8);
-            const uintptr_t hi = lo + (uintptr_t)n * kGroups8 * 4;
-            const uintptr_t a0 = (lo + 15) & ~uintptr_t(15), a1 = hi & ~uintptr_t(15);
-            if (a1 > a0) ptx::bulk_prefetch_l2(reinterpret_cast<const void *>(a0), (uint32_t)(a1 - a0));
-          }
-        }
-      }
-      if (++pk >= ppc.ntiles) {
-        pk = 0;
-        pvalid = walk_next(pw, a, share, ppc);
-      }
-    };
-    for (int d = 0; d < kPrefetch; ++d) prefetch_next();
     while (ok && walk_next(w, a, share, pc)) {
       if (npc > 0 && !warp_wait(bar + C::bQEmpty, (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
       if (lane == 0) {
@@ -275,7 +236,6 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
           ptx::tma_load_2d(sQ + c * H * 128, &mapQ, bar + C::bQFull, 64 * c, pc.b * H);
       }
       for (int k = 0; k < pc.ntiles && ok; ++k) {
-        prefetch_next();
         const int tok0 = pc.tok_begin + kTileTok * k;
         const bool manual = tok0 + kTileTok > pc.ctx;     // tile runs past the sequence end
         int y = (int)kv_rows;

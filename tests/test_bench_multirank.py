@@ -85,3 +85,30 @@ def test_reference_arm_on_nonzero_rank_does_no_work(monkeypatch, capsys):
 
     bench.run_reference(A())
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.timeout(180)
+def test_gpus_flag_starts_one_rank_per_gpu():
+    """`python bench.py --gpus 2` started as a plain process starts the two
+    ranks itself (torch.distributed.run on 127.0.0.1); each joins the process
+    group (gloo here, without a GPU) and rank 0 reports both."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--launch-check"],
+                       capture_output=True, text=True, timeout=170, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    assert lines[0]["world"] == 2 and lines[0]["ranks"] == [0, 1]
+
+
+def test_rank_launch_command_matches_the_driver_form():
+    cmd = bench.rank_launch_command(4, ["--gpus", "4", "--steps", "3"], 29500)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd and cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]
