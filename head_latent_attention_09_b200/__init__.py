@@ -34,7 +34,7 @@ EXPORTED = (
     "mla_noalloc_scratch_bytes", "mla_set_rope_scaling",
     "mla_fp8_scale_groups", "mla_cache_append_fp8_workspace_size", "mla_cache_append_fp8",
     "mla_quantize_rows_fp8", "mla_decode_attn_fp8", "mla_selftest_wait_timeout",
-    "mla_set_strict",
+    "mla_set_strict", "mla_decode_attn_range", "mla_combine_splits_f32", "mla_merge_ranges",
 )
 
 
@@ -89,6 +89,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_decode_attn_fp8": (i, [vp, vp, vp, vp, ll, vp, i, vp, i, i, vp, sz, vp]),
         "mla_selftest_wait_timeout": (i, [vp, ll, vp]),
         "mla_set_strict": (i, [vp, i]),
+        "mla_decode_attn_range": (i, [vp, vp, vp, ll, vp, i, vp, vp, i, i, vp, sz, vp]),
+        "mla_combine_splits_f32": (i, [vp, vp, sz, i, i, vp, vp, vp]),
+        "mla_merge_ranges": (i, [vp, vp, vp, i, i, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -220,6 +223,23 @@ def mla_decode_attn(handle, q_abs, cache, cache_len, block_table, max_blocks_per
     _check(load().mla_decode_attn(handle, _ptr(q_abs), _ptr(cache), cache_len, _ptr(block_table),
                                   max_blocks_per_seq, _ptr(ctx_len), B, num_parts,
                                   _ptr(workspace), ws_bytes, _stream(stream)), "mla_decode_attn")
+
+
+def mla_decode_attn_range(handle, q_abs, cache, cache_len, block_table, max_blocks_per_seq, ctx_begin,
+                          ctx_len, B, num_parts, workspace, ws_bytes, stream=None):
+    _check(load().mla_decode_attn_range(handle, _ptr(q_abs), _ptr(cache), cache_len, _ptr(block_table),
+                                        max_blocks_per_seq, _ptr(ctx_begin), _ptr(ctx_len), B, num_parts,
+                                        _ptr(workspace), ws_bytes, _stream(stream)), "mla_decode_attn_range")
+
+
+def mla_combine_splits_f32(handle, workspace, ws_bytes, B, num_parts, ctx_lat, lse, stream=None):
+    _check(load().mla_combine_splits_f32(handle, _ptr(workspace), ws_bytes, B, num_parts, _ptr(ctx_lat),
+                                         _ptr(lse), _stream(stream)), "mla_combine_splits_f32")
+
+
+def mla_merge_ranges(handle, ctx_parts, lse_parts, R, B, ctx_lat, lse=None, stream=None):
+    _check(load().mla_merge_ranges(handle, _ptr(ctx_parts), _ptr(lse_parts), R, B, _ptr(ctx_lat), _ptr(lse),
+                                   _stream(stream)), "mla_merge_ranges")
 
 
 def mla_combine_splits(handle, workspace, ws_bytes, B, num_parts, ctx_lat, lse=None, stream=None):

@@ -226,8 +226,9 @@ namespace {
 // Decode attention over a cache in cfg.dtype (kv_scale NULL) or of FP8 codes
 // with their group scales.
 int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float *kv_scale,
-                long long cache_len, const int *block_table, int max_blocks_per_seq, const int *ctx_len,
-                int B, int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
+                long long cache_len, const int *block_table, int max_blocks_per_seq, const int *ctx_begin,
+                const int *ctx_len, int B, int num_parts, void *workspace, size_t ws_bytes,
+                mla_stream_t stream) {
   if (!h || B < 0 || num_parts < 0 || cache_len < 0) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if (!q_abs || !cache || !ctx_len) return MLA_ERR_INVALID_ARG;
@@ -242,7 +243,7 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
   // pages of its block-table row.
   const long long cap = c.page_size > 0 ? (long long)max_blocks_per_seq * c.page_size : cache_len;
   const long long cap_i = cap < 0x7fffffffLL ? cap : 0x7fffffffLL;
-  cudaError_t e = launch_plan(ctx_len, B, P, cap_i, (char *)workspace, L, h->d_status, s);
+  cudaError_t e = launch_plan(ctx_begin, ctx_len, B, P, cap_i, (char *)workspace, L, h->d_status, s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   AttnArgs a;
   a.q_abs = q_abs;
@@ -278,7 +279,7 @@ int mla_decode_attn(mla_handle *h, const void *q_abs, const void *cache, long lo
                     const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
                     int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
   Range range("mla_decode_attn");
-  return decode_attn(h, q_abs, cache, nullptr, cache_len, block_table, max_blocks_per_seq, ctx_len, B,
+  return decode_attn(h, q_abs, cache, nullptr, cache_len, block_table, max_blocks_per_seq, nullptr, ctx_len, B,
                      num_parts, workspace, ws_bytes, stream);
 }
 
@@ -288,7 +289,16 @@ int mla_decode_attn_fp8(mla_handle *h, const void *q_abs, const void *cache, con
                         mla_stream_t stream) {
   Range range("mla_decode_attn_fp8");
   if (!kv_scale && h && B > 0) return MLA_ERR_INVALID_ARG;
-  return decode_attn(h, q_abs, cache, kv_scale, cache_len, block_table, max_blocks_per_seq, ctx_len, B,
+  return decode_attn(h, q_abs, cache, kv_scale, cache_len, block_table, max_blocks_per_seq, nullptr, ctx_len, B,
+                     num_parts, workspace, ws_bytes, stream);
+}
+
+int mla_decode_attn_range(mla_handle *h, const void *q_abs, const void *cache, long long cache_len,
+                          const int *block_table, int max_blocks_per_seq, const int *ctx_begin, const int *ctx_len,
+                          int B, int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream) {
+  Range range("mla_decode_attn_range");
+  if (!ctx_begin && h && B > 0) return MLA_ERR_INVALID_ARG;
+  return decode_attn(h, q_abs, cache, nullptr, cache_len, block_table, max_blocks_per_seq, ctx_begin, ctx_len, B,
                      num_parts, workspace, ws_bytes, stream);
 }
 
@@ -354,6 +364,28 @@ int mla_combine_splits(mla_handle *h, const void *workspace, size_t ws_bytes, in
   if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   return from_cuda(launch_combine(h->cfg, (const char *)workspace, L, B, ctx_lat, lse,
                                   (cudaStream_t)stream));
+}
+
+int mla_combine_splits_f32(mla_handle *h, const void *workspace, size_t ws_bytes, int B, int num_parts,
+                           float *ctx_lat, float *lse, mla_stream_t stream) {
+  Range range("mla_combine_splits_f32");
+  if (!h || B < 0 || num_parts < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!ctx_lat || !lse) return MLA_ERR_INVALID_ARG;
+  const int P = num_parts == 0 ? default_parts(h) : num_parts;
+  const WsLayout L = ws_layout(h->cfg, B, P);
+  if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  return from_cuda(launch_combine(h->cfg, (const char *)workspace, L, B, ctx_lat, lse, (cudaStream_t)stream,
+                                  true));
+}
+
+int mla_merge_ranges(mla_handle *h, const float *ctx_parts, const float *lse_parts, int R, int B, void *ctx_lat,
+                     float *lse, mla_stream_t stream) {
+  Range range("mla_merge_ranges");
+  if (!h || R < 0 || B < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (R == 0 || !ctx_parts || !lse_parts || !ctx_lat) return MLA_ERR_INVALID_ARG;
+  return from_cuda(launch_merge_ranges(h->cfg, ctx_parts, lse_parts, R, B, ctx_lat, lse, (cudaStream_t)stream));
 }
 
 int mla_out_proj(mla_handle *h, const void *ctx_lat, const void *w_uv, const void *w_o, void *o,

@@ -124,7 +124,7 @@ struct WsHeader {
 struct WsLayout {
   size_t tile_prefix_off;  // int64 [B+1]
   size_t piece_base_off;   // int64 [B+1]
-  size_t ctx_off;          // int32 [B]: each sequence's length as attended (clamped by the plan)
+  size_t ctx_off;          // int32 [2][B]: each sequence's end and first token as attended (clamped by the plan)
   size_t opart_off;        // float [max_pieces, n_h, d_c]
   size_t lse_off;          // float [max_pieces, n_h]
   size_t total;
@@ -142,7 +142,7 @@ inline WsLayout ws_layout(const mla_config &cfg, int B, int P) {
   L.piece_base_off = off;
   off = align_up(off + sizeof(long long) * (size_t)(B + 1), 256);
   L.ctx_off = off;
-  off = align_up(off + sizeof(int) * (size_t)(B > 0 ? B : 1), 256);
+  off = align_up(off + 2 * sizeof(int) * (size_t)(B > 0 ? B : 1), 256);
   L.opart_off = off;
   off = align_up(off + sizeof(float) * (size_t)L.max_pieces * cfg.n_h * cfg.d_c, 256);
   L.lse_off = off;
@@ -174,21 +174,33 @@ struct AttnArgs {
 // ---------------------------------------------------------------------------
 // Launchers (return cudaGetLastError() of the launch).
 // ---------------------------------------------------------------------------
-// The plan clamps every length to [0, cap] (cap: the tokens the cache can
-// address for one sequence), flags any length outside it in the status word,
-// and stores the clamped lengths in the workspace; every attention kernel reads
-// those instead of ctx_len, so that the plan's tiles and the kernels agree.
-cudaError_t launch_plan(const int *ctx_len, int B, int P, long long cap, char *ws, const WsLayout &L,
-                        unsigned *status, cudaStream_t s);
+// The plan attends tokens [begin_b, end_b) of sequence b: end_b = ctx_len[b]
+// clamped to [0, cap] (cap: the tokens the cache can address for one
+// sequence), begin_b = ctx_begin[b] (0 when ctx_begin is NULL) rounded down to
+// a multiple of kTile and clamped to [0, end_b].  Any value it has to change
+// is flagged in the status word.  It stores both in the workspace; every
+// attention kernel reads those instead of the caller's arrays, so that the
+// plan's tiles and the kernels' token ranges agree.
+cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, char *ws,
+                        const WsLayout &L, unsigned *status, cudaStream_t s);
 
-// The clamped length of sequence b, as the plan stored it.
+// The clamped end (context length) of sequence b, as the plan stored it.
 __device__ __forceinline__ int plan_ctx(const char *ws, const WsLayout &L, int b) {
   return reinterpret_cast<const int *>(ws + L.ctx_off)[b];
 }
+// The first attended token of sequence b (a multiple of kTile).
+__device__ __forceinline__ int plan_begin_tok(const char *ws, const WsLayout &L, int b, int B) {
+  return reinterpret_cast<const int *>(ws + L.ctx_off)[B + b];
+}
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s);
+// With out_f32, ctx_lat is written in float32 whatever cfg.dtype.
 cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
-                           void *ctx_lat, float *lse, cudaStream_t s);
+                           void *ctx_lat, float *lse, cudaStream_t s, bool out_f32 = false);
+// Merge of R float32 token-range results [R, B, n_h, d_c] with their
+// log-sum-exps [R, B, n_h] into ctx_lat [B, n_h, d_c] (cfg.dtype) and lse.
+cudaError_t launch_merge_ranges(const mla_config &cfg, const float *parts, const float *lse_parts, int R, int B,
+                                void *ctx_lat, float *lse, cudaStream_t s);
 
 cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int T,
                                const int *start_pos, const void *w_dkv, const void *w_kr,

@@ -60,14 +60,15 @@ __device__ long long block_exclusive_scan(long long v, long long *smem, long lon
   return incl - v;
 }
 
-__global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, int P_req, long long cap,
-                                                    char *ws, WsLayout L, unsigned *status) {
+__global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const int *ctx_len, int B, int P_req,
+                                                    long long cap, char *ws, WsLayout L, unsigned *status) {
   pdl_trigger();
   pdl_wait();   // the workspace may still be read by the previous step's combine
   __shared__ long long scan[1024];
   long long *tile_prefix = reinterpret_cast<long long *>(ws + L.tile_prefix_off);
   long long *piece_base = reinterpret_cast<long long *>(ws + L.piece_base_off);
-  int *ctx_eff = reinterpret_cast<int *>(ws + L.ctx_off);
+  int *ctx_eff = reinterpret_cast<int *>(ws + L.ctx_off);   // [B] ends, then [B] first tokens
+  int *beg_eff = ctx_eff + B;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (B + nt - 1) / nt;
   const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
@@ -81,14 +82,21 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, i
       atomicOr(status, kStatusBounds);
       c = c < 0 ? 0 : cap;
     }
+    long long g = ctx_begin ? ctx_begin[b] : 0;
+    if (g < 0 || g > c || g % kTile != 0) {
+      atomicOr(status, kStatusBounds);
+      g = g < 0 ? 0 : (g > c ? c : g);
+      g -= g % kTile;
+    }
     ctx_eff[b] = (int)c;
-    local += ceil_div_ll(c, kTile);
+    beg_eff[b] = (int)g;
+    local += ceil_div_ll(c - g, kTile);
   }
   long long Ttot;
   long long run = block_exclusive_scan(local, scan, &Ttot);
   for (int b = b0; b < b1; ++b) {
     tile_prefix[b] = run;
-    run += ceil_div_ll(ctx_eff[b], kTile);
+    run += ceil_div_ll(ctx_eff[b] - beg_eff[b], kTile);
   }
   if (tid == 0) tile_prefix[B] = Ttot;
   const long long P = Ttot < (long long)P_req ? Ttot : (long long)P_req;
@@ -96,7 +104,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, i
   long long local_pieces = 0;
   for (int b = b0; b < b1; ++b) {
     long long s = tile_prefix[b];
-    long long t = ceil_div_ll(ctx_eff[b], kTile);
+    long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], kTile);
     if (t > 0) local_pieces += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
   long long n_pieces;
@@ -104,7 +112,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_len, int B, i
   for (int b = b0; b < b1; ++b) {
     piece_base[b] = prun;
     long long s = tile_prefix[b];
-    long long t = ceil_div_ll(ctx_eff[b], kTile);
+    long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], kTile);
     if (t > 0) prun += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
   if (tid == 0) {
@@ -168,8 +176,9 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
     if (s0 >= s1) continue;
     const long long piece = pb[b] + (w - plan_share_of_tile(tp[b], P, Ttot));
     const int ctx = plan_ctx(a.ws, a.L, b);
-    const long long p_begin = (s0 - tp[b]) * kTile;
-    const long long p_end = min((long long)ctx, (s1 - tp[b]) * kTile);
+    const long long beg = plan_begin_tok(a.ws, a.L, b, a.B);
+    const long long p_begin = beg + (s0 - tp[b]) * kTile;
+    const long long p_end = min((long long)ctx, beg + (s1 - tp[b]) * kTile);
 
     float q[kQPerLane];
 #pragma unroll
@@ -432,9 +441,9 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const T *o, const T *w
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_plan(const int *ctx_len, int B, int P, long long cap, char *ws, const WsLayout &L,
-                        unsigned *status, cudaStream_t s) {
-  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_len, B, P, cap, ws, L, status);
+cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, char *ws,
+                        const WsLayout &L, unsigned *status, cudaStream_t s) {
+  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_begin, ctx_len, B, P, cap, ws, L, status);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s) {
@@ -524,13 +533,14 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(const char *ws, WsLayo
 }
 
 cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
-                           void *ctx_lat, float *lse, cudaStream_t s) {
-  const size_t esz = cfg.dtype == MLA_FP32 ? 4 : 2;
+                           void *ctx_lat, float *lse, cudaStream_t s, bool out_f32) {
+  const bool f32 = out_f32 || cfg.dtype == MLA_FP32;
+  const size_t esz = f32 ? 4 : 2;
   if (cfg.d_c % 4 == 0 && cfg.d_c <= 512 && ((uintptr_t)ctx_lat % (4 * esz)) == 0 &&
       ((uintptr_t)ws % 16) == 0) {
     const long long rows = (long long)B * cfg.n_h;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
-    if (cfg.dtype == MLA_FP32)
+    if (f32)
       return launch_pdl(combine_vec_kernel<float>, dim3(blocks), dim3(256), 0, s, 1, ws, L, B, cfg.n_h, cfg.d_c,
                         (float *)ctx_lat, lse);
     else
@@ -538,11 +548,59 @@ cudaError_t launch_combine(const mla_config &cfg, const char *ws, const WsLayout
                         cfg.d_c, (__nv_bfloat16 *)ctx_lat, lse);
   }
   dim3 grid(B, cfg.n_h);
-  if (cfg.dtype == MLA_FP32)
+  if (f32)
     return launch_pdl(combine_kernel<float>, grid, dim3(128), 0, s, 1, ws, L, cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
   else
     return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(128), 0, s, 1, ws, L, cfg.n_h, cfg.d_c,
                       (__nv_bfloat16 *)ctx_lat, lse);
+}
+
+// ---------------------------------------------------------------------------
+// merge of R token-range results (split-KV across devices): one warp per
+// (sequence, head) row; the same log-sum-exp algebra as the combine, over the
+// R float32 results [R, B, n_h, d_c] and their log-sum-exps [R, B, n_h], in
+// range order.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) merge_ranges_kernel(const float *parts, const float *lse_parts, int R,
+                                                           int B, int n_h, int d_c, T *ctx_lat, float *lse_out) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + warp;   // = b * n_h + h
+  const long long rows = (long long)B * n_h;
+  if (row >= rows) return;
+  float m = -CUDART_INF_F;
+  for (int r = lane; r < R; r += 32) m = fmaxf(m, lse_parts[r * rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  T *dst = ctx_lat + row * d_c;
+  if (m == -CUDART_INF_F) {
+    for (int f = lane; f < d_c; f += 32) dst[f] = from_f<T>(0.f);
+    if (lse_out && lane == 0) lse_out[row] = -CUDART_INF_F;
+    return;
+  }
+  float tot = 0.f;
+  for (int r = lane; r < R; r += 32) tot += expf(lse_parts[r * rows + row] - m);
+  tot = warp_sum(tot);
+  const float inv = 1.f / tot;
+  for (int f = lane; f < d_c; f += 32) {
+    float acc = 0.f;
+    for (int r = 0; r < R; ++r) acc += expf(lse_parts[r * rows + row] - m) * inv * parts[(r * rows + row) * d_c + f];
+    dst[f] = from_f<T>(acc);
+  }
+  if (lse_out && lane == 0) lse_out[row] = m + logf(tot);
+}
+
+cudaError_t launch_merge_ranges(const mla_config &cfg, const float *parts, const float *lse_parts, int R, int B,
+                                void *ctx_lat, float *lse, cudaStream_t s) {
+  const long long rows = (long long)B * cfg.n_h;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  if (cfg.dtype == MLA_FP32)
+    return launch_pdl(merge_ranges_kernel<float>, dim3(blocks), dim3(256), 0, s, 1, parts, lse_parts, R, B,
+                      cfg.n_h, cfg.d_c, (float *)ctx_lat, lse);
+  return launch_pdl(merge_ranges_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, s, 1, parts, lse_parts, R, B,
+                    cfg.n_h, cfg.d_c, (__nv_bfloat16 *)ctx_lat, lse);
 }
 
 cudaError_t launch_append_simt(const mla_config &cfg, const void *h, int B, int T,

@@ -211,6 +211,26 @@ int mla_decode_attn(mla_handle *handle, const void *q_abs, const void *cache, lo
                     const int *block_table, int max_blocks_per_seq, const int *ctx_len, int B,
                     int num_parts, void *workspace, size_t ws_bytes, mla_stream_t stream);
 
+/* Decode attention over a token range of each sequence: tokens
+ * ctx_begin[b] .. ctx_len[b]-1 of sequence b instead of 0 .. ctx_len[b]-1;
+ * otherwise as mla_decode_attn (same workspace, same partials, merged by
+ * mla_combine_splits or mla_combine_splits_f32).  This is the per-device step
+ * of split-KV across devices for long contexts: each device holds and attends
+ * one token range of every sequence, and the per-range results are merged
+ * with mla_merge_ranges (the "DeepSeek-V3" note's decode deployment runs
+ * attention data-parallel with sequence parallelism; the merge is the
+ * log-sum-exp algebra of the split combine).
+ *   ctx_begin device int32 [B]; each value a multiple of 64 in [0, ctx_len[b]].
+ *             Other values set MLA_ERR_DEVICE_BOUNDS in the status word and are
+ *             clamped into that range and rounded down to a multiple of 64.
+ *   With a paged cache the block table needs entries only for the blocks of
+ *   the range (the others may be -1): a device's pool can hold just its range.
+ * Errors as mla_decode_attn; INVALID_ARG for a NULL ctx_begin. */
+int mla_decode_attn_range(mla_handle *handle, const void *q_abs, const void *cache, long long cache_len,
+                          const int *block_table, int max_blocks_per_seq, const int *ctx_begin,
+                          const int *ctx_len, int B, int num_parts, void *workspace, size_t ws_bytes,
+                          mla_stream_t stream);
+
 /* Merge the partials of the preceding mla_decode_attn on the same workspace:
  * m = max_s lse_s, ctx_lat = sum_s e^(lse_s - m) O_s / sum_s e^(lse_s - m),
  * lse = m + log sum_s e^(lse_s - m).
@@ -218,6 +238,24 @@ int mla_decode_attn(mla_handle *handle, const void *q_abs, const void *cache, lo
  * B and num_parts must equal those given to mla_decode_attn. */
 int mla_combine_splits(mla_handle *handle, const void *workspace, size_t ws_bytes, int B,
                        int num_parts, void *ctx_lat, float *lse, mla_stream_t stream);
+
+/* The same merge written in float32 whatever cfg.dtype: ctx_lat [B, n_h, d_c]
+ * float32 and lse [B, n_h] float32 (not NULL), the per-range result that
+ * devices exchange before mla_merge_ranges. */
+int mla_combine_splits_f32(mla_handle *handle, const void *workspace, size_t ws_bytes, int B,
+                           int num_parts, float *ctx_lat, float *lse, mla_stream_t stream);
+
+/* Merge the results of R token ranges of the same B sequences (split-KV across
+ * devices), in range order, with the combine's algebra: per (b, i),
+ * m = max_r lse_r, ctx_lat = sum_r e^(lse_r - m) ctx_r / sum_r e^(lse_r - m),
+ * lse = m + log sum_r e^(lse_r - m); a range with lse = -inf (no tokens)
+ * carries no weight, and if every range is empty the row is zero with
+ * lse = -inf.
+ *   ctx_parts [R, B, n_h, d_c] float32, lse_parts [R, B, n_h] float32 (device)
+ *   ctx_lat [B, n_h, d_c] (cfg.dtype), lse [B, n_h] float32 or NULL.
+ * Errors: INVALID_ARG (NULL pointers, R <= 0 with B > 0), CUDA. */
+int mla_merge_ranges(mla_handle *handle, const float *ctx_parts, const float *lse_parts, int R, int B,
+                     void *ctx_lat, float *lse, mla_stream_t stream);
 
 /* Output projection (V2 App. C, W^UV absorbed to the output side; V3 note u_t):
  *   o[b,i,:] = W^UV_i ctx_lat[b,i,:]      o [B, n_h, d_h]
