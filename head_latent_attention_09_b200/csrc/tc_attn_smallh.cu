@@ -1,27 +1,43 @@
 // Split-KV decode attention over the latent cache for few heads (n_h = 16 or
-// 32; DeepSeek-V2-Lite shapes: d_c = 512, d_h^R = 64, bf16), one CTA per SM.
+// 32; DeepSeek-V2-Lite shapes: d_c = 512, d_h^R = 64), one CTA per SM.
 //
 // Same result as the 128-head kernel (per piece: ctx_i = softmax(q_abs_i .
 // rows / sqrt(d_h + d_h^R)) . c and its log-sum-exp), but with few heads the
-// tensor core's M dimension is taken by tokens instead (the transposed form):
-//   S^T = K Q^T      M = 64 tokens, N = n_h heads, K = 576 (nine 64-col chunks)
-//   O^T += V^T P^T   M = 64 latent columns per MMA (eight blocks), N = n_h,
-//                    K = 64 tokens
-// A 64-token tile of the cache is read from HBM once into nine 8 KB chunks of
-// a 24-slot ring; each chunk serves both products.  This path is HBM-bound
-// (30 flop/byte), so the tile is small and the ring deep.  Per-head softmax
-// statistics are reductions across tokens, i.e. across threads: warp shuffles
-// over the 16 lanes of each M=64 accumulator quarter, then shared memory.
+// tensor core's M dimension is taken by tokens and latent columns instead
+// (the transposed form), 128 at a time:
+//   S^T = K Q^T      M = 128 tokens, N = n_h heads, K = 576 (nine 64-col chunks)
+//   O^T += V^T P^T   M = 128 latent columns per MMA (four blocks), N = n_h,
+//                    K = 128 tokens
+// A tcgen05.mma instruction takes at least ~124 cycles however little it
+// computes (measured), so this path is bound by the number of MMA
+// instructions per cached token: M = 128 needs 68 per 128 tokens, half of
+// what M = 64 needs.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 tensor-memory
-// allocation and MMA issue, warps 2-5 softmax / rescale / epilogue.
+// A 128-token tile of the cache is read from HBM once, as nine 16 KB chunks
+// (128 rows x 64 columns): the rotary chunk into a ring of its own (it only
+// feeds S), and the eight latent chunks as four pairs into a ring of 32 KB
+// pair slots, where each pair is the MN-major A operand of one O^T block (the
+// two chunks 16 KB apart).  Both products read the same staged chunks.  A
+// tile holds its pair slots until its P.V; the MMAs of the next tile's S that
+// have their data already (its rotary chunk, and one pair where the ring has a
+// fifth slot) are issued before that P.V, so that the tensor core works
+// while the softmax runs.
+//
+// Per-head softmax statistics are reductions across tokens, i.e. across
+// threads: warp shuffles over 32 lanes, then shared memory across the warps.
+//
+// Warp roles: warp 0 TMA producer, warp 1 tensor-memory allocation and MMA
+// issue, warps 2-5 softmax / rescale / epilogue.
 //
 // FP8 cache (E4M3 codes, a float32 scale per token and 128-channel group):
-// the producer stages each 64 x 64 chunk of codes (4 KB) by TMA, and four
-// more warps (6-9) widen it into the bf16 ring slot the MMAs read, applying
-// the group scale on the way (code * sigma rounded to bf16).  HBM then
-// carries 576 B + 20 B of scales per token instead of 1152 B; the products,
-// the softmax and the epilogue are those of the bf16 cache.
+// the producer stages each 128 x 64 chunk of codes (8 KB) by TMA, and four
+// more warps (6-9) widen it into the bf16 chunk the MMAs read, applying the
+// group scale on the way (code * sigma rounded to bf16).  HBM then carries
+// 576 B + 20 B of scales per token instead of 1152 B; the products, the
+// softmax and the epilogue are those of the bf16 cache.
+//
+// Every wait is bounded; a wait that runs out flags MLA_ERR_TIMEOUT and the
+// kernel winds down without further waits.
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
@@ -30,49 +46,44 @@
 namespace mla {
 namespace {
 
-constexpr int kChunk = 8192;               // [64 rows x 128 B]
-constexpr int kChunk8 = 4096;              // FP8 staging: [64 rows x 64 B]
-constexpr int kTileTok = 64;
+constexpr int kTileTok = 128;              // tokens per tile (MMA M of S^T)
+constexpr int kChunk = 16384;              // bf16 chunk: 128 rows x 128 B
+constexpr int kPair = 2 * kChunk;          // latent pair slot: chunks 2b, 2b + 1
+constexpr int kChunk8 = 8192;              // FP8 staging chunk: 128 rows x 64 B
 constexpr float kRescale = 8.0f;
 constexpr int kGroups8 = 5;                // scale groups of a 576-wide row
 
-#ifndef MLA_F8_CONV_WARPS
-#define MLA_F8_CONV_WARPS 4
-#endif
-#ifndef MLA_F8_RING
-#define MLA_F8_RING 21
-#endif
-#ifndef MLA_F8_STAGE16
-#define MLA_F8_STAGE16 6
-#endif
-
 template <int H, bool F8>
 struct Cfg {
-  static constexpr int kConvWarps = F8 ? MLA_F8_CONV_WARPS : 0;   // FP8 converter warps (4 or 8)
+  static constexpr int kConvWarps = F8 ? 4 : 0;                 // FP8 converter warps
   static constexpr int kThreads = 192 + 32 * kConvWarps;
-  // Ring chunk slots.  A tile holds its nine slots until its P.V is done,
-  // which is issued after the next tile's S: at least two tiles' worth.
-  static constexpr int kNS = F8 ? (H <= 16 ? MLA_F8_RING : 18) : (H <= 16 ? 24 : 18);
-  static constexpr int kNSt = F8 ? (H <= 16 ? MLA_F8_STAGE16 : 8) : 0;  // FP8 staging chunks
-  static_assert(!F8 || kNS >= 18, "the ring must hold two tiles");
-  static constexpr int kQ = 9 * H * 128;                    // H rows x 576
-  static constexpr int kPT = H * 128;                       // P^T: H rows x 64 tokens
+  static constexpr int kNL = (!F8 && H <= 16) ? 5 : 4;          // latent pair slots (a tile takes 4)
+  static constexpr int kNR = (F8 && H > 16) ? 1 : 2;            // rotary chunk slots
+  static constexpr int kNSt = F8 ? (H <= 16 ? 4 : 3) : 0;       // FP8 staging chunks
+  static constexpr int kEarlyPairs = kNL - 4;                   // next tile's pairs issued before P.V
+  static constexpr bool kEarlyRope = kNR >= 2;                  // next tile's rotary chunk likewise
+  static constexpr int kQ = 9 * H * 128;                        // H rows x 576, nine 64-column chunks
+  static constexpr int kPT = 2 * H * 128;                       // P^T: H rows x 128 tokens, two 64-token chunks
   static constexpr int kOffQ = 0;
-  static constexpr int kOffRing = (kQ + 1023) / 1024 * 1024;
-  static constexpr int kOffStage = kOffRing + kNS * kChunk;
+  static constexpr int kOffLat = (kQ + 1023) / 1024 * 1024;
+  static constexpr int kOffRope = kOffLat + kNL * kPair;
+  static constexpr int kOffStage = kOffRope + kNR * kChunk;
   static constexpr int kOffP = kOffStage + kNSt * kChunk8;
-  static constexpr int kOffRed = kOffP + 2 * ((kPT + 1023) / 1024 * 1024);  // float [2][4][H] max, [4][H] sum
+  static constexpr int kPStride = (kPT + 1023) / 1024 * 1024;
+  static constexpr int kOffRed = kOffP + 2 * kPStride;          // float [2][4][H] max, [4][H] sum
   static constexpr int kOffBar = kOffRed + 12 * H * 4;
   // barriers
-  static constexpr int bFull = 0, bEmpty = kNS, bQFull = 2 * kNS, bQEmpty = bQFull + 1, bSFull = bQEmpty + 1,
-                       bPFull = bSFull + 2, bPFree = bPFull + 2, bODone = bPFree + 2, bOFree = bODone + 2,
-                       bXchg = bOFree + 1, bLsum = bXchg + 2, bStFull = bLsum + 1, bStEmpty = bStFull + kNSt,
-                       kNumBars = bStEmpty + kNSt;
+  static constexpr int bLatFull = 0, bLatEmpty = kNL, bRopeFull = 2 * kNL, bRopeEmpty = bRopeFull + kNR,
+                       bStFull = bRopeEmpty + kNR, bStEmpty = bStFull + kNSt, bQFull = bStEmpty + kNSt,
+                       bQEmpty = bQFull + 1, bSFull = bQEmpty + 1, bPFull = bSFull + 2, bPFree = bPFull + 2,
+                       bODone = bPFree + 2, bOFree = bODone + 2, bXchg = bOFree + 1, bLsum = bXchg + 2,
+                       kNumBars = bLsum + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;
-  static constexpr uint32_t kTmemCols = 10 * H <= 256 ? 256 : 512;  // S^T 2 x H, O^T 8 x H
+  static constexpr uint32_t kTmemCols = 6 * H <= 128 ? 128 : 256;   // S^T 2 x H, O^T 4 x H
   static constexpr uint32_t kColO = 2 * H;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static_assert(kNL >= 4, "a tile takes four pair slots");
 };
 
 // Two E4M3 codes (low byte first) times sigma, as a bf16 pair.
@@ -147,6 +158,19 @@ __device__ __forceinline__ long long kv_row(const AttnArgs &a, int b, int t) {
   return (long long)blk * kTile + (t % kTile);
 }
 
+// Row coordinate of the 64-row block of cache rows starting at token t0 of the
+// piece's sequence, or an out-of-range row (TMA then fills zeros) when the
+// block starts at or past the piece's end.
+__device__ __forceinline__ int block_row(const AttnArgs &a, const Piece &p, int t0, long long kv_rows) {
+  if (t0 >= p.tok_end) return (int)kv_rows;
+  const long long r = kv_row(a, p.b, t0);
+  if (r < 0) {
+    atomicOr(a.status, kStatusBounds);
+    return (int)kv_rows;
+  }
+  return (int)r;
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned *status, volatile int *abort) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, status, abort);
@@ -156,22 +180,67 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
   return ok;
 }
 
+// A ring of slots consumed in fill order: slot and phase parity of the next use.
+struct RingPos {
+  int slot = 0;
+  uint32_t phase = 0;
+  int round = 0;
+  __device__ void advance(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+      ++round;
+    }
+  }
+};
+
+// Hand copy of the 64-row half of a tile that holds the sequence's end: rows
+// [t0, ctx) of columns [64c, 64c + 64), zeros for rows [ctx, t0 + 64), so
+// that no unwritten cache row (possibly NaN) reaches P.V.  bf16: 128-byte
+// rows with the 128-byte swizzle; FP8: 64-byte rows, no swizzle.  The whole
+// warp copies, every lane issuing all its loads before its stores (a half
+// lies inside one 64-token page, so its rows are consecutive).
+template <bool F8>
+__device__ __forceinline__ void hand_copy_half(const AttnArgs &a, const Piece &p, int t0, int c, uint8_t *dst) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kUnits = F8 ? 4 : 8;          // 16-byte units per row
+  constexpr int kPer = 64 * kUnits / 32;      // units per lane
+  const long long r0 = kv_row(a, p.b, t0);
+  if (r0 < 0 && lane == 0) atomicOr(a.status, kStatusBounds);
+  uint4 v[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int u = lane + 32 * k, row = u / kUnits, cc = u % kUnits;
+    v[k] = make_uint4(0, 0, 0, 0);
+    if (r0 >= 0 && t0 + row < p.ctx)
+      v[k] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(a.cache) +
+                                              (r0 + row) * (F8 ? 576 : 1152) + (F8 ? 64 * c : 128 * c) + 16 * cc);
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int u = lane + 32 * k, row = u / kUnits, cc = u % kUnits;
+    const int off = F8 ? row * 64 + 16 * cc : row * 128 + ((cc ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4 *>(dst + off) = v[k];
+  }
+}
+
 template <int H, bool F8>
 __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
     attn_smallh_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapKV,
+                       const __grid_constant__ CUtensorMap mapKV64, const __grid_constant__ CUtensorMap mapPair,
                        const AttnArgs a, const long long kv_rows) {
   using C = Cfg<H, F8>;
-  constexpr int NS = C::kNS;
-  // Staging chunks as a divisor for the FP8 code paths; without FP8 those
+  constexpr int NL = C::kNL, NR = C::kNR;
+  // Staging slots as a divisor for the FP8 code paths; without FP8 those
   // paths never run and there are no staging barriers (C::kNSt = 0).
   constexpr int NSt = C::kNSt > 0 ? C::kNSt : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + C::kOffQ;
-  uint8_t *sRing = sm + C::kOffRing;
-  uint8_t *sP = sm + C::kOffP;
+  uint8_t *sLat = sm + C::kOffLat;
+  uint8_t *sRope = sm + C::kOffRope;
   uint8_t *sStage = sm + C::kOffStage;
-  constexpr int kPStride = (C::kPT + 1023) / 1024 * 1024;
+  uint8_t *sP = sm + C::kOffP;
   float *red_m = reinterpret_cast<float *>(sm + C::kOffRed);  // [2][4][H]
   float *red_s = red_m + 8 * H;                                // [4][H]
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
@@ -183,9 +252,13 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
   pdl_trigger();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      ptx::mbar_init(bar + C::bFull + s, F8 ? C::kConvWarps : 1);   // FP8: every converter warp
-      ptx::mbar_init(bar + C::bEmpty + s, 1);
+    for (int s = 0; s < NL; ++s) {
+      ptx::mbar_init(bar + C::bLatFull + s, F8 ? 2 * C::kConvWarps : 1);   // FP8: both chunks, every converter
+      ptx::mbar_init(bar + C::bLatEmpty + s, 1);
+    }
+    for (int s = 0; s < NR; ++s) {
+      ptx::mbar_init(bar + C::bRopeFull + s, F8 ? C::kConvWarps : 1);
+      ptx::mbar_init(bar + C::bRopeEmpty + s, 1);
     }
     for (int s = 0; s < C::kNSt; ++s) {
       ptx::mbar_init(bar + C::bStFull + s, 1);
@@ -197,10 +270,9 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       ptx::mbar_init(bar + C::bSFull + i, 1);
       ptx::mbar_init(bar + C::bPFull + i, 4);
       ptx::mbar_init(bar + C::bPFree + i, 1);
+      ptx::mbar_init(bar + C::bODone + i, 1);
       ptx::mbar_init(bar + C::bXchg + i, 4);
     }
-    ptx::mbar_init(bar + C::bODone, 1);
-    ptx::mbar_init(bar + C::bODone + 1, 1);
     ptx::mbar_init(bar + C::bOFree, 4);
     ptx::mbar_init(bar + C::bLsum, 4);
     *abort_flag = 0;
@@ -220,15 +292,26 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
 
   if (warp == 0) {
     // -------------------------------------------------------------- producer
+    // Per tile, in the order the MMAs consume them: the rotary chunk, then
+    // the four latent pairs (bf16), or the nine chunks of codes into the
+    // staging ring (FP8: rotary chunk first, then latent chunks 0-7).
     Walk w;
     walk_init(w, a, share);
     Piece pc;
-    int sc = 0, npc = 0;
+    RingPos lat, rope, stg;
+    int npc = 0;
     bool ok = true;
     if (lane == 0) {
       ptx::tma_prefetch_desc(&mapQ);
       ptx::tma_prefetch_desc(&mapKV);
+      ptx::tma_prefetch_desc(&mapKV64);
+      if (!F8) ptx::tma_prefetch_desc(&mapPair);
     }
+    // Waits (lane 0) for a slot's previous use to be released; warp-uniform.
+    auto slot_free = [&](uint64_t *empty, const RingPos &r) -> bool {
+      if (r.round == 0) return true;
+      return warp_wait(empty, r.phase ^ 1u, a.status, abort_flag);
+    };
     while (ok && walk_next(w, a, share, pc)) {
       if (npc > 0 && !warp_wait(bar + C::bQEmpty, (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
       if (lane == 0) {
@@ -238,113 +321,151 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       }
       for (int k = 0; k < pc.ntiles && ok; ++k) {
         const int tok0 = pc.tok_begin + kTileTok * k;
-        const bool manual = tok0 + kTileTok > pc.ctx;     // tile runs past the sequence end
-        int y = (int)kv_rows;
-        if (!manual) {
-          const long long r = kv_row(a, pc.b, tok0);
-          if (r >= 0) y = (int)r;
-          else if (lane == 0) atomicOr(a.status, kStatusBounds);
+        // Each 64-row half of the tile: wholly inside the sequence (TMA from
+        // its rows), wholly past its end (TMA from an out-of-range row: zeros),
+        // or holding its end (hand copy).
+        int kind[2], yy[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int t = tok0 + 64 * h2;
+          kind[h2] = t + 64 <= pc.ctx ? 0 : (t >= pc.ctx ? 1 : 2);
+          int y = (int)kv_rows;
+          if (kind[h2] == 0 && lane == 0) y = block_row(a, pc, t, kv_rows);
+          yy[h2] = __shfl_sync(0xffffffffu, y, 0);
         }
-        for (int c = 0; c < 9 && F8; ++c) {
-          // FP8: stage the 64 x 64 chunk of codes for the converter warps
-          const int s = sc % NSt;
-          if (sc >= NSt && !warp_wait(bar + C::bStEmpty + s, ((sc / NSt) - 1) & 1, a.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t *dst = sStage + s * kChunk8;
-          if (manual) {
-            for (int u = lane; u < 64 * 4; u += 32) {
-              const int row = u >> 2, cc = u & 3;
-              const int t = tok0 + row;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (t < pc.ctx) {
-                const long long r = kv_row(a, pc.b, t);
-                if (r >= 0)
-                  v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(a.cache) + r * 576 +
-                                                       64 * c + 16 * cc);
-                else
-                  atomicOr(a.status, kStatusBounds);
-              }
-              *reinterpret_cast<uint4 *>(dst + row * 64 + 16 * cc) = v;
-            }
-            ptx::fence_proxy_async_smem();   // later TMA writes to this slot come after these
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar + C::bStFull + s);
-          } else if (lane == 0) {
-            ptx::mbar_arrive_expect_tx(bar + C::bStFull + s, kChunk8);
-            ptx::tma_load_2d(dst, &mapKV, bar + C::bStFull + s, 64 * c, y);
-          }
-          ++sc;
-        }
-        for (int c = 0; c < 9 && !F8; ++c) {
-          const int s = sc % NS;
-          if (sc >= NS && !warp_wait(bar + C::bEmpty + s, ((sc / NS) - 1) & 1, a.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t *dst = sRing + s * kChunk;
-          if (manual) {
-            // copy valid rows by hand, zero the rest (no unwritten row reaches P V)
-            for (int u = lane; u < 64 * 8; u += 32) {
-              const int row = u >> 3, cc = u & 7;
-              const int t = tok0 + row;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (t < pc.ctx) {
-                const long long r = kv_row(a, pc.b, t);
-                if (r >= 0)
-                  v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.cache) +
-                                                       r * 576 + 64 * c + 8 * cc);
-                else
-                  atomicOr(a.status, kStatusBounds);
-              }
-              *reinterpret_cast<uint4 *>(dst + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
-            }
+        const bool whole = a.page_size == 0 && kind[0] == 0 && kind[1] == 0 && yy[0] < kv_rows &&
+                           yy[1] == yy[0] + 64;
+        const bool partial = kind[0] == 2 || kind[1] == 2;
+        // One chunk (column block c) into `dst` as two 64-row halves `half`
+        // bytes apart; the barrier is armed with the bytes the TMA brings.
+        auto stage_chunk = [&](uint8_t *dst, int c, int half, uint32_t &tx) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2)
+            if (kind[h2] == 2) hand_copy_half<F8>(a, pc, tok0 + 64 * h2, c, dst + h2 * half);
+          tx += (kind[0] != 2 ? half : 0) + (kind[1] != 2 ? half : 0);
+        };
+        auto issue_chunk = [&](uint8_t *dst, int c, int half, const CUtensorMap *m64, uint64_t *full) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2)
+            if (kind[h2] != 2) ptx::tma_load_2d(dst + h2 * half, m64, full, 64 * c, yy[h2]);
+        };
+        // After any hand copy: make it visible to the tensor core, then arm.
+        auto arm = [&](uint64_t *full, uint32_t tx) {
+          if (partial) {
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar + C::bFull + s);
-          } else if (lane == 0) {
-            ptx::mbar_arrive_expect_tx(bar + C::bFull + s, kChunk);
-            ptx::tma_load_2d(dst, &mapKV, bar + C::bFull + s, 64 * c, y);
           }
-          ++sc;
+          if (lane == 0) ptx::mbar_arrive_expect_tx(full, tx);
+        };
+        if (F8) {
+          // nine chunks of codes, rotary first
+          for (int j = 0; j < 9 && ok; ++j) {
+            const int c = j == 0 ? 8 : j - 1;
+            uint64_t *full = bar + C::bStFull + stg.slot;
+            if (!slot_free(bar + C::bStEmpty + stg.slot, stg)) { ok = false; break; }
+            uint8_t *dst = sStage + stg.slot * kChunk8;
+            uint32_t tx = 0;
+            stage_chunk(dst, c, kChunk8 / 2, tx);
+            arm(full, tx);
+            if (lane == 0) issue_chunk(dst, c, kChunk8 / 2, &mapKV64, full);
+            stg.advance(NSt);
+          }
+          continue;
+        }
+        // bf16: the rotary chunk
+        {
+          uint64_t *full = bar + C::bRopeFull + rope.slot;
+          if (!slot_free(bar + C::bRopeEmpty + rope.slot, rope)) { ok = false; break; }
+          uint8_t *dst = sRope + rope.slot * kChunk;
+          if (whole) {
+            if (lane == 0) {
+              ptx::mbar_arrive_expect_tx(full, kChunk);
+              ptx::tma_load_2d(dst, &mapKV, full, 512, yy[0]);
+            }
+          } else {
+            uint32_t tx = 0;
+            stage_chunk(dst, 8, kChunk / 2, tx);
+            arm(full, tx);
+            if (lane == 0) issue_chunk(dst, 8, kChunk / 2, &mapKV64, full);
+          }
+          rope.advance(NR);
+        }
+        // the four latent pairs
+        for (int pb = 0; pb < 4 && ok; ++pb) {
+          uint64_t *full = bar + C::bLatFull + lat.slot;
+          if (!slot_free(bar + C::bLatEmpty + lat.slot, lat)) { ok = false; break; }
+          uint8_t *dst = sLat + lat.slot * kPair;
+          if (whole) {
+            if (lane == 0) {
+              // one 3D box: 128 rows x chunks 2pb, 2pb + 1
+              ptx::mbar_arrive_expect_tx(full, kPair);
+              ptx::tma_load_3d(dst, &mapPair, full, 0, yy[0], 2 * pb);
+            }
+          } else {
+            uint32_t tx = 0;
+            stage_chunk(dst, 2 * pb, kChunk / 2, tx);
+            stage_chunk(dst + kChunk, 2 * pb + 1, kChunk / 2, tx);
+            arm(full, tx);
+            if (lane == 0) {
+              issue_chunk(dst, 2 * pb, kChunk / 2, &mapKV64, full);
+              issue_chunk(dst + kChunk, 2 * pb + 1, kChunk / 2, &mapKV64, full);
+            }
+          }
+          lat.advance(NL);
         }
       }
       ++npc;
     }
-    if (*abort_flag) {
-      const unsigned long long t0 = ptx::globaltimer();
-      while (ptx::globaltimer() - t0 < 100000ull) {}
-    }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(64, H, false, false);
-      constexpr uint32_t idO = idesc_bf16(64, H, true, false);
+      constexpr uint32_t idS = idesc_bf16(128, H, false, false);
+      constexpr uint32_t idO = idesc_bf16(128, H, true, false);
       Walk w;
       walk_init(w, a, share);
       Piece pc;
-      int sc = 0, npc = 0, i = 0;
+      RingPos lat, rope;   // next slot to consume
+      int npc = 0, i = 0;
       bool ok = true;
-      struct Prev { int i, first, npc, slot0; } prev{0, 0, 0, 0};
-      bool have_prev = false;
-      const uint32_t q0 = ptx::smem_u32(sQ), r0 = ptx::smem_u32(sRing), p0 = ptx::smem_u32(sP);
-      auto pv = [&](const Prev &t) -> bool {
+      const uint32_t q0 = ptx::smem_u32(sQ), l0 = ptx::smem_u32(sLat), r0 = ptx::smem_u32(sRope),
+                     p0 = ptx::smem_u32(sP);
+      // S^T chunk c of tile i from the staged rows at address `src`.
+      auto s_chunk = [&](uint32_t src, int c, uint32_t dS, bool first) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t ad = ptx::sdesc(src + 32 * j, 16, 1024, 2);                   // K rows
+          const uint64_t bd = ptx::sdesc(q0 + c * H * 128 + 32 * j, 16, 1024, 2);     // Q rows
+          ptx::mma_bf16_ss(dS, ad, bd, idS, (first && j == 0) ? 0u : 1u);
+        }
+      };
+      // Chunks of S^T(i) issued ahead of P.V(i-1) (count of pairs, rotary chunk done).
+      int early_pairs = 0;
+      bool early_rope = false;
+      int lat_first = 0;        // pair slots of the tile whose S is being issued start here
+      auto wait_full = [&](uint64_t *b, uint32_t ph) -> bool {
+        if (!ptx::mbar_wait(b, ph, a.status, abort_flag)) return false;
+        ptx::tc_fence_after();
+        return true;
+      };
+      struct Tile { int i, first, npc, lat0; };
+      auto pv = [&](const Tile &t) -> bool {
         if (t.first && t.npc > 0 && !ptx::mbar_wait(bar + C::bOFree, (t.npc - 1) & 1, a.status, abort_flag))
           return false;
-        if (!ptx::mbar_wait(bar + C::bPFull + (t.i & 1), (t.i >> 1) & 1, a.status, abort_flag)) return false;
-        ptx::tc_fence_after();
-        const uint32_t pt = p0 + (t.i & 1) * kPStride;
-        for (int f = 0; f < 8; ++f) {
-          const uint32_t slot = r0 + ((t.slot0 + f) % NS) * kChunk;
+        if (!wait_full(bar + C::bPFull + (t.i & 1), (t.i >> 1) & 1)) return false;
+        const uint32_t pt = p0 + (t.i & 1) * C::kPStride;
+        for (int pb = 0; pb < 4; ++pb) {
+          const int slot = (t.lat0 + pb) % NL;
+          const uint32_t src = l0 + slot * kPair;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t ad = ptx::sdesc(slot + j * 2048, kChunk, 1024, 2);   // V^T, MN-major
-            const uint64_t bd = ptx::sdesc(pt + j * 32, 16, 1024, 2);          // P^T, K-major
-            ptx::mma_bf16_ss(tmem + C::kColO + f * H, ad, bd, idO, (t.first && j == 0) ? 0u : 1u);
+          for (int j = 0; j < 8; ++j) {
+            // A = V^T: chunks 2pb, 2pb + 1 (16 KB apart, MN-major) x tokens 16j..;
+            // B = P^T: H rows x the same tokens (K-major, 64-token chunks)
+            const uint64_t ad = ptx::sdesc(src + 2048 * j, kChunk, 1024, 2);
+            const uint64_t bd = ptx::sdesc(pt + (j >> 2) * H * 128 + 32 * (j & 3), 16, 1024, 2);
+            ptx::mma_bf16_ss(tmem + C::kColO + pb * H, ad, bd, idO, (t.first && j == 0) ? 0u : 1u);
           }
+          ptx::mma_commit(bar + C::bLatEmpty + slot);
         }
-        for (int c = 0; c < 9; ++c) ptx::mma_commit(bar + C::bEmpty + (t.slot0 + c) % NS);
         ptx::mma_commit(bar + C::bPFree + (t.i & 1));
         ptx::mma_commit(bar + C::bODone + (t.i & 1));
         return true;
@@ -352,39 +473,60 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       while (ok && walk_next(w, a, share, pc)) {
         if (!ptx::mbar_wait(bar + C::bQFull, npc & 1, a.status, abort_flag)) { ok = false; break; }
         for (int k = 0; k < pc.ntiles && ok; ++k) {
-          const int slot0 = sc % NS;
-          for (int c = 0; c < 9; ++c) {
-            const int s = sc % NS;
-            if (!ptx::mbar_wait(bar + C::bFull + s, (sc / NS) & 1, a.status, abort_flag)) { ok = false; break; }
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint64_t ad = ptx::sdesc(r0 + s * kChunk + 32 * j, 16, 1024, 2);       // K rows
-              const uint64_t bd = ptx::sdesc(q0 + c * H * 128 + 32 * j, 16, 1024, 2);      // Q rows
-              ptx::mma_bf16_ss(tmem + (i & 1) * H, ad, bd, idS, (c | j) != 0 ? 1u : 0u);
-            }
-            ++sc;
+          const uint32_t dS = tmem + (i & 1) * H;
+          // the rest of S^T(i): the rotary chunk and pairs not issued early
+          if (!early_rope) {
+            if (!wait_full(bar + C::bRopeFull + rope.slot, rope.phase)) { ok = false; break; }
+            s_chunk(r0 + rope.slot * kChunk, 8, dS, true);
+          }
+          const int rope_slot = rope.slot;
+          rope.advance(NR);
+          for (int pb = early_pairs; pb < 4; ++pb) {
+            if (!wait_full(bar + C::bLatFull + lat.slot, lat.phase)) { ok = false; break; }
+            const uint32_t src = l0 + lat.slot * kPair;
+            s_chunk(src, 2 * pb, dS, false);
+            s_chunk(src + kChunk, 2 * pb + 1, dS, false);
+            lat.advance(NL);
           }
           if (!ok) break;
+          ptx::mma_commit(bar + C::bRopeEmpty + rope_slot);   // the rotary chunk only feeds S
           ptx::mma_commit(bar + C::bSFull + (i & 1));
           if (k == pc.ntiles - 1) ptx::mma_commit(bar + C::bQEmpty);
-          if (have_prev && !pv(prev)) { ok = false; break; }
-          prev = {i, k == 0 ? 1 : 0, npc, slot0};
-          have_prev = true;
+          const int this_lat0 = lat_first;
+          // S^T(i+1) chunks whose data needs no slot of tile i, within the piece
+          early_pairs = 0;
+          early_rope = false;
+          if (k + 1 < pc.ntiles) {
+            const uint32_t dN = tmem + ((i + 1) & 1) * H;
+            if (C::kEarlyRope) {
+              if (!wait_full(bar + C::bRopeFull + rope.slot, rope.phase)) { ok = false; break; }
+              s_chunk(r0 + rope.slot * kChunk, 8, dN, true);
+              early_rope = true;
+            }
+            for (int pb = 0; pb < C::kEarlyPairs; ++pb) {
+              if (!wait_full(bar + C::bLatFull + lat.slot, lat.phase)) { ok = false; break; }
+              const uint32_t src = l0 + lat.slot * kPair;
+              s_chunk(src, 2 * pb, dN, !early_rope && pb == 0);
+              s_chunk(src + kChunk, 2 * pb + 1, dN, false);
+              lat.advance(NL);
+              ++early_pairs;
+            }
+            if (!ok) break;
+          }
+          lat_first = (this_lat0 + 4) % NL;
+          // P.V of this tile (its pairs are released as they are consumed)
+          if (!pv({i, k == 0 ? 1 : 0, npc, this_lat0})) { ok = false; break; }
           ++i;
         }
         ++npc;
       }
-      if (ok && have_prev) pv(prev);
     }
   } else if (warp < 6) {
     // --------------------------------------- softmax, rescale and epilogue
-    // M = 64 accumulators live in lanes 0-15 of each 32-lane quarter: this
-    // thread's token (S^T row) or latent column within a block (O^T row) is
-    // 16 * q + lane for lane < 16.
+    // S^T row (token) and O^T row (latent column within a block) of this
+    // thread: 32 q + lane.
     const int q = warp & 3;
-    const bool act = lane < 16;
-    const int row = 16 * q + (lane & 15);
+    const int row = 32 * q + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     float *opart = reinterpret_cast<float *>(a.ws + a.L.opart_off);
     float *lse_out = reinterpret_cast<float *>(a.ws + a.L.lse_off);
@@ -402,7 +544,7 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       }
       for (int k = 0; k < pc.ntiles; ++k, ++i) {
         const int tok = pc.tok_begin + kTileTok * k + row;
-        const bool valid = act && tok < pc.tok_end;
+        const bool valid = tok < pc.tok_end;
         if (!warp_wait(bar + C::bSFull + (i & 1), (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         float s[H];
@@ -414,24 +556,14 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) s[16 * c + j] = valid ? __uint_as_float(r[j]) * a.scale_log2 : -CUDART_INF_F;
         }
-        // per-head maximum over the tile's 64 tokens
-        float mx[H];
+        // per-head maximum over the tile's 128 tokens: 32 lanes, then 4 warps
+        float *rm = red_m + (i & 1) * 4 * H;
 #pragma unroll
         for (int hh = 0; hh < H; ++hh) {
           float v = s[hh];
 #pragma unroll
-          for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          mx[hh] = v;
-        }
-        float *rm = red_m + (i & 1) * 4 * H;
-        if (lane < 16) {
-#pragma unroll
-          for (int hb = 0; hb < H; hb += 16) {
-            float v = mx[hb];
-#pragma unroll
-            for (int j = 1; j < 16; ++j) v = lane == j ? mx[hb + j] : v;
-            rm[q * H + hb + lane] = v;
-          }
+          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (lane == (hh & 31)) rm[q * H + hh] = v;
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar + C::bXchg + (i & 1));
@@ -452,35 +584,34 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
         float p[H];
 #pragma unroll
         for (int hh = 0; hh < H; ++hh) {
-          p[hh] = exp2f(s[hh] - m_run[hh]);
+          p[hh] = ptx::exp2_approx(s[hh] - m_run[hh]);
           l_part[hh] += p[hh];
         }
         if (i >= 2 && !warp_wait(bar + C::bPFree + (i & 1), ((i >> 1) - 1) & 1, a.status, abort_flag)) {
           ok = false;
           break;
         }
-        if (act) {
-          // P^T: K-major rows of 64 tokens (128 B) per head, 16-byte units swizzled by row
-          uint8_t *pt = sP + (i & 1) * kPStride;
-          const int unit = row >> 3, inunit = (row & 7) * 2;
+        {
+          // P^T: K-major rows of 64 tokens (128 B) per head in two chunks,
+          // 16-byte units swizzled by row
+          uint8_t *pt = sP + (i & 1) * C::kPStride + (row >> 6) * H * 128;
+          const int rr = row & 63, unit = rr >> 3, inunit = (rr & 7) * 2;
 #pragma unroll
           for (int hh = 0; hh < H; ++hh)
             *reinterpret_cast<__nv_bfloat16 *>(pt + hh * 128 + ((unit ^ (hh & 7)) << 4) + inunit) =
                 __float2bfloat16_rn(p[hh]);
         }
-        if (any_rescale) {
-          // P.V of the previous tile must be complete before O^T is rescaled.
-          // o_done[b] completes for the P.V of tiles b, b+2, ...; S^T of this
-          // tile being complete implies every P.V up to tile i-2 is (MMAs of
-          // one thread complete in order), so this wait is never more than
-          // one phase away from the barrier's state.
+        if (__any_sync(0xffffffffu, any_rescale)) {
+          // P.V of the previous tile must be complete before O^T is rescaled
+          // (o_done[(i-1)&1] completes with it; nothing later is issued before
+          // this tile's P is full).
           if (!warp_wait(bar + C::bODone + ((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
 #pragma unroll 1
-          for (int f = 0; f < 8; ++f) {
+          for (int f = 0; f < 4; ++f) {
 #pragma unroll
             for (int c = 0; c < H / 16; ++c) {
               uint32_t r[16];
@@ -499,22 +630,13 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
         if (lane == 0) ptx::mbar_arrive(bar + C::bPFull + (i & 1));
       }
       if (!ok) break;
-      // ---- epilogue: per-head sums across the 64 token rows, then O^T / l
+      // ---- epilogue: per-head sums across the 128 token rows, then O^T / l
 #pragma unroll
       for (int hh = 0; hh < H; ++hh) {
-        float v = act ? l_part[hh] : 0.f;
+        float v = l_part[hh];
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        l_part[hh] = v;
-      }
-      if (lane < 16) {
-#pragma unroll
-        for (int hb = 0; hb < H; hb += 16) {
-          float v = l_part[hb];
-#pragma unroll
-          for (int j = 1; j < 16; ++j) v = lane == j ? l_part[hb + j] : v;
-          red_s[q * H + hb + lane] = v;
-        }
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == (hh & 31)) red_s[q * H + hh] = v;
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar + C::bLsum);
@@ -530,18 +652,16 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       if (!warp_wait(bar + C::bODone + ((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
 #pragma unroll 1
-      for (int f = 0; f < 8; ++f) {
+      for (int f = 0; f < 4; ++f) {
 #pragma unroll
         for (int c = 0; c < H / 16; ++c) {
           uint32_t r[16];
           ptx::tmem_ld16(lane_addr + C::kColO + f * H + 16 * c, r);
           ptx::tmem_ld_wait();
-          if (act) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int hh = 16 * c + j;
-              opart[(pc.piece * a.n_h + hh) * (long long)a.d_c + 64 * f + row] = __uint_as_float(r[j]) * inv[hh];
-            }
+          for (int j = 0; j < 16; ++j) {
+            const int hh = 16 * c + j;
+            opart[(pc.piece * a.n_h + hh) * (long long)a.d_c + 128 * f + row] = __uint_as_float(r[j]) * inv[hh];
           }
         }
       }
@@ -552,45 +672,56 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
     }
   } else if (F8) {
     // ------------------------------------------ FP8 converters (warps 6 ..)
-    // A chunk is 64 rows x 4 units of 16 codes.  Thread ct handles unit ct%4
-    // of rows ct/4, ct/4 + RS, ... (RS = rows covered by all converters at
-    // once): 16 codes become 32 bytes of bf16, two 16-byte units of the
-    // 128-byte-swizzled ring row.
-    constexpr int RS = (C::kConvWarps > 0 ? C::kConvWarps : 4) * 8, NR = 64 / RS;
+    // A staged chunk is 128 rows x 4 units of 16 codes.  Thread ct handles
+    // unit ct % 4 of rows ct / 4 + 32 rr (rr = 0..3): 16 codes become 32 bytes
+    // of bf16, two 16-byte units of the 128-byte-swizzled chunk.  Chunks come
+    // in the producer's order: the rotary chunk, then latent chunks 0-7.
+    constexpr int RS = 32, NRR = kTileTok / RS;
     const int ct = (warp - 6) * 32 + lane;
     const int r0 = ct >> 2, u = ct & 3;
     Walk w;
     walk_init(w, a, share);
     Piece pc;
-    int sc = 0;
+    RingPos stg, lat, rope;
     bool ok = true;
+    auto slot_free = [&](uint64_t *empty, const RingPos &r) -> bool {
+      if (r.round == 0) return true;
+      return warp_wait(empty, r.phase ^ 1u, a.status, abort_flag);
+    };
     while (ok && walk_next(w, a, share, pc)) {
       for (int k = 0; k < pc.ntiles && ok; ++k) {
         const int tok0 = pc.tok_begin + kTileTok * k;
-        float sig[NR][kGroups8];
+        float sig[NRR][kGroups8];
 #pragma unroll
-        for (int rr = 0; rr < NR; ++rr) {
+        for (int rr = 0; rr < NRR; ++rr) {
           const int t = tok0 + r0 + RS * rr;
           const long long r = t < pc.ctx ? kv_row(a, pc.b, t) : -1;
 #pragma unroll
           for (int g = 0; g < kGroups8; ++g) sig[rr][g] = r >= 0 ? a.kv_scale[r * kGroups8 + g] : 0.f;
         }
-        for (int c = 0; c < 9; ++c) {
-          const int st = sc % NSt, s = sc % NS;
-          if (!warp_wait(bar + C::bStFull + st, (sc / NSt) & 1, a.status, abort_flag)) { ok = false; break; }
-          if (sc >= NS && !warp_wait(bar + C::bEmpty + s, ((sc / NS) - 1) & 1, a.status, abort_flag)) {
-            ok = false;
-            break;
+        for (int j = 0; j < 9; ++j) {
+          const int c = j == 0 ? 8 : j - 1;
+          if (!warp_wait(bar + C::bStFull + stg.slot, stg.phase, a.status, abort_flag)) { ok = false; break; }
+          uint8_t *dst;
+          uint64_t *full;
+          if (c == 8) {
+            if (!slot_free(bar + C::bRopeEmpty + rope.slot, rope)) { ok = false; break; }
+            dst = sRope + rope.slot * kChunk;
+            full = bar + C::bRopeFull + rope.slot;
+          } else {
+            if ((c & 1) == 0 && !slot_free(bar + C::bLatEmpty + lat.slot, lat)) { ok = false; break; }
+            dst = sLat + lat.slot * kPair + (c & 1) * kChunk;
+            full = bar + C::bLatFull + lat.slot;
           }
           const int g = c >> 1;   // chunks 0-7: c^KV groups 0-3; chunk 8: the k^R group
 #pragma unroll
-          for (int rr = 0; rr < NR; ++rr) {
-            const int row = r0 + RS * rr;
+          for (int rr = 0; rr < NRR; ++rr) {
+            const int rw = r0 + RS * rr;
             // select the group's scale without indexing the array at run time
             float sg = sig[rr][0];
 #pragma unroll
             for (int gg = 1; gg < kGroups8; ++gg) sg = g == gg ? sig[rr][gg] : sg;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(sStage + st * kChunk8 + row * 64 + 16 * u);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(sStage + stg.slot * kChunk8 + rw * 64 + 16 * u);
             uint4 lo, hi;
             lo.x = e4m3x2_to_bf16x2(raw.x, sg);
             lo.y = e4m3x2_to_bf16x2(raw.x >> 16, sg);
@@ -600,17 +731,19 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
             hi.y = e4m3x2_to_bf16x2(raw.z >> 16, sg);
             hi.z = e4m3x2_to_bf16x2(raw.w, sg);
             hi.w = e4m3x2_to_bf16x2(raw.w >> 16, sg);
-            uint8_t *dst = sRing + s * kChunk + row * 128;
-            *reinterpret_cast<uint4 *>(dst + (((2 * u) ^ (row & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4 *>(dst + (((2 * u + 1) ^ (row & 7)) << 4)) = hi;
+            uint8_t *d = dst + rw * 128;
+            *reinterpret_cast<uint4 *>(d + (((2 * u) ^ (rw & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4 *>(d + (((2 * u + 1) ^ (rw & 7)) << 4)) = hi;
           }
           ptx::fence_proxy_async_smem();   // the MMAs read the slot through the async proxy
           __syncwarp();
           if (lane == 0) {
-            ptx::mbar_arrive(bar + C::bFull + s);
-            ptx::mbar_arrive(bar + C::bStEmpty + st);
+            ptx::mbar_arrive(full);
+            ptx::mbar_arrive(bar + C::bStEmpty + stg.slot);
           }
-          ++sc;
+          stg.advance(NSt);
+          if (c == 8) rope.advance(NR);
+          else if (c & 1) lat.advance(NL);
         }
       }
     }
@@ -630,22 +763,36 @@ cudaError_t launch_h(const AttnArgs &a, int P, cudaStream_t s) {
   using C = Cfg<H, F8>;
   const long long rows = a.page_size ? a.cache_len * kTile : (long long)a.B * a.cache_len;
   if (rows <= 0 || rows >= (1ll << 31) - 256) return cudaErrorNotSupported;
-  CUtensorMap mq, mkv;
+  CUtensorMap mq, mkv, mkv64, mpair;
   const uint64_t dq[2] = {576, (uint64_t)a.B * H};
   const uint64_t dkv[2] = {576, (uint64_t)rows};
   const uint64_t st[1] = {576 * 2};
   const uint64_t st8[1] = {576};
-  const uint32_t bq[2] = {64, (uint32_t)H}, bkv[2] = {64, 64};
+  const uint32_t bq[2] = {64, (uint32_t)H}, bkv[2] = {64, kTileTok}, bkv64[2] = {64, 64};
   if (!encode_map_bf16(&mq, a.q_abs, 2, dq, st, bq, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorNotSupported;
-  const bool kv_ok = F8 ? encode_map_u8(&mkv, a.cache, 2, dkv, st8, bkv, CU_TENSOR_MAP_SWIZZLE_NONE)
-                        : encode_map_bf16(&mkv, a.cache, 2, dkv, st, bkv, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!kv_ok) return cudaErrorNotSupported;
+  if (F8) {
+    // codes: 64-byte rows, no swizzle (the converters swizzle the bf16 they write)
+    if (!encode_map_u8(&mkv64, a.cache, 2, dkv, st8, bkv64, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorNotSupported;
+    mkv = mkv64;
+    mpair = mkv64;
+  } else {
+    // The cache viewed as [9 chunks][rows][64 columns]: one box of 128 rows x 2
+    // chunks lands as two 16 KB row-major chunks, a latent pair slot.
+    const uint64_t dkv3[3] = {64, (uint64_t)rows, 9};
+    const uint64_t st3[2] = {576 * 2, 64 * 2};
+    const uint32_t bpair[3] = {64, kTileTok, 2};
+    if (!encode_map_bf16(&mkv, a.cache, 2, dkv, st, bkv, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_bf16(&mkv64, a.cache, 2, dkv, st, bkv64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_bf16(&mpair, a.cache, 3, dkv3, st3, bpair, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorNotSupported;
+  }
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t e = once_per_device(configured, [] {
     return cudaFuncSetAttribute(attn_smallh_kernel<H, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_smallh_kernel<H, F8>, dim3(P), dim3(C::kThreads), C::kSmem, s, 1, mq, mkv, a, rows);
+  return launch_pdl(attn_smallh_kernel<H, F8>, dim3(P), dim3(C::kThreads), C::kSmem, s, 1, mq, mkv, mkv64, mpair,
+                    a, rows);
 }
 
 }  // namespace
