@@ -10,6 +10,12 @@
 //
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates tensor
 // memory and issues MMAs, warps 2-5 run the epilogue.
+//
+// Loads come in groups of G consecutive 64-wide K chunks, one TMA box of G
+// chunks per operand and m tile (3D/4D boxes whose outer dimension steps
+// through the chunks): a thread issuing cp.async.bulk.tensor copies sustains
+// about two copies per microsecond (measured), so these short, weight-
+// streaming GEMMs need few and large copies.
 #include <math_constants.h>
 #include <string.h>
 
@@ -71,7 +77,8 @@ bool encode_map_u8(CUtensorMap *map, const void *base, int rank, const uint64_t 
 namespace {
 
 constexpr int kGemmThreads = 192;
-constexpr int kMaxStages = 8;           // pipeline depth is chosen per launch (<= this)
+constexpr int kMaxStages = 8;           // K-chunk slots of the ring (<= this), a multiple of the group
+constexpr int kMaxGroups = kMaxStages;  // load groups of the ring
 constexpr int kKChunk = 64;           // bf16 elements per 128-byte swizzled row
 constexpr int kABytes = 128 * kKChunk * 2;
 
@@ -80,14 +87,15 @@ enum EpiMode : int { kEpiAbsorb = 0, kEpiOutProj = 1, kEpiWo = 2, kEpiAppend = 3
 struct GemmParams {
   int mode;
   int num_k_chunks;   // K / 64 of the whole product
-  int stages;         // pipeline stages of this launch (<= kMaxStages)
+  int stages;         // K-chunk slots of the ring (<= kMaxStages, a multiple of group)
+  int group;          // K chunks per TMA load group (1, 2 or 4)
   int ksplit;         // K slices per output tile (1, or a cluster of ksplit CTAs along x)
   int mt_per_cta;     // 128-row m tiles one CTA computes, sharing its B tiles (1 when ksplit > 1)
   int m_tiles;        // m tiles of the whole product
   int M_valid;        // valid output features (rows of the product)
   int N;              // valid columns (tokens or sequences)
   int a_split_tile;   // m-tiles >= a_split_tile read map A1 (append: W_KR)
-  int a1_rows;        // rows of map A1's box (bytes of that A tile = a1_rows * 128)
+  int a1_rows;        // rows of map A1's box (<= 128; its chunks are a1_rows * 128 B apart)
   int a_row_per_z;    // added to A's row coordinate per blockIdx.z
   int b_is_3d;        // B map is [N][Z][K] with the head index as middle coordinate
   __nv_bfloat16 *out;
@@ -131,14 +139,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = g.stages;
+  const int G = g.group;
+  const int NG = S / G;                          // load groups in the ring
   const int MT = g.mt_per_cta;
-  const int kStage = MT * kABytes + kBBytes;   // one K chunk: MT A tiles, then the shared B tile
+  // Ring layout, per load group gs: MT A blocks of G chunks (G x 16 KB each),
+  // then the shared B block of G chunks (G x kBBytes).
+  const int kGroupBytes = G * (MT * kABytes + kBBytes);
   const bool split = g.ksplit > 1;
-  // The stage ring; with a K split it is reused afterwards for this CTA's fp32 partial.
-  const int region = split && 128 * BN * 4 > S * kStage ? 128 * BN * 4 : S * kStage;
+  // The ring; with a K split it is reused afterwards for this CTA's fp32 partial.
+  const int region = split && 128 * BN * 4 > NG * kGroupBytes ? 128 * BN * 4 : NG * kGroupBytes;
   uint64_t *full = reinterpret_cast<uint64_t *>(base + region);
-  uint64_t *empty = full + kMaxStages;
-  uint64_t *accf = empty + kMaxStages;
+  uint64_t *empty = full + kMaxGroups;
+  uint64_t *accf = empty + kMaxGroups;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   long long *s_row = reinterpret_cast<long long *>(base + region + 256);
@@ -154,6 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int per = (g.num_k_chunks + g.ksplit - 1) / g.ksplit;
   const int kc0 = zs * per;
   const int nk = max(0, min(g.num_k_chunks, kc0 + per) - kc0);   // K chunks of this CTA
+  const int ngrp = (nk + G - 1) / G;                               // load groups of this CTA
   const int m0 = mt * 128, n0 = nt * BN;
   const bool use_a1 = mt >= g.a_split_tile;   // (only with MT = 1)
   uint32_t tmem_cols = 32;
@@ -161,7 +174,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_trigger();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < NG; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
@@ -185,67 +198,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t a_bytes = use_a1 ? (uint32_t)g.a1_rows * 128u : (uint32_t)kABytes;
       ptx::tma_prefetch_desc(mA);
       ptx::tma_prefetch_desc(&mapB);
-      // The weights (A) never depend on earlier kernels: the first stages'
-      // A tiles are requested before waiting for those kernels, the
-      // activations (B) after.
-      const int pre = nk < S ? nk : S;
-      auto load_a = [&](int kl) {
-        const int s = kl % S, kc = kc0 + kl;
-        uint8_t *sa = base + s * kStage;
-        ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)mcount * a_bytes + (uint32_t)kBBytes);
+      // The weights (A) never depend on earlier kernels: the first groups'
+      // A blocks are requested before waiting for those kernels, the
+      // activations (B) after.  A group always loads G whole chunks (a last
+      // group past the slice's end loads chunks its MMAs skip).
+      const int pre = ngrp < NG ? ngrp : NG;
+      auto load_a = [&](int gi) {
+        const int s = gi % NG, kc = kc0 + gi * G;
+        uint8_t *sa = base + s * kGroupBytes;
+        ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)G * ((uint32_t)mcount * a_bytes + (uint32_t)kBBytes));
         for (int t = 0; t < mcount; ++t) {
-          uint8_t *st = sa + t * kABytes;
+          uint8_t *st = sa + t * G * kABytes;
           if (A_MN) {
-            const int krow = z * g.a_row_per_z + kc * kKChunk;
-            ptx::tma_load_2d(st, mA, &full[s], a_m0 + 128 * t, krow);
-            ptx::tma_load_2d(st + kABytes / 2, mA, &full[s], a_m0 + 128 * t + 64, krow);
+            // [2 m halves][64 G k rows][64 m]: m chunks 2 (mt + t), +1
+            ptx::tma_load_3d(st, mA, &full[s], 0, z * g.a_row_per_z + kc * kKChunk, 2 * (a_m0 / 128 + t));
           } else {
-            ptx::tma_load_2d(st, mA, &full[s], kc * kKChunk, z * g.a_row_per_z + a_m0 + 128 * t);
+            // [G chunks][rows][64 k]
+            ptx::tma_load_3d(st, mA, &full[s], 0, z * g.a_row_per_z + a_m0 + 128 * t, kc);
           }
         }
       };
-      auto load_b = [&](int kl) {
-        const int s = kl % S, kc = kc0 + kl;
-        uint8_t *sb = base + s * kStage + MT * kABytes;
-        if (g.b_is_3d) ptx::tma_load_3d(sb, &mapB, &full[s], kc * kKChunk, z, n0);
-        else ptx::tma_load_2d(sb, &mapB, &full[s], kc * kKChunk, n0);
+      auto load_b = [&](int gi) {
+        const int s = gi % NG, kc = kc0 + gi * G;
+        uint8_t *sb = base + s * kGroupBytes + MT * G * kABytes;
+        if (g.b_is_3d) ptx::tma_load_4d(sb, &mapB, &full[s], 0, n0, kc, z);
+        else ptx::tma_load_3d(sb, &mapB, &full[s], 0, n0, kc);
       };
-      for (int kl = 0; kl < pre; ++kl) load_a(kl);
+      for (int gi = 0; gi < pre; ++gi) load_a(gi);
       pdl_wait();
-      for (int kl = 0; kl < pre; ++kl) load_b(kl);
+      for (int gi = 0; gi < pre; ++gi) load_b(gi);
       int issued = pre;
-      for (int kl = pre; kl < nk; ++kl) {
-        const int s = kl % S;
-        if (!ptx::mbar_wait(&empty[s], ((kl / S) - 1) & 1, g.status, abort_flag)) break;
+      for (int gi = pre; gi < ngrp; ++gi) {
+        const int s = gi % NG;
+        if (!ptx::mbar_wait(&empty[s], ((gi / NG) - 1) & 1, g.status, abort_flag)) break;
         ++issued;
-        load_a(kl);
-        load_b(kl);
+        load_a(gi);
+        load_b(gi);
       }
       // Drain: do not leave while loads into this CTA's shared memory are in flight.
-      for (int kl = issued - S > 0 ? issued - S : 0; kl < issued; ++kl) {
+      for (int gi = issued - NG > 0 ? issued - NG : 0; gi < issued; ++gi) {
         volatile int no_abort = 0;
-        ptx::mbar_wait(&full[kl % S], (kl / S) & 1, g.status, &no_abort);
+        ptx::mbar_wait(&full[gi % NG], (gi / NG) & 1, g.status, &no_abort);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, BN, A_MN, false);
-      for (int kl = 0; kl < nk; ++kl) {
-        const int s = kl % S;
-        if (!ptx::mbar_wait(&full[s], (kl / S) & 1, g.status, abort_flag)) break;
+      for (int gi = 0; gi < ngrp; ++gi) {
+        const int s = gi % NG;
+        if (!ptx::mbar_wait(&full[s], (gi / NG) & 1, g.status, abort_flag)) break;
         ptx::tc_fence_after();
-        const uint32_t sa = ptx::smem_u32(base + s * kStage);
-        const uint32_t sb = sa + MT * kABytes;
-        for (int t = 0; t < mcount; ++t) {
-          const uint32_t st = sa + t * kABytes;
+        const uint32_t sa = ptx::smem_u32(base + s * kGroupBytes);
+        const uint32_t sb = sa + MT * G * kABytes;
+        // K-major A chunks lie a box's rows x 128 B apart (a shorter A1 box
+        // leaves the tile's last rows holding other data: those output rows
+        // are past M_valid and never written)
+        const uint32_t a_step = use_a1 ? (uint32_t)g.a1_rows * 128u : (uint32_t)kABytes;
+        for (int j = 0; j < G && gi * G + j < nk; ++j) {
+          const int kl = gi * G + j;
+          for (int t = 0; t < mcount; ++t) {
+            const uint32_t st = sa + t * G * kABytes;
 #pragma unroll
-          for (int j = 0; j < kKChunk / 16; ++j) {
-            // A: K-major rows of 128 B (advance 32 B per 16-element k step), or
-            //    MN-major: 64-wide m chunks 8 KB apart, k rows 128 B apart.
-            const uint64_t ad = A_MN ? ptx::sdesc(st + j * 2048, kABytes / 2, 1024, 2)
-                                     : ptx::sdesc(st + j * 32, 16, 1024, 2);
-            const uint64_t bd = ptx::sdesc(sb + j * 32, 16, 1024, 2);
-            ptx::mma_bf16_ss(tmem + t * BN, ad, bd, idesc, (kl | j) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < kKChunk / 16; ++kk) {
+              // A: K-major rows of 128 B (advance 32 B per 16-element k step), or
+              //    MN-major: 64-wide m halves G * 8 KB apart, k rows 128 B apart.
+              const uint64_t ad = A_MN ? ptx::sdesc(st + j * 8192 + kk * 2048, G * 8192, 1024, 2)
+                                       : ptx::sdesc(st + j * a_step + kk * 32, 16, 1024, 2);
+              const uint64_t bd = ptx::sdesc(sb + j * kBBytes + kk * 32, 16, 1024, 2);
+              ptx::mma_bf16_ss(tmem + t * BN, ad, bd, idesc, (kl | kk) != 0 ? 1u : 0u);
+            }
           }
         }
         ptx::mma_commit(&empty[s]);
@@ -431,19 +452,36 @@ constexpr int b_bytes() { return BN * kKChunk * 2; }
 template <int BN>
 constexpr size_t smem_tail() { return 256 + (size_t)BN * (8 + 4); }
 
+size_t smem_tail_of(int bn) { return 256 + (size_t)bn * (8 + 4); }
+
+// Group G (K chunks per TMA box): G divides the slice's chunk count when it
+// can, and the ring holds two groups (or the whole slice) in shared memory.
+int pick_group(int per, int bn, int mt) {
+  const int chunk = mt * kABytes + bn * kKChunk * 2;
+  int max_chunks = (int)((kSmemLimit - 1024 - smem_tail_of(bn)) / chunk);
+  if (max_chunks > kMaxStages) max_chunks = kMaxStages;
+  for (int cand : {4, 2})
+    if (per % cand == 0 && (2 * cand <= max_chunks || (per == cand && cand <= max_chunks))) return cand;
+  return 1;
+}
+
 template <int BN, bool A_MN>
 cudaError_t launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, GemmParams g,
                         int mtiles, int ntiles, int nz, cudaStream_t s) {
   if (g.mt_per_cta < 1 || (g.ksplit > 1 && g.mt_per_cta != 1) || g.mt_per_cta * BN > 512)
     return cudaErrorNotSupported;
   g.m_tiles = mtiles;
-  const int stage = g.mt_per_cta * kABytes + b_bytes<BN>();
+  const int chunk = g.mt_per_cta * kABytes + b_bytes<BN>();   // one K chunk's A and B
   const int per = (g.num_k_chunks + g.ksplit - 1) / g.ksplit;
-  int max_st = (int)((kSmemLimit - 1024 - smem_tail<BN>()) / stage);
-  if (max_st > kMaxStages) max_st = kMaxStages;
-  if (max_st < 1) return cudaErrorNotSupported;
-  g.stages = per < max_st ? (per > 0 ? per : 1) : max_st;
-  size_t region = (size_t)g.stages * stage;
+  int max_chunks = (int)((kSmemLimit - 1024 - smem_tail<BN>()) / chunk);
+  if (max_chunks > kMaxStages) max_chunks = kMaxStages;
+  const int G = g.group;
+  if (G < 1 || max_chunks < G) return cudaErrorNotSupported;
+  int ng = max_chunks / G;
+  const int need = (per + G - 1) / G;
+  if (ng > need) ng = need > 0 ? need : 1;
+  g.stages = ng * G;
+  size_t region = (size_t)g.stages * chunk;
   if (g.ksplit > 1 && (size_t)128 * BN * 4 > region) region = (size_t)128 * BN * 4;
   const size_t smem = 1024 + region + smem_tail<BN>();
   if (smem > kSmemLimit) return cudaErrorNotSupported;
@@ -468,28 +506,71 @@ int pick_ksplit(long long ctas, int num_k_chunks) {
   return ks;
 }
 
-template <bool A_MN>
-cudaError_t dispatch_bn(int N, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
-                        GemmParams g, int mtiles, int z, cudaStream_t s, int bn) {
-  const int ntiles = (N + bn - 1) / bn;
-  if (g.mt_per_cta == 0) g.mt_per_cta = 1;
-  if (g.ksplit == 0)
-    g.ksplit = g.mt_per_cta > 1 ? 1 : pick_ksplit((long long)mtiles * ntiles * z, g.num_k_chunks);
-  switch (bn) {
-    case 16: return launch_gemm<16, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
-    case 32: return launch_gemm<32, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
-    case 64: return launch_gemm<64, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
-    case 128: return launch_gemm<128, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
-    default: return launch_gemm<256, A_MN>(a0, a1, b, g, mtiles, ntiles, z, s);
-  }
-}
-
 int pick_bn(long long N) {
   if (N <= 16) return 16;
   if (N <= 32) return 32;
   if (N <= 64) return 64;
   if (N <= 128) return 128;
   return 256;
+}
+
+// Tensor maps of one launch: A (two, for a product whose rows come from two
+// weights) and B, built for the chosen group G and N tile bn.
+struct Maps {
+  CUtensorMap a0, a1, b;
+};
+
+// Chooses bn, the K split and the group, lets `encode(G, bn, maps)` build the
+// tensor maps, and launches.
+template <bool A_MN, typename Encode>
+cudaError_t dispatch(int N, GemmParams g, int mtiles, int z, cudaStream_t s, Encode encode) {
+  const int bn = pick_bn(N);
+  const int ntiles = (N + bn - 1) / bn;
+  if (g.mt_per_cta == 0) g.mt_per_cta = 1;
+  if (g.ksplit == 0)
+    g.ksplit = g.mt_per_cta > 1 ? 1 : pick_ksplit((long long)mtiles * ntiles * z, g.num_k_chunks);
+  const int per = (g.num_k_chunks + g.ksplit - 1) / g.ksplit;
+  g.group = pick_group(per, bn, g.mt_per_cta);
+  Maps m;
+  if (!encode(g.group, bn, m)) return cudaErrorNotSupported;
+  switch (bn) {
+    case 16: return launch_gemm<16, A_MN>(m.a0, m.a1, m.b, g, mtiles, ntiles, z, s);
+    case 32: return launch_gemm<32, A_MN>(m.a0, m.a1, m.b, g, mtiles, ntiles, z, s);
+    case 64: return launch_gemm<64, A_MN>(m.a0, m.a1, m.b, g, mtiles, ntiles, z, s);
+    case 128: return launch_gemm<128, A_MN>(m.a0, m.a1, m.b, g, mtiles, ntiles, z, s);
+    default: return launch_gemm<256, A_MN>(m.a0, m.a1, m.b, g, mtiles, ntiles, z, s);
+  }
+}
+
+// A, K-major: a row-major weight [rows][K] viewed as [K/64 chunks][rows][64];
+// a box of G chunks x box_rows rows (rows past the weight are zero-filled).
+bool map_a_kmajor(CUtensorMap *m, const void *w, uint64_t K, uint64_t rows, int G, uint32_t box_rows = 128) {
+  const uint64_t d[3] = {64, rows, K / 64};
+  const uint64_t st[2] = {K * 2, 128};
+  const uint32_t box[3] = {64, box_rows, (uint32_t)G};
+  return encode_map_bf16(m, w, 3, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// A, MN-major: a row-major weight [K rows][M] viewed as [M/64 chunks][K][64];
+// a box of 2 m chunks (one 128-row m tile) x 64 G k rows.
+bool map_a_mnmajor(CUtensorMap *m, const void *w, uint64_t M, uint64_t krows, int G) {
+  const uint64_t d[3] = {64, krows, M / 64};
+  const uint64_t st[2] = {M * 2, 128};
+  const uint32_t box[3] = {64, (uint32_t)(64 * G), 2};
+  return encode_map_bf16(m, w, 3, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// B: row-major activations [N][K] viewed as [K/64][N][64]; a box of G chunks x bn rows.
+bool map_b(CUtensorMap *m, const void *x, uint64_t K, uint64_t N, int bn, int G) {
+  const uint64_t d[3] = {64, N, K / 64};
+  const uint64_t st[2] = {K * 2, 128};
+  const uint32_t box[3] = {64, (uint32_t)bn, (uint32_t)G};
+  return encode_map_bf16(m, x, 3, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// B per head: activations [N][Z][K] viewed as [Z][K/64][N][64]; a box of G chunks x bn rows of one head.
+bool map_b_heads(CUtensorMap *m, const void *x, uint64_t K, uint64_t Z, uint64_t N, int bn, int G) {
+  const uint64_t d[4] = {64, N, K / 64, Z};
+  const uint64_t st[3] = {Z * K * 2, 128, K * 2};
+  const uint32_t box[4] = {64, (uint32_t)bn, (uint32_t)G, 1};
+  return encode_map_bf16(m, x, 4, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -507,24 +588,10 @@ GemmParams blank_params() {
 // ---------------------------------------------------------------------------
 cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void *q_rope, const int *pos,
                              const void *w_uk, void *q_abs, int B, const double *theta, cudaStream_t s) {
-  if (!aligned16(q_nope) || !aligned16(w_uk)) return cudaErrorNotSupported;
-  const int bn = pick_bn(B);
-  CUtensorMap ma, mb;
-  const uint64_t da[2] = {(uint64_t)c.d_c, (uint64_t)c.n_h * c.d_h};
-  const uint64_t sa[1] = {(uint64_t)c.d_c * 2};
-  const uint32_t ba[2] = {64, 64};
-  const uint64_t db[3] = {(uint64_t)c.d_h, (uint64_t)c.n_h, (uint64_t)B};
-  const uint64_t sb[2] = {(uint64_t)c.d_h * 2, (uint64_t)c.n_h * c.d_h * 2};
-  const uint32_t bb[3] = {64, 1, (uint32_t)bn};
-  if (!encode_map_bf16(&ma, w_uk, 2, da, sa, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mb, q_nope, 3, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorNotSupported;
+  if (!aligned16(q_nope) || !aligned16(w_uk) || c.d_h % 64 != 0) return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiAbsorb;
-  // One m tile per CTA: 512 short CTAs measured faster here (30.7 us at B=64)
-  // than 256 or 128 CTAs that share q^C across 2 or 4 tiles (32.9 / 41.0 us),
-  // whose single TMA-issuing thread then streams twice or four times as many
-  // boxes.
+  // One m tile per CTA (512 CTAs at DeepSeek-V2 shapes).
   g.mt_per_cta = 1;
   g.num_k_chunks = c.d_h / kKChunk;
   g.M_valid = c.d_c;
@@ -540,23 +607,17 @@ cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void
   g.d_c = c.d_c;
   g.d_r = c.d_r;
   g.n_h = c.n_h;
-  return dispatch_bn<true>(B, ma, ma, mb, g, c.d_c / 128, c.n_h, s, bn);
+  return dispatch<true>(B, g, c.d_c / 128, c.n_h, s, [&](int G, int bn, Maps &m) {
+    // W^UK [n_h d_h, d_c]: row k of head z is k-row z d_h + k, the d_c columns are m.
+    if (!map_a_mnmajor(&m.a0, w_uk, c.d_c, (uint64_t)c.n_h * c.d_h, G)) return false;
+    m.a1 = m.a0;
+    return map_b_heads(&m.b, q_nope, c.d_h, c.n_h, B, bn, G);
+  });
 }
 
 cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const void *w_uv, void *o, int B,
                               cudaStream_t s) {
   if (!aligned16(ctx_lat) || !aligned16(w_uv) || c.d_h % 128 != 0) return cudaErrorNotSupported;
-  const int bn = pick_bn(B);
-  CUtensorMap ma, mb;
-  const uint64_t da[2] = {(uint64_t)c.d_c, (uint64_t)c.n_h * c.d_h};
-  const uint64_t sa[1] = {(uint64_t)c.d_c * 2};
-  const uint32_t ba[2] = {64, 128};
-  const uint64_t db[3] = {(uint64_t)c.d_c, (uint64_t)c.n_h, (uint64_t)B};
-  const uint64_t sb[2] = {(uint64_t)c.d_c * 2, (uint64_t)c.n_h * c.d_c * 2};
-  const uint32_t bb[3] = {64, 1, (uint32_t)bn};
-  if (!encode_map_bf16(&ma, w_uv, 2, da, sa, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mb, ctx_lat, 3, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiOutProj;
   g.num_k_chunks = c.d_c / kKChunk;
@@ -567,23 +628,16 @@ cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const vo
   g.out = (__nv_bfloat16 *)o;
   g.out_ld = (long long)c.n_h * c.d_h;
   g.out_z = c.d_h;
-  return dispatch_bn<false>(B, ma, ma, mb, g, c.d_h / 128, c.n_h, s, bn);
+  return dispatch<false>(B, g, c.d_h / 128, c.n_h, s, [&](int G, int bn, Maps &m) {
+    if (!map_a_kmajor(&m.a0, w_uv, c.d_c, (uint64_t)c.n_h * c.d_h, G)) return false;
+    m.a1 = m.a0;
+    return map_b_heads(&m.b, ctx_lat, c.d_c, c.n_h, B, bn, G);
+  });
 }
 
 cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, cudaStream_t s) {
   // y[N, M] = x[N, K] w[M, K]^T, bf16 in and out, fp32 accumulation.
   if (!aligned16(x) || !aligned16(w) || K % 64 != 0 || M <= 0 || N <= 0) return cudaErrorNotSupported;
-  const int bn = pick_bn(N);
-  CUtensorMap ma, mb;
-  const uint64_t da[2] = {(uint64_t)K, (uint64_t)M};
-  const uint64_t sa[1] = {(uint64_t)K * 2};
-  const uint32_t ba[2] = {64, 128};
-  const uint64_t db[2] = {(uint64_t)K, (uint64_t)N};
-  const uint64_t sb[1] = {(uint64_t)K * 2};
-  const uint32_t bb[2] = {64, (uint32_t)bn};
-  if (!encode_map_bf16(&ma, w, 2, da, sa, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mb, x, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiWo;
   g.num_k_chunks = K / kKChunk;
@@ -591,7 +645,11 @@ cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K
   g.N = N;
   g.out = (__nv_bfloat16 *)y;
   g.out_ld = M;
-  return dispatch_bn<false>(N, ma, ma, mb, g, (M + 127) / 128, 1, s, bn);
+  return dispatch<false>(N, g, (M + 127) / 128, 1, s, [&](int G, int bn, Maps &m) {
+    if (!map_a_kmajor(&m.a0, w, K, M, G)) return false;
+    m.a1 = m.a0;
+    return map_b(&m.b, x, K, N, bn, G);
+  });
 }
 
 cudaError_t launch_wo_tc(const mla_config &c, const void *o, const void *w_o, void *u, int B, cudaStream_t s) {
@@ -605,27 +663,13 @@ cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, c
   if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr)) return cudaErrorNotSupported;
   const long long N = (long long)B * T;
   if (N > 65535LL * 256) return cudaErrorNotSupported;
-  const int bn = pick_bn(N);
-  const int a1_rows = c.d_r < 128 ? c.d_r : 128;
-  CUtensorMap m0, m1, mb;
-  const uint64_t d0[2] = {(uint64_t)c.d_model, (uint64_t)c.d_c};
-  const uint64_t d1[2] = {(uint64_t)c.d_model, (uint64_t)c.d_r};
-  const uint64_t sw[1] = {(uint64_t)c.d_model * 2};
-  const uint32_t b0[2] = {64, 128};
-  const uint32_t b1[2] = {64, (uint32_t)a1_rows};
-  const uint64_t db[2] = {(uint64_t)c.d_model, (uint64_t)N};
-  const uint32_t bb[2] = {64, (uint32_t)bn};
-  if (!encode_map_bf16(&m0, w_dkv, 2, d0, sw, b0, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&m1, w_kr, 2, d1, sw, b1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_bf16(&mb, h, 2, db, sw, bb, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiAppend;
   g.num_k_chunks = c.d_model / kKChunk;
   g.M_valid = c.d_c + c.d_r;
   g.N = (int)N;
   g.a_split_tile = c.d_c / 128;
-  g.a1_rows = a1_rows;
+  g.a1_rows = c.d_r < 128 ? c.d_r : 128;
   g.out = (__nv_bfloat16 *)cache;
   g.theta = theta;
   g.d_c = c.d_c;
@@ -639,7 +683,12 @@ cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, c
   g.out_f32 = rows_out;
   g.status = status;
   const int mtiles = c.d_c / 128 + (c.d_r + 127) / 128;
-  return dispatch_bn<false>((int)N, m0, m1, mb, g, mtiles, 1, s, bn);
+  return dispatch<false>((int)N, g, mtiles, 1, s, [&](int G, int bn, Maps &m) {
+    // W^DKV rows form the c^KV tiles, W^KR (d_r rows) the last tile
+    return map_a_kmajor(&m.a0, w_dkv, c.d_model, c.d_c, G) &&
+           map_a_kmajor(&m.a1, w_kr, c.d_model, c.d_r, G, (uint32_t)g.a1_rows) &&
+           map_b(&m.b, h, c.d_model, N, bn, G);
+  });
 }
 
 }  // namespace mla
