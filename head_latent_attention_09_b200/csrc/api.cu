@@ -57,6 +57,17 @@ int default_parts(const mla_handle *h) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Appends to theta[0 .. nth) (double) the float pairs (hi, lo) with
+// hi + lo = theta[k] to about 2^-48 (the second half of the table).
+void split_theta(double *theta, int nth) {
+  float *pairs = reinterpret_cast<float *>(theta + nth);
+  for (int k = 0; k < nth; ++k) {
+    const float hi = (float)theta[k];
+    pairs[2 * k] = hi;
+    pairs[2 * k + 1] = (float)(theta[k] - (double)hi);
+  }
+}
+
 // Strict mode: a tensor-core kernel that exists for the configuration but
 // could not take the call's arguments is not replaced by a CUDA-core kernel.
 bool strict_refuses(const mla_handle *h, bool tc_exists, cudaError_t e) {
@@ -117,12 +128,13 @@ int mla_create(const mla_config *cfg, mla_handle **out) {
     return MLA_ERR_CUDA;
   }
   const int nth = cfg->d_r / 2;
-  double *theta = (double *)malloc(sizeof(double) * nth);
+  double *theta = (double *)malloc(2 * sizeof(double) * nth);
   for (int k = 0; k < nth; ++k) theta[k] = pow(cfg->rope_base, -2.0 * k / (double)cfg->d_r);
+  split_theta(theta, nth);
   cudaError_t e = cudaMalloc(&h->d_status, sizeof(unsigned));
-  if (e == cudaSuccess) e = cudaMalloc(&h->d_theta, sizeof(double) * nth);
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_theta, 2 * sizeof(double) * nth);
   if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(unsigned));
-  if (e == cudaSuccess) e = cudaMemcpy(h->d_theta, theta, sizeof(double) * nth, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->d_theta, theta, 2 * sizeof(double) * nth, cudaMemcpyHostToDevice);
   free(theta);
   if (e != cudaSuccess) {
     mla_destroy(h);
@@ -148,7 +160,7 @@ int mla_set_rope_scaling(mla_handle *h, double factor, int original_ctx, double 
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   if (dev != h->device) return MLA_ERR_INVALID_ARG;
   const int d_r = h->cfg.d_r, nth = d_r / 2;
-  double *theta = (double *)malloc(sizeof(double) * (nth > 0 ? nth : 1));
+  double *theta = (double *)malloc(2 * sizeof(double) * (nth > 0 ? nth : 1));
   if (!theta) return MLA_ERR_CUDA;
   for (int k = 0; k < nth; ++k) {
     const double th = pow(h->cfg.rope_base, -2.0 * k / (double)d_r);
@@ -160,7 +172,8 @@ int mla_set_rope_scaling(mla_handle *h, double factor, int original_ctx, double 
     }
     theta[k] = keep * th + (1.0 - keep) * th / factor;
   }
-  const cudaError_t e = cudaMemcpy(h->d_theta, theta, sizeof(double) * nth, cudaMemcpyHostToDevice);
+  split_theta(theta, nth);
+  const cudaError_t e = cudaMemcpy(h->d_theta, theta, 2 * sizeof(double) * nth, cudaMemcpyHostToDevice);
   free(theta);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   const double m = factor > 1.0 ? mscale_coef * log(factor) + 1.0 : 1.0;

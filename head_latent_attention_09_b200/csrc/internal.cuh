@@ -43,6 +43,31 @@ enum GemmKind : int { kGemmSimt = 0, kGemmTc = 1 };
 
 namespace mla {
 
+// cos and sin of the rotary angle pos * theta in single precision, accurate
+// at positions up to 2^24.  theta is given as an unevaluated float sum
+// hi + lo (its double value split in two); the product pos * hi is kept with
+// its exact rounding error (fma), so the angle carries ~2^-48 relative error
+// (a plain float product would err by ~1e-2 rad near position 131072), and it
+// is reduced to [-pi, pi] with a three-part split of 2 pi (Cody and Waite).
+// Error of the reduced angle: a few 1e-7 rad; the hardware sine and cosine on
+// [-pi, pi] add at most ~4e-7 (far below the bf16 rounding of the results).
+__device__ __forceinline__ void rope_sincos(int pos, float2 theta, float *s, float *c) {
+  const float p = (float)pos;                                   // exact below 2^24
+  const float a_hi = p * theta.x;
+  const float a_lo = fmaf(p, theta.x, -a_hi) + p * theta.y;
+  const float k = rintf(a_hi * 0.15915494309189535f);          // whole turns
+  float r = fmaf(-k, 6.28125f, a_hi);                           // 2 pi = 6.28125 + 1.93548e-3 - 1.74846e-7
+  r = fmaf(-k, 1.9354820251464844e-3f, r);
+  r = fmaf(-k, -1.7484555314695172e-7f, r);
+  __sincosf(r + a_lo, s, c);
+}
+
+// The handle's frequency table: theta_k in double [d_r / 2], then the same
+// values split into float pairs (hi, lo) [d_r / 2], in one allocation.
+__host__ __device__ inline const float2 *theta_pairs(const double *theta, int d_r) {
+  return reinterpret_cast<const float2 *>(theta + d_r / 2);
+}
+
 // Programmatic dependent launch.  Kernels of this library are launched so
 // that the next kernel in the stream may begin while the current one
 // finishes (its set-up overlapping the tail); each kernel signals that its
@@ -86,7 +111,7 @@ struct mla_handle {
   int device;
   int num_sms;
   unsigned *d_status;  // device status word (kStatus* bits)
-  double *d_theta;     // device [d_r/2] RoPE frequencies theta_k
+  double *d_theta;     // device RoPE frequencies theta_k: [d_r/2] double, then [d_r/2] float (hi, lo) pairs
   double score_mult;   // YaRN temperature t multiplying every score (1 without scaling)
   int attn_kind;       // mla::AttnKind
   int gemm_kind;       // mla::GemmKind

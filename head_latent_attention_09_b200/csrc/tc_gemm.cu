@@ -104,7 +104,7 @@ struct GemmParams {
   // absorb: rotary part of the query
   const __nv_bfloat16 *q_rope;
   const int *pos;
-  const double *theta;
+  const float2 *theta;   // rotary frequencies as float (hi, lo) pairs
   int d_c, d_r, n_h;
   // append: destination rows
   int T;
@@ -297,6 +297,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
+    if (g.mode == kEpiAbsorb && zs == 0) {
+      // Rotary part of the absorbed query, q_abs[b, z, d_c + 2k (+1)] =
+      // RoPE(q_rope[b, z], pos[b]): independent of the product, so done while
+      // the MMAs run, shared out over the head's m-tile CTAs.  Eight elements
+      // per thread at a time, all their loads issued before any use.
+      const int npair = g.d_r / 2;
+      const int ncol = min(BN, g.N - n0);
+      const int total = ncol * npair;
+      const int stride = 128 * g.m_tiles;
+      for (int idx0 = et + 128 * mt; idx0 < total; idx0 += stride * 8) {
+        __nv_bfloat162 xr[8];
+        int pp[8];
+        float2 th[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int idx = idx0 + stride * u;
+          if (idx < total) {
+            const int n = n0 + idx / npair, k = idx % npair;
+            xr[u] = *reinterpret_cast<const __nv_bfloat162 *>(g.q_rope + ((long long)n * g.n_h + z) * g.d_r + 2 * k);
+            pp[u] = g.pos[n];
+            th[u] = g.theta[k];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int idx = idx0 + stride * u;
+          if (idx < total) {
+            const int n = n0 + idx / npair, k = idx % npair;
+            const float x0 = __low2float(xr[u]), x1 = __high2float(xr[u]);
+            float s, c;
+            rope_sincos(pp[u], th[u], &s, &c);
+            *reinterpret_cast<__nv_bfloat162 *>(g.out + (long long)n * g.out_ld + (long long)z * g.out_z + g.d_c +
+                                                2 * k) = __floats2bfloat162_rn(x0 * c - x1 * s, x0 * s + x1 * c);
+          }
+        }
+      }
+    }
     const bool ok = ptx::mbar_wait(accf, 0, g.status, abort_flag);
     ptx::tc_fence_after();
     const int q = warp & 3;
@@ -336,9 +373,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
               const int k = m_local >> 1;
               if (mm_ok && n < g.N && k < g.d_r / 2) {
-                double sn, cs;
-                sincos((double)s_pos[c0 + j] * g.theta[k], &sn, &cs);
-                const float c = (float)cs, s = (float)sn;
+                float s, c;
+                rope_sincos(s_pos[c0 + j], g.theta[k], &s, &c);
                 v = (lane & 1) ? partner * s + v * c : v * c - partner * s;
               }
             }
@@ -354,22 +390,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-      }
-    }
-    if (g.mode == kEpiAbsorb && mt == 0 && zs == 0) {
-      // rotary part of the absorbed query: q_abs[b, z, d_c + 2k (+1)] = RoPE(q_rope[b, z], pos[b])
-      const int npair = g.d_r / 2;
-      const int ncol = min(BN, g.N - n0);
-      for (int idx = et; idx < ncol * npair; idx += 128) {
-        const int n = n0 + idx / npair, k = idx % npair;
-        const long long src = ((long long)n * g.n_h + z) * g.d_r + 2 * k;
-        const float x0 = __bfloat162float(g.q_rope[src]), x1 = __bfloat162float(g.q_rope[src + 1]);
-        double sn, cs;
-        sincos((double)g.pos[n] * g.theta[k], &sn, &cs);
-        const float c = (float)cs, s = (float)sn;
-        __nv_bfloat16 *dst = g.out + (long long)n * g.out_ld + (long long)z * g.out_z + g.d_c + 2 * k;
-        dst[0] = __float2bfloat16_rn(x0 * c - x1 * s);
-        dst[1] = __float2bfloat16_rn(x0 * s + x1 * c);
       }
     }
   }
@@ -413,9 +433,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int e = 0; e < 4; e += 2) {
             const int k = (ml + e) >> 1;
             if (k < g.d_r / 2) {
-              double sn, cs;
-              sincos((double)s_pos[c] * g.theta[k], &sn, &cs);
-              const float co = (float)cs, si = (float)sn;
+              float si, co;
+              rope_sincos(s_pos[c], g.theta[k], &si, &co);
               const float x0 = v[e], x1 = v[e + 1];
               v[e] = x0 * co - x1 * si;
               v[e + 1] = x0 * si + x1 * co;
@@ -603,7 +622,7 @@ cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void
   g.out_z = c.d_c + c.d_r;
   g.q_rope = (const __nv_bfloat16 *)q_rope;
   g.pos = pos;
-  g.theta = theta;
+  g.theta = theta_pairs(theta, c.d_r);
   g.d_c = c.d_c;
   g.d_r = c.d_r;
   g.n_h = c.n_h;
@@ -671,7 +690,7 @@ cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, c
   g.a_split_tile = c.d_c / 128;
   g.a1_rows = c.d_r < 128 ? c.d_r : 128;
   g.out = (__nv_bfloat16 *)cache;
-  g.theta = theta;
+  g.theta = theta_pairs(theta, c.d_r);
   g.d_c = c.d_c;
   g.d_r = c.d_r;
   g.T = T;
