@@ -51,6 +51,8 @@ def parse():
                     help="skip the separate timings of the other workloads (V2-Lite, ragged paged, 128K)")
     ap.add_argument("--attn-samples", type=int, default=200,
                     help="attention calls timed one by one for the median and p10/p90")
+    ap.add_argument("--fused", action="store_true",
+                    help="finish the step with mla_combine_out_proj instead of mla_combine_splits + mla_out_proj")
     ap.add_argument("--launch-check", action="store_true",
                     help="only start the ranks, join the process group (gloo without a GPU) and "
                          "report the ranks seen; no GPU work")
@@ -553,6 +555,15 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
+    def finish(o_out, lse_out):
+        # merge of the split partials and the output projection: two calls
+        # (the faster in the step, measured), or (--fused) mla_combine_out_proj
+        if args.fused:
+            M.mla_combine_out_proj(handle, ws, ws_bytes, B, P, w_uv, None, o_out, None, None, lse_out, sh)
+        else:
+            M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse_out, sh)
+            M.mla_out_proj(handle, ctx_lat, w_uv, None, o_out, None, B, sh)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -565,12 +576,9 @@ def run_ours(args):
         M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, ctx_d, B, P, ws, ws_bytes, sh)
         if ev is not None:
             ev[3].record(stream)
-        M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
+        finish(o, lse)
         if ev is not None:
             ev[4].record(stream)
-        M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
-        if ev is not None:
-            ev[5].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -588,8 +596,7 @@ def run_ours(args):
         ev[0].record(stream)
         M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, ctx_d, B, P, ws, ws_bytes, sh)
         ev[1].record(stream)
-        M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
-        M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+        finish(o, lse)
 
     clocks = ClockSampler(dev)
     clocks.start()
@@ -614,13 +621,29 @@ def run_ours(args):
 
     # ---- per-call breakdown (a separate pass after the timed region: events
     # between every call, so no call overlaps its neighbours here)
-    call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     for i in range(args.steps):
         step(call_ev[i])
     torch.cuda.synchronize()
-    names = ["cache_append", "absorb_q", "decode_attn", "combine_splits", "out_proj"]
+    names = ["cache_append", "absorb_q", "decode_attn",
+             "combine_out_proj" if args.fused else "combine_splits + out_proj"]
     per_call = {n: float(np.mean([ev[j].elapsed_time(ev[j + 1]) for ev in call_ev])) * 1e3
                 for j, n in enumerate(names)}
+    # the two calls each on its own, and the fused call (same workspace)
+    two_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        two_ev[i][0].record(stream)
+        M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
+        two_ev[i][1].record(stream)
+        M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+        two_ev[i][2].record(stream)
+        M.mla_combine_out_proj(handle, ws, ws_bytes, B, P, w_uv, None, o, None, None, lse, sh)
+        two_ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    per_call["combine_splits"] = float(np.mean([e[0].elapsed_time(e[1]) for e in two_ev])) * 1e3
+    per_call["out_proj"] = float(np.mean([e[1].elapsed_time(e[2]) for e in two_ev])) * 1e3
+    per_call["combine_out_proj (fused, not in the step)" if not args.fused else "combine_out_proj (fused)"] = \
+        float(np.mean([e[2].elapsed_time(e[3]) for e in two_ev])) * 1e3
 
     # ---- the attention call alone, timed one call at a time (the latent
     # cache is larger than L2, so every call reads it from HBM): median and
@@ -685,8 +708,7 @@ def run_ours(args):
                            None, 0, sh)
         M.mla_absorb_q(handle, dev_in["q_nope"], dev_in["q_rope"], dev_in["pos"], w_uk, q_abs, B, sh)
         M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, dev_in["ctx"], B, P, ws, ws_bytes, sh)
-        M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
-        M.mla_out_proj(handle, ctx_lat, w_uv, None, o, None, B, sh)
+        finish(o, lse)
         o_host.copy_(o, non_blocking=True)
 
     for _ in range(3):
@@ -735,8 +757,7 @@ def run_ours(args):
             M.mla_cache_append(handle, d["h_new"], B, 1, d["pos"], w_dkv, w_kr, cache, cap, None, 0, sh)
             M.mla_absorb_q(handle, d["q_nope"], d["q_rope"], d["pos"], w_uk, q_abs, B, sh)
             M.mla_decode_attn(handle, q_abs, cache, cap, None, 0, d["ctx"], B, P, ws, ws_bytes, sh)
-            M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse, sh)
-            M.mla_out_proj(handle, ctx_lat, w_uv, None, outs[k], None, B, sh)
+            finish(outs[k], lse)
             done[k].record(stream)
             d2h_s.wait_event(done[k])
             with torch.cuda.stream(d2h_s):
@@ -837,7 +858,9 @@ def run_ours(args):
             "median_frac": attn_bytes / (float(np.median(attn_samples_us)) * 1e-6) / 1e9 / hbm_peak,
             "tokens_scanned_per_s": ctx_sum / (float(np.median(attn_samples_us)) * 1e-6),
             "note": "mla_decode_attn alone, one call per event pair, after the timed region"},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": (5 if args.fused else 6) * args.steps,
+        "step_calls": ("mla_cache_append, mla_absorb_q, mla_decode_attn (plan + attention), " +
+                       ("mla_combine_out_proj" if args.fused else "mla_combine_splits, mla_out_proj")),
         "per_call_us": per_call,
         "per_call_note": "separate pass after the timed region, events between all calls",
         "clocks": clk,

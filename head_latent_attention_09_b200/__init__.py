@@ -35,6 +35,7 @@ EXPORTED = (
     "mla_fp8_scale_groups", "mla_cache_append_fp8_workspace_size", "mla_cache_append_fp8",
     "mla_quantize_rows_fp8", "mla_decode_attn_fp8", "mla_selftest_wait_timeout",
     "mla_set_strict", "mla_decode_attn_range", "mla_combine_splits_f32", "mla_merge_ranges",
+    "mla_combine_out_proj",
 )
 
 
@@ -92,6 +93,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_decode_attn_range": (i, [vp, vp, vp, ll, vp, i, vp, vp, i, i, vp, sz, vp]),
         "mla_combine_splits_f32": (i, [vp, vp, sz, i, i, vp, vp, vp]),
         "mla_merge_ranges": (i, [vp, vp, vp, i, i, vp, vp, vp]),
+        "mla_combine_out_proj": (i, [vp, vp, sz, i, i, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -257,6 +259,13 @@ def mla_query_proj(handle, x, B, w_dq, d_cq, w_uq, w_qr, c_q, q_nope, q_rope, st
 def mla_out_proj(handle, ctx_lat, w_uv, w_o, o, u, B, stream=None):
     _check(load().mla_out_proj(handle, _ptr(ctx_lat), _ptr(w_uv), _ptr(w_o), _ptr(o), _ptr(u), B,
                                _stream(stream)), "mla_out_proj")
+
+
+def mla_combine_out_proj(handle, workspace, ws_bytes, B, num_parts, w_uv, w_o, o, u=None, ctx_lat=None, lse=None,
+                         stream=None):
+    _check(load().mla_combine_out_proj(handle, _ptr(workspace), ws_bytes, B, num_parts, _ptr(w_uv), _ptr(w_o),
+                                       _ptr(o), _ptr(u), _ptr(ctx_lat), _ptr(lse), _stream(stream)),
+           "mla_combine_out_proj")
 
 
 def mla_get_device_status(handle, stream=None) -> int:

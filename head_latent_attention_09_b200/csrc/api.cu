@@ -219,7 +219,7 @@ int mla_absorb_q(mla_handle *h, const void *q_nope, const void *q_rope, const in
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaErrorNotSupported;
   if (h->gemm_kind == kGemmTc)
-    e = launch_absorb_tc(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, s);
+    e = launch_absorb_tc(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, h->d_status, s);
   if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported)
     e = launch_absorb_simt(h->cfg, q_nope, q_rope, pos, w_uk, q_abs, B, h->d_theta, s);
@@ -409,13 +409,41 @@ int mla_out_proj(mla_handle *h, const void *ctx_lat, const void *w_uv, const voi
   if (!ctx_lat || !w_uv || !o || (w_o && !u)) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaErrorNotSupported;
-  if (h->gemm_kind == kGemmTc) e = launch_outproj_tc(h->cfg, ctx_lat, w_uv, o, B, s);
+  if (h->gemm_kind == kGemmTc) e = launch_outproj_tc(h->cfg, ctx_lat, w_uv, o, B, h->d_status, s);
   if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
   if (e == cudaErrorNotSupported) e = launch_outproj_simt(h->cfg, ctx_lat, w_uv, o, B, s);
   if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
   if (w_o) {
     e = cudaErrorNotSupported;
-    if (h->gemm_kind == kGemmTc) e = launch_wo_tc(h->cfg, o, w_o, u, B, s);
+    if (h->gemm_kind == kGemmTc) e = launch_wo_tc(h->cfg, o, w_o, u, B, h->d_status, s);
+    if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
+    if (e == cudaErrorNotSupported) e = launch_wo_simt(h->cfg, o, w_o, u, B, s);
+    if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+int mla_combine_out_proj(mla_handle *h, const void *workspace, size_t ws_bytes, int B, int num_parts,
+                         const void *w_uv, const void *w_o, void *o, void *u, void *ctx_lat, float *lse,
+                         mla_stream_t stream) {
+  Range range("mla_combine_out_proj");
+  if (!h || B < 0 || num_parts < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!w_uv || !o || (w_o && !u)) return MLA_ERR_INVALID_ARG;
+  const int P = num_parts == 0 ? default_parts(h) : num_parts;
+  const WsLayout L = ws_layout(h->cfg, B, P);
+  if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const char *ws = (const char *)workspace;
+  cudaError_t e = cudaErrorNotSupported;
+  if (h->gemm_kind == kGemmTc)
+    e = launch_combine_outproj_tc(h->cfg, ws, L, B, w_uv, o, ctx_lat, lse, h->d_status, s);
+  if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
+  if (e == cudaErrorNotSupported) e = launch_combine_outproj_simt(h->cfg, ws, L, B, w_uv, o, ctx_lat, lse, s);
+  if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
+  if (w_o) {
+    e = cudaErrorNotSupported;
+    if (h->gemm_kind == kGemmTc) e = launch_wo_tc(h->cfg, o, w_o, u, B, h->d_status, s);
     if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return MLA_ERR_UNSUPPORTED;
     if (e == cudaErrorNotSupported) e = launch_wo_simt(h->cfg, o, w_o, u, B, s);
     if (e != cudaSuccess) return e == cudaErrorNotSupported ? MLA_ERR_UNSUPPORTED : MLA_ERR_CUDA;
@@ -429,7 +457,7 @@ namespace {
 cudaError_t linear(const mla_handle *h, const void *x, const void *w, void *y, int M, int K, int N,
                    cudaStream_t s) {
   cudaError_t e = cudaErrorNotSupported;
-  if (h->gemm_kind == kGemmTc) e = launch_linear_tc(x, w, y, M, K, N, s);
+  if (h->gemm_kind == kGemmTc) e = launch_linear_tc(x, w, y, M, K, N, h->d_status, s);
   if (strict_refuses(h, h->gemm_kind == kGemmTc, e)) return e;   // reported as MLA_ERR_UNSUPPORTED
   if (e == cudaErrorNotSupported) e = launch_linear_simt(x, w, y, M, K, N, h->cfg.dtype == MLA_FP32, s);
   return e;

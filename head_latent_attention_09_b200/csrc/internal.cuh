@@ -150,13 +150,19 @@ struct WsLayout {
   size_t tile_prefix_off;  // int64 [B+1]
   size_t piece_base_off;   // int64 [B+1]
   size_t ctx_off;          // int32 [2][B]: each sequence's end and first token as attended (clamped by the plan)
-  size_t opart_off;        // float [max_pieces, n_h, d_c]
-  size_t lse_off;          // float [max_pieces, n_h]
+  size_t opart_off;        // float [n_h, max_pieces, d_c]: a head's pieces are consecutive rows
+  size_t lse_off;          // float [n_h, max_pieces]
   size_t total;
   long long max_pieces;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Row of (piece, head) in the partials (units of d_c floats) and index of its
+// log-sum-exp.
+__host__ __device__ inline long long part_row(const WsLayout &L, long long piece, int head) {
+  return (long long)head * L.max_pieces + piece;
+}
 
 inline WsLayout ws_layout(const mla_config &cfg, int B, int P) {
   WsLayout L;
@@ -245,6 +251,9 @@ cudaError_t launch_absorb_simt(const mla_config &cfg, const void *q_nope, const 
                                const double *theta, cudaStream_t s);
 cudaError_t launch_outproj_simt(const mla_config &cfg, const void *ctx_lat, const void *w_uv,
                                 void *o, int B, cudaStream_t s);
+// CUDA-core form of the fused combine and output projection (any dtype/shape).
+cudaError_t launch_combine_outproj_simt(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
+                                        const void *w_uv, void *o, void *ctx_lat, float *lse, cudaStream_t s);
 cudaError_t launch_wo_simt(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
                            cudaStream_t s);
 // y[N, M] = x[N, K] w[M, K]^T (row-major, the config's dtype).
@@ -261,12 +270,19 @@ cudaError_t launch_append_tc(const mla_config &cfg, const void *h, int B, int T,
                              cudaStream_t s, float *rows_out = nullptr);
 cudaError_t launch_absorb_tc(const mla_config &cfg, const void *q_nope, const void *q_rope,
                              const int *pos, const void *w_uk, void *q_abs, int B,
-                             const double *theta, cudaStream_t s);
+                             const double *theta, unsigned *status, cudaStream_t s);
 cudaError_t launch_outproj_tc(const mla_config &cfg, const void *ctx_lat, const void *w_uv,
-                              void *o, int B, cudaStream_t s);
+                              void *o, int B, unsigned *status, cudaStream_t s);
 cudaError_t launch_wo_tc(const mla_config &cfg, const void *o, const void *w_o, void *u, int B,
-                         cudaStream_t s);
-cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, cudaStream_t s);
+                         unsigned *status, cudaStream_t s);
+cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, unsigned *status,
+                             cudaStream_t s);
+// Split combine fused with the output projection: o[b, i] = W^UV_i ctx_lat[b, i]
+// with ctx_lat merged from the workspace's partials inside the kernel
+// (written out too when ctx_lat is set; lse likewise).
+cudaError_t launch_combine_outproj_tc(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
+                                      const void *w_uv, void *o, void *ctx_lat, float *lse, unsigned *status,
+                                      cudaStream_t s);
 cudaError_t launch_attn_tc_pair(const AttnArgs &a, int P, cudaStream_t s);
 cudaError_t launch_attn_tc_smallh(const AttnArgs &a, int P, cudaStream_t s);
 

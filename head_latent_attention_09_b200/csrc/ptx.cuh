@@ -395,5 +395,7 @@ bool encode_map_bf16(CUtensorMap *map, const void *base, int rank, const uint64_
 // The same for a byte tensor (FP8 codes).
 bool encode_map_u8(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                    const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz);
+bool encode_map_f32(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                    const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz);
 
 }  // namespace mla

@@ -223,14 +223,14 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
       m = m_new;
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    float *dst = opart + (piece * a.n_h + h) * (long long)a.d_c;
+    float *dst = opart + part_row(a.L, piece, h) * (long long)a.d_c;
 #pragma unroll
     for (int j = 0; j < kOPerLane; ++j) {
       const int f = lane + 32 * j;
       if (f < a.d_c) dst[f] = o[j] * inv;
     }
     if (lane == 0)
-      lse[piece * a.n_h + h] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+      lse[part_row(a.L, piece, h)] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
   }
 }
 
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const char *ws, WsLayout L
   const float *op = reinterpret_cast<const float *>(ws + L.opart_off);
   const long long p0 = pb[b], p1 = pb[b + 1];
   float m = -CUDART_INF_F;
-  for (long long p = p0; p < p1; ++p) m = fmaxf(m, lse[p * n_h + h]);
+  for (long long p = p0; p < p1; ++p) m = fmaxf(m, lse[part_row(L, p, h)]);
   T *dst = ctx_lat + ((long long)b * n_h + h) * d_c;
   if (m == -CUDART_INF_F) {
     for (int f = threadIdx.x; f < d_c; f += blockDim.x) dst[f] = from_f<T>(0.f);
@@ -256,12 +256,12 @@ __global__ void __launch_bounds__(128) combine_kernel(const char *ws, WsLayout L
     return;
   }
   float tot = 0.f;
-  for (long long p = p0; p < p1; ++p) tot += expf(lse[p * n_h + h] - m);
+  for (long long p = p0; p < p1; ++p) tot += expf(lse[part_row(L, p, h)] - m);
   const float inv = 1.f / tot;
   for (int f = threadIdx.x; f < d_c; f += blockDim.x) {
     float acc = 0.f;
     for (long long p = p0; p < p1; ++p)
-      acc += expf(lse[p * n_h + h] - m) * op[(p * n_h + h) * (long long)d_c + f];
+      acc += expf(lse[part_row(L, p, h)] - m) * op[part_row(L, p, h) * (long long)d_c + f];
     dst[f] = from_f<T>(acc * inv);
   }
   if (lse_out && threadIdx.x == 0) lse_out[(long long)b * n_h + h] = m + logf(tot);
@@ -422,6 +422,64 @@ __global__ void __launch_bounds__(256) outproj_simt_kernel(const T *ctx, const T
   }
 }
 
+// Split combine fused with the output projection, CUDA-core form: one block
+// per (sequence, head).  The merge is the vectorised combine's arithmetic per
+// element (weights exp(lse_p - max) / sum, accumulated in piece order), the
+// merged row is rounded to the dtype as ctx_lat would be, and the projection
+// is the output-projection kernel's, reading the row from shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_outproj_simt_kernel(const char *ws, WsLayout L, int n_h, int d_h,
+                                                                   int d_c, const T *w_uv, T *o, T *ctx_lat,
+                                                                   float *lse_out) {
+  extern __shared__ float sctx[];   // [d_c]
+  __shared__ float s_m, s_inv;
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const long long row = (long long)b * n_h + h;
+  const long long *pb = reinterpret_cast<const long long *>(ws + L.piece_base_off);
+  const float *lse = reinterpret_cast<const float *>(ws + L.lse_off);
+  const float *op = reinterpret_cast<const float *>(ws + L.opart_off);
+  const long long p0 = pb[b], p1 = pb[b + 1];
+  if (warp == 0) {
+    float m = -CUDART_INF_F;
+    for (long long p = p0 + lane; p < p1; p += 32) m = fmaxf(m, lse[part_row(L, p, h)]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float tot = 0.f;
+    if (m != -CUDART_INF_F)
+      for (long long p = p0 + lane; p < p1; p += 32) tot += expf(lse[part_row(L, p, h)] - m);
+    tot = warp_sum(tot);
+    if (lane == 0) {
+      s_m = m;
+      s_inv = m == -CUDART_INF_F ? 0.f : 1.f / tot;
+      if (lse_out) lse_out[row] = m == -CUDART_INF_F ? -CUDART_INF_F : m + logf(tot);
+    }
+  }
+  __syncthreads();
+  const float m = s_m, inv = s_inv;
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
+    float acc = 0.f;
+    if (m != -CUDART_INF_F)
+      for (long long p = p0; p < p1; ++p) {
+        const float w = expf(lse[part_row(L, p, h)] - m) * inv;
+        acc += w * op[part_row(L, p, h) * (long long)d_c + c];
+      }
+    const T v = from_f<T>(acc);
+    if (ctx_lat) ctx_lat[row * d_c + c] = v;
+    sctx[c] = to_f(v);
+  }
+  __syncthreads();
+  for (int r = warp; r < d_h; r += nw) {
+    const T *wr = w_uv + ((long long)h * d_h + r) * d_c;
+    float acc = 0.f;
+    for (int k = lane; k < d_c; k += 32) acc += to_f(wr[k]) * sctx[k];
+    acc = warp_sum(acc);
+    if (lane == 0) o[row * d_h + r] = from_f<T>(acc);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) linear_simt_kernel(const T *o, const T *w_o, T *u, int K, int d) {
   const int b = blockIdx.x;
@@ -491,7 +549,7 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(const char *ws, WsLayo
   const float *op = reinterpret_cast<const float *>(ws + L.opart_off);
   const long long p0 = pb[b], p1 = pb[b + 1];
   float m = -CUDART_INF_F;
-  for (long long p = p0 + lane; p < p1; p += 32) m = fmaxf(m, lse[p * n_h + h]);
+  for (long long p = p0 + lane; p < p1; p += 32) m = fmaxf(m, lse[part_row(L, p, h)]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   T *dst = ctx_lat + row * d_c;
@@ -502,7 +560,7 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(const char *ws, WsLayo
     return;
   }
   float tot = 0.f;
-  for (long long p = p0 + lane; p < p1; p += 32) tot += expf(lse[p * n_h + h] - m);
+  for (long long p = p0 + lane; p < p1; p += 32) tot += expf(lse[part_row(L, p, h)] - m);
   tot = warp_sum(tot);
   const float inv = 1.f / tot;
   float4 acc[4];
@@ -510,8 +568,8 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(const char *ws, WsLayo
   for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (long long p = p0; p < p1; ++p) {
-    const float w = expf(lse[p * n_h + h] - m) * inv;
-    const float4 *src = reinterpret_cast<const float4 *>(op + (p * n_h + h) * (long long)d_c);
+    const float w = expf(lse[part_row(L, p, h)] - m) * inv;
+    const float4 *src = reinterpret_cast<const float4 *>(op + part_row(L, p, h) * (long long)d_c);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int f = lane + 32 * i;
@@ -671,6 +729,19 @@ cudaError_t launch_outproj_simt(const mla_config &cfg, const void *ctx_lat, cons
         (const __nv_bfloat16 *)ctx_lat, (const __nv_bfloat16 *)w_uv, (__nv_bfloat16 *)o, cfg.n_h,
         cfg.d_h, cfg.d_c);
   return cudaGetLastError();
+}
+
+cudaError_t launch_combine_outproj_simt(const mla_config &cfg, const char *ws, const WsLayout &L, int B,
+                                        const void *w_uv, void *o, void *ctx_lat, float *lse, cudaStream_t s) {
+  if (B > 0x7fffffff || cfg.n_h > 65535) return cudaErrorNotSupported;
+  const dim3 grid(B, cfg.n_h);
+  const size_t smem = sizeof(float) * cfg.d_c;
+  if (cfg.dtype == MLA_FP32)
+    return launch_pdl(combine_outproj_simt_kernel<float>, grid, dim3(256), smem, s, 1, ws, L, cfg.n_h, cfg.d_h,
+                      cfg.d_c, (const float *)w_uv, (float *)o, (float *)ctx_lat, lse);
+  return launch_pdl(combine_outproj_simt_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, 1, ws, L, cfg.n_h,
+                    cfg.d_h, cfg.d_c, (const __nv_bfloat16 *)w_uv, (__nv_bfloat16 *)o, (__nv_bfloat16 *)ctx_lat,
+                    lse);
 }
 
 cudaError_t launch_linear_simt(const void *x, const void *w, void *y, int M, int K, int N, bool fp32,

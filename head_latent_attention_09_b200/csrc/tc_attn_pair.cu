@@ -620,7 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       const int head = 64 * (int)rank + h;
-      float *dst = opart + (pc.piece * a.n_h + head) * (long long)a.d_c + 128 * th;
+      float *dst = opart + part_row(a.L, pc.piece, head) * (long long)a.d_c + 128 * th;
 #pragma unroll 1
       for (int c = 0; c < 16; ++c) {
         uint32_t r[16];
@@ -634,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                           __uint_as_float(r[j + 2]) * inv, __uint_as_float(r[j + 3]) * inv);
       }
       if (th == 0)
-        lse_out[pc.piece * a.n_h + head] =
+        lse_out[part_row(a.L, pc.piece, head)] =
             lsum > 0.f ? (m_run + log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
       ptx::tc_fence_before();
       __syncwarp();

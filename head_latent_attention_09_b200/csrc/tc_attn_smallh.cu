@@ -647,7 +647,7 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
         const float l = red_s[hh] + red_s[H + hh] + red_s[2 * H + hh] + red_s[3 * H + hh];
         inv[hh] = l > 0.f ? 1.f / l : 0.f;
         if (q == 0 && lane == 0)
-          lse_out[pc.piece * a.n_h + hh] = l > 0.f ? (m_run[hh] + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+          lse_out[part_row(a.L, pc.piece, hh)] = l > 0.f ? (m_run[hh] + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
       }
       if (!warp_wait(bar + C::bODone + ((i - 1) & 1), ((i - 1) >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int hh = 16 * c + j;
-            opart[(pc.piece * a.n_h + hh) * (long long)a.d_c + 128 * f + row] = __uint_as_float(r[j]) * inv[hh];
+            opart[part_row(a.L, pc.piece, hh) * (long long)a.d_c + 128 * f + row] = __uint_as_float(r[j]) * inv[hh];
           }
         }
       }

@@ -74,6 +74,11 @@ bool encode_map_u8(CUtensorMap *map, const void *base, int rank, const uint64_t 
   return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides, box, swz);
 }
 
+bool encode_map_f32(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                    const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, rank, dims, strides, box, swz);
+}
+
 namespace {
 
 constexpr int kGemmThreads = 192;
@@ -606,7 +611,8 @@ GemmParams blank_params() {
 
 // ---------------------------------------------------------------------------
 cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void *q_rope, const int *pos,
-                             const void *w_uk, void *q_abs, int B, const double *theta, cudaStream_t s) {
+                             const void *w_uk, void *q_abs, int B, const double *theta, unsigned *status,
+                             cudaStream_t s) {
   if (!aligned16(q_nope) || !aligned16(w_uk) || c.d_h % 64 != 0) return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiAbsorb;
@@ -626,6 +632,7 @@ cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void
   g.d_c = c.d_c;
   g.d_r = c.d_r;
   g.n_h = c.n_h;
+  g.status = status;
   return dispatch<true>(B, g, c.d_c / 128, c.n_h, s, [&](int G, int bn, Maps &m) {
     // W^UK [n_h d_h, d_c]: row k of head z is k-row z d_h + k, the d_c columns are m.
     if (!map_a_mnmajor(&m.a0, w_uk, c.d_c, (uint64_t)c.n_h * c.d_h, G)) return false;
@@ -635,7 +642,7 @@ cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void
 }
 
 cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const void *w_uv, void *o, int B,
-                              cudaStream_t s) {
+                              unsigned *status, cudaStream_t s) {
   if (!aligned16(ctx_lat) || !aligned16(w_uv) || c.d_h % 128 != 0) return cudaErrorNotSupported;
   GemmParams g = blank_params();
   g.mode = kEpiOutProj;
@@ -647,6 +654,7 @@ cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const vo
   g.out = (__nv_bfloat16 *)o;
   g.out_ld = (long long)c.n_h * c.d_h;
   g.out_z = c.d_h;
+  g.status = status;
   return dispatch<false>(B, g, c.d_h / 128, c.n_h, s, [&](int G, int bn, Maps &m) {
     if (!map_a_kmajor(&m.a0, w_uv, c.d_c, (uint64_t)c.n_h * c.d_h, G)) return false;
     m.a1 = m.a0;
@@ -654,7 +662,8 @@ cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const vo
   });
 }
 
-cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, cudaStream_t s) {
+cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K, int N, unsigned *status,
+                             cudaStream_t s) {
   // y[N, M] = x[N, K] w[M, K]^T, bf16 in and out, fp32 accumulation.
   if (!aligned16(x) || !aligned16(w) || K % 64 != 0 || M <= 0 || N <= 0) return cudaErrorNotSupported;
   GemmParams g = blank_params();
@@ -664,6 +673,7 @@ cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K
   g.N = N;
   g.out = (__nv_bfloat16 *)y;
   g.out_ld = M;
+  g.status = status;
   return dispatch<false>(N, g, (M + 127) / 128, 1, s, [&](int G, int bn, Maps &m) {
     if (!map_a_kmajor(&m.a0, w, K, M, G)) return false;
     m.a1 = m.a0;
@@ -671,8 +681,9 @@ cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K
   });
 }
 
-cudaError_t launch_wo_tc(const mla_config &c, const void *o, const void *w_o, void *u, int B, cudaStream_t s) {
-  return launch_linear_tc(o, w_o, u, c.d_model, c.n_h * c.d_h, B, s);
+cudaError_t launch_wo_tc(const mla_config &c, const void *o, const void *w_o, void *u, int B, unsigned *status,
+                         cudaStream_t s) {
+  return launch_linear_tc(o, w_o, u, c.d_model, c.n_h * c.d_h, B, status, s);
 }
 
 cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, const int *start_pos,

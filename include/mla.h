@@ -264,6 +264,26 @@ int mla_merge_ranges(mla_handle *handle, const float *ctx_parts, const float *ls
 int mla_out_proj(mla_handle *handle, const void *ctx_lat, const void *w_uv, const void *w_o,
                  void *o, void *u, int B, mla_stream_t stream);
 
+/* mla_combine_splits followed by mla_out_proj as one step: the partials of
+ * the preceding mla_decode_attn on the same workspace are merged inside the
+ * output projection (the log-sum-exp algebra of mla_combine_splits, then
+ * o[b,i,:] = W^UV_i ctx_lat[b,i,:], V2 App. C), so the merged latents do not
+ * make a round trip through device memory.
+ *   w_uv [n_h*d_h, d_c]; o [B, n_h, d_h]; w_o / u as mla_out_proj.
+ *   ctx_lat [B, n_h, d_c] (cfg.dtype) or NULL: when given it receives the
+ *   merged latents, the same values mla_combine_splits writes; lse [B, n_h]
+ *   float32 or NULL likewise.
+ * B and num_parts must equal those given to mla_decode_attn.  The merged
+ * latents enter the projection rounded to cfg.dtype, as with the two calls.
+ * bf16 with d_h a multiple of 128 and d_c a multiple of 128 up to 512 runs one
+ * tcgen05 kernel; other shapes run a CUDA-core kernel (refused under strict
+ * mode where the tensor-core kernel exists but cannot take the arguments).
+ * Errors: INVALID_ARG (NULL handle, w_uv or o; w_o without u; negative B or
+ * num_parts), WORKSPACE, UNSUPPORTED, CUDA. */
+int mla_combine_out_proj(mla_handle *handle, const void *workspace, size_t ws_bytes, int B, int num_parts,
+                         const void *w_uv, const void *w_o, void *o, void *u, void *ctx_lat, float *lse,
+                         mla_stream_t stream);
+
 /* Self-test of the device-side time-out path: launches one wait on a barrier
  * that nothing completes, which gives up after limit_ns nanoseconds (1e3 ..
  * 1e9) and sets the time-out bit in the handle's status word, exactly as a

@@ -134,8 +134,12 @@ class DeviceCache:
         return to_host(self.data[b, torch.from_numpy(pos).to(self.data.device)])
 
 
-def run_decode_step(wl, num_parts=0, with_wo=False, dev="cuda", keep=False, fill_rows=None):
-    """One decode step for every sequence of the workload.  Returns host arrays."""
+def run_decode_step(wl, num_parts=0, with_wo=False, dev="cuda", keep=False, fill_rows=None, fused=False):
+    """One decode step for every sequence of the workload.  Returns host arrays.
+
+    With fused=True the same workspace is then also finished by
+    mla_combine_out_proj, twice: with ctx_lat and lse written ("fused_*") and
+    with both left out ("fused_o_bare")."""
     handle = create_handle(wl)
     try:
         wnp = draw_weights(wl, with_wo=with_wo)
@@ -179,6 +183,18 @@ def run_decode_step(wl, num_parts=0, with_wo=False, dev="cuda", keep=False, fill
                           ctx_d, B, P, ws, ws_bytes)
         M.mla_combine_splits(handle, ws, ws_bytes, B, P, ctx_lat, lse)
         M.mla_out_proj(handle, ctx_lat, w["w_uv"], w.get("w_o"), o, u, B)
+        fused_out = {}
+        if fused:
+            ctx_f = torch.full_like(ctx_lat, float("nan"))
+            lse_f = torch.full_like(lse, float("nan"))
+            o_f = torch.full_like(o, float("nan"))
+            u_f = torch.full_like(u, float("nan")) if with_wo else None
+            M.mla_combine_out_proj(handle, ws, ws_bytes, B, P, w["w_uv"], w.get("w_o"), o_f, u_f, ctx_f, lse_f)
+            o_bare = torch.full_like(o, float("nan"))
+            u_bare = torch.full_like(u, float("nan")) if with_wo else None
+            M.mla_combine_out_proj(handle, ws, ws_bytes, B, P, w["w_uv"], w.get("w_o"), o_bare, u_bare)
+            fused_out = {"fused_ctx_lat": to_host(ctx_f), "fused_lse": to_host(lse_f), "fused_o": to_host(o_f),
+                         "fused_u": to_host(u_f) if with_wo else None, "fused_o_bare": to_host(o_bare)}
         st = M.mla_get_device_status(handle)
         if st != M.MLA_OK:
             raise M.MlaError(st, "device status")
@@ -188,6 +204,7 @@ def run_decode_step(wl, num_parts=0, with_wo=False, dev="cuda", keep=False, fill
             "cache_new_rows": np.stack([cache.rows_of(b, [max(int(ctx[b]) - 1, 0)])[0]
                                         for b in range(B)]),
             "ctx": ctx,
+            **fused_out,
         }
         if keep:
             out["_cache"] = cache
