@@ -56,7 +56,13 @@ constexpr int kGroups8 = 5;                // scale groups of a 576-wide row
 template <int H, bool F8>
 struct Cfg {
   static constexpr int kConvWarps = F8 ? 4 : 0;                 // FP8 converter warps
-  static constexpr int kThreads = 192 + 32 * kConvWarps;
+  // bf16: a second TMA producer, warp 6 (the rotary chunk and latent pairs
+  // 2-3 of every tile; warp 0 the query and pairs 0-1).  A thread issuing
+  // cp.async.bulk.tensor copies sustains about two per microsecond, and a
+  // paged tile takes 18 of them (two 64-token pages x nine chunks).
+  static constexpr int kProducers = F8 ? 1 : 2;
+  static constexpr int kProd1Warp = 6;
+  static constexpr int kThreads = 192 + 32 * kConvWarps + 32 * (kProducers - 1);
   static constexpr int kNL = (!F8 && H <= 16) ? 5 : 4;          // latent pair slots (a tile takes 4)
   static constexpr int kNR = (F8 && H > 16) ? 1 : 2;            // rotary chunk slots
   static constexpr int kNSt = F8 ? (H <= 16 ? 4 : 3) : 0;       // FP8 staging chunks
@@ -290,11 +296,16 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
   // the query and the cache it wrote are read.
   pdl_wait();
 
-  if (warp == 0) {
-    // -------------------------------------------------------------- producer
+  if (warp == 0 || (C::kProducers > 1 && warp == C::kProd1Warp)) {
+    // ------------------------------------------------------------- producers
     // Per tile, in the order the MMAs consume them: the rotary chunk, then
     // the four latent pairs (bf16), or the nine chunks of codes into the
-    // staging ring (FP8: rotary chunk first, then latent chunks 0-7).
+    // staging ring (FP8: rotary chunk first, then latent chunks 0-7).  With
+    // two producers each walks every tile and ring position but fills only
+    // its own slots: producer 0 the query and pairs 0-1, producer 1 the
+    // rotary chunk and pairs 2-3.
+    const int pid = warp == 0 ? 0 : 1;
+    const bool own_rope = pid == C::kProducers - 1;
     Walk w;
     walk_init(w, a, share);
     Piece pc;
@@ -313,11 +324,13 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
       return warp_wait(empty, r.phase ^ 1u, a.status, abort_flag);
     };
     while (ok && walk_next(w, a, share, pc)) {
-      if (npc > 0 && !warp_wait(bar + C::bQEmpty, (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
-      if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(bar + C::bQFull, C::kQ);
-        for (int c = 0; c < 9; ++c)
-          ptx::tma_load_2d(sQ + c * H * 128, &mapQ, bar + C::bQFull, 64 * c, pc.b * H);
+      if (pid == 0) {
+        if (npc > 0 && !warp_wait(bar + C::bQEmpty, (npc - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(bar + C::bQFull, C::kQ);
+          for (int c = 0; c < 9; ++c)
+            ptx::tma_load_2d(sQ + c * H * 128, &mapQ, bar + C::bQFull, 64 * c, pc.b * H);
+        }
       }
       for (int k = 0; k < pc.ntiles && ok; ++k) {
         const int tok0 = pc.tok_begin + kTileTok * k;
@@ -373,7 +386,9 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
           continue;
         }
         // bf16: the rotary chunk
-        {
+        if (!own_rope) {
+          rope.advance(NR);
+        } else {
           uint64_t *full = bar + C::bRopeFull + rope.slot;
           if (!slot_free(bar + C::bRopeEmpty + rope.slot, rope)) { ok = false; break; }
           uint8_t *dst = sRope + rope.slot * kChunk;
@@ -392,6 +407,10 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
         }
         // the four latent pairs
         for (int pb = 0; pb < 4 && ok; ++pb) {
+          if (C::kProducers > 1 && (pb >> 1) != pid) {
+            lat.advance(NL);
+            continue;
+          }
           uint64_t *full = bar + C::bLatFull + lat.slot;
           if (!slot_free(bar + C::bLatEmpty + lat.slot, lat)) { ok = false; break; }
           uint8_t *dst = sLat + lat.slot * kPair;
