@@ -42,29 +42,42 @@ __device__ __forceinline__ long long cache_row(int b, long long p, long long cac
 }
 
 // ---------------------------------------------------------------------------
-// plan: one block of 1024 threads
+// plan: one block of up to 1024 threads (a multiple of 32)
 // ---------------------------------------------------------------------------
+// Exclusive prefix sum over the block (thread order), and the total: a
+// shuffle scan within each warp, then one warp scans the warp totals.
+// `smem` holds 32 values.
 __device__ long long block_exclusive_scan(long long v, long long *smem, long long *total) {
-  const int tid = threadIdx.x, n = blockDim.x;
-  smem[tid] = v;
-  __syncthreads();
-  for (int off = 1; off < n; off <<= 1) {
-    long long add = tid >= off ? smem[tid - off] : 0;
-    __syncthreads();
-    smem[tid] += add;
-    __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  long long incl = smem[tid];
-  *total = smem[n - 1];
+  if (lane == 31) smem[warp] = x;
   __syncthreads();
-  return incl - v;
+  if (warp == 0) {
+    long long t = lane < nw ? smem[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < nw) smem[lane] = t;   // inclusive prefix of the warp totals
+  }
+  __syncthreads();
+  const long long before = warp > 0 ? smem[warp - 1] : 0;
+  *total = smem[nw - 1];
+  __syncthreads();   // smem is reused by the next scan
+  return before + x - v;
 }
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const int *ctx_len, int B, int P_req,
                                                     long long cap, char *ws, WsLayout L, unsigned *status) {
   pdl_trigger();
   pdl_wait();   // the workspace may still be read by the previous step's combine
-  __shared__ long long scan[1024];
+  __shared__ long long scan[32];
   long long *tile_prefix = reinterpret_cast<long long *>(ws + L.tile_prefix_off);
   long long *piece_base = reinterpret_cast<long long *>(ws + L.piece_base_off);
   int *ctx_eff = reinterpret_cast<int *>(ws + L.ctx_off);   // [B] ends, then [B] first tokens
@@ -501,7 +514,9 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const T *o, const T *w
 // ---------------------------------------------------------------------------
 cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, char *ws,
                         const WsLayout &L, unsigned *status, cudaStream_t s) {
-  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_begin, ctx_len, B, P, cap, ws, L, status);
+  // one thread per sequence up to 1024 (each thread takes a run of sequences beyond)
+  const int threads = B >= 1024 ? 1024 : (B <= 32 ? 32 : (B + 31) / 32 * 32);
+  return launch_pdl(plan_kernel, dim3(1), dim3(threads), 0, s, 1, ctx_begin, ctx_len, B, P, cap, ws, L, status);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s) {

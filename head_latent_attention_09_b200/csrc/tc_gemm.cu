@@ -121,6 +121,7 @@ struct GemmParams {
   // append: when set, token n's row goes to out_f32[n * (d_c + d_r) ..] in
   // float32 (for a later FP8 quantisation) instead of to the cache
   float *out_f32;
+  int vec_out;        // bf16 outputs aligned for 16-byte stores (rows of 128 contiguous features)
   unsigned *status;
 };
 
@@ -339,7 +340,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-    const bool ok = ptx::mbar_wait(accf, 0, g.status, abort_flag);
+    // One thread polls the accumulator barrier and the other epilogue threads
+    // wait on a named barrier, which takes no issue slots: with every
+    // epilogue warp polling, the polls of the CTAs sharing an SM slowed each
+    // other's epilogues several-fold (measured).
+    if (et == 0) ptx::mbar_wait(accf, 0, g.status, abort_flag);
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+    const bool ok = !*abort_flag;   // the same for every epilogue thread
     ptx::tc_fence_after();
     const int q = warp & 3;
     const int m_local = q * 32 + lane;
@@ -359,40 +366,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) red[(c0 + j) * 128 + m_local] = have ? __uint_as_float(r[j]) : 0.f;
       }
-    } else if (ok) {
+    } else {
+      const bool go = ok;
+      // With vec_out, bf16 outputs go through shared memory (the ring, free
+      // once the accumulator is complete): each warp writes its 32 rows of a
+      // block of up to 64 columns as [column][128 rows], then the four warps
+      // store 16-byte pieces of each column's 128 contiguous output rows.
+      const bool vec = go && g.vec_out && g.out_f32 == nullptr;
+      __nv_bfloat16 *stg = reinterpret_cast<__nv_bfloat16 *>(base);
 #pragma unroll 1
-      for (int t = 0; t < mcount; ++t) {
+      for (int t = 0; t < mcount && go; ++t) {
         // m tile mt + t: rows m0 + 128 t .., accumulator columns t * BN ..
         const int mm = m + 128 * t;
         const bool mm_ok = mm < g.M_valid;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(t * BN + c0), r);
-          ptx::tmem_ld_wait();
+        for (int cb = 0; cb < BN; cb += 64) {
+          const int ncb = BN < 64 ? BN : 64;
+#pragma unroll 1
+          for (int c0 = cb; c0 < cb + ncb; c0 += 16) {
+            uint32_t r[16];
+            ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(t * BN + c0), r);
+            ptx::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + c0 + j;
-            float v = __uint_as_float(r[j]);
-            if (rope_tile) {
-              const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
-              const int k = m_local >> 1;
-              if (mm_ok && n < g.N && k < g.d_r / 2) {
-                float s, c;
-                rope_sincos(s_pos[c0 + j], g.theta[k], &s, &c);
-                v = (lane & 1) ? partner * s + v * c : v * c - partner * s;
+            for (int j = 0; j < 16; ++j) {
+              const int n = n0 + c0 + j;
+              float v = __uint_as_float(r[j]);
+              if (rope_tile) {
+                const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
+                const int k = m_local >> 1;
+                if (mm_ok && n < g.N && k < g.d_r / 2) {
+                  float s, c;
+                  rope_sincos(s_pos[c0 + j], g.theta[k], &s, &c);
+                  v = (lane & 1) ? partner * s + v * c : v * c - partner * s;
+                }
+              }
+              if (vec) {
+                stg[(c0 - cb + j) * 128 + m_local] = __float2bfloat16_rn(v);
+                continue;
+              }
+              if (!mm_ok || n >= g.N) continue;
+              if (g.mode == kEpiAppend) {
+                const long long row = s_row[c0 + j];
+                if (row >= 0) {
+                  if (g.out_f32) g.out_f32[row * (long long)(g.d_c + g.d_r) + mm] = v;
+                  else g.out[row * (long long)(g.d_c + g.d_r) + mm] = __float2bfloat16_rn(v);
+                }
+              } else {
+                g.out[(long long)n * g.out_ld + (long long)z * g.out_z + mm] = __float2bfloat16_rn(v);
               }
             }
-            if (!mm_ok || n >= g.N) continue;
-            if (g.mode == kEpiAppend) {
-              const long long row = s_row[c0 + j];
-              if (row >= 0) {
-                if (g.out_f32) g.out_f32[row * (long long)(g.d_c + g.d_r) + mm] = v;
-                else g.out[row * (long long)(g.d_c + g.d_r) + mm] = __float2bfloat16_rn(v);
+          }
+          if (vec) {
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const int mt0 = m0 + 128 * t;
+            for (int idx = et; idx < ncb * 16; idx += 128) {
+              const int cl = idx >> 4, u = idx & 15, n = n0 + cb + cl, mrow = mt0 + 8 * u;
+              if (n >= g.N || mrow >= g.M_valid) continue;
+              __nv_bfloat16 *dst;
+              if (g.mode == kEpiAppend) {
+                const long long row = s_row[cb + cl];
+                if (row < 0) continue;
+                dst = g.out + row * (long long)(g.d_c + g.d_r) + mrow;
+              } else {
+                dst = g.out + (long long)n * g.out_ld + (long long)z * g.out_z + mrow;
               }
-            } else {
-              g.out[(long long)n * g.out_ld + (long long)z * g.out_z + mm] = __float2bfloat16_rn(v);
+              *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(stg + cl * 128 + 8 * u);
             }
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // the staging block is reused
           }
         }
       }
@@ -421,13 +461,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int idx = threadIdx.x; idx < BN * R4; idx += kGemmThreads) {
         const int c = idx / R4, ml = zs * R + 4 * (idx % R4);
         const uint32_t off = (uint32_t)((c * 128 + ml) * 4);
+        // every peer's float4 in flight at once, summed in cluster-rank order
+        float4 pv[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          if (p < ks) pv[p] = ptx::ld_shared_cluster_v4f(ptx::mapa_peer(red + off, (uint32_t)p));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p = 0; p < ks; ++p) {
-          const float4 v = ptx::ld_shared_cluster_v4f(ptx::mapa_peer(red + off, (uint32_t)p));
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          if (p < ks) {
+            acc.x += pv[p].x;
+            acc.y += pv[p].y;
+            acc.z += pv[p].z;
+            acc.w += pv[p].w;
+          }
         }
         const int n = n0 + c;
         if (n >= g.N) continue;
@@ -446,19 +493,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
+        __nv_bfloat16 *dst = nullptr;
+        float *dst32 = nullptr;
+        if (g.mode == kEpiAppend) {
+          const long long row = s_row[c];
+          if (row < 0) continue;
+          if (g.out_f32) dst32 = g.out_f32 + row * (long long)(g.d_c + g.d_r) + m0 + ml;
+          else dst = g.out + row * (long long)(g.d_c + g.d_r) + m0 + ml;
+        } else {
+          dst = g.out + (long long)n * g.out_ld + (long long)z * g.out_z + m0 + ml;
+        }
+        if (dst && g.vec_out && m0 + ml + 4 <= g.M_valid) {
+          // four consecutive rows: one 8-byte store
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+          *reinterpret_cast<uint2 *>(dst) = pk;
+          continue;
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int m = m0 + ml + e;
-          if (m >= g.M_valid) continue;
-          if (g.mode == kEpiAppend) {
-            const long long row = s_row[c];
-            if (row >= 0) {
-              if (g.out_f32) g.out_f32[row * (long long)(g.d_c + g.d_r) + m] = v[e];
-              else g.out[row * (long long)(g.d_c + g.d_r) + m] = __float2bfloat16_rn(v[e]);
-            }
-          } else {
-            g.out[(long long)n * g.out_ld + (long long)z * g.out_z + m] = __float2bfloat16_rn(v[e]);
-          }
+          if (m0 + ml + e >= g.M_valid) continue;
+          if (dst32) dst32[e] = v[e];
+          else dst[e] = __float2bfloat16_rn(v[e]);
         }
       }
     } else if (threadIdx.x == 0) {
@@ -633,6 +691,7 @@ cudaError_t launch_absorb_tc(const mla_config &c, const void *q_nope, const void
   g.d_r = c.d_r;
   g.n_h = c.n_h;
   g.status = status;
+  g.vec_out = aligned16(q_abs) && c.d_c % 8 == 0 && c.d_r % 8 == 0;
   return dispatch<true>(B, g, c.d_c / 128, c.n_h, s, [&](int G, int bn, Maps &m) {
     // W^UK [n_h d_h, d_c]: row k of head z is k-row z d_h + k, the d_c columns are m.
     if (!map_a_mnmajor(&m.a0, w_uk, c.d_c, (uint64_t)c.n_h * c.d_h, G)) return false;
@@ -655,6 +714,7 @@ cudaError_t launch_outproj_tc(const mla_config &c, const void *ctx_lat, const vo
   g.out_ld = (long long)c.n_h * c.d_h;
   g.out_z = c.d_h;
   g.status = status;
+  g.vec_out = aligned16(o);
   return dispatch<false>(B, g, c.d_h / 128, c.n_h, s, [&](int G, int bn, Maps &m) {
     if (!map_a_kmajor(&m.a0, w_uv, c.d_c, (uint64_t)c.n_h * c.d_h, G)) return false;
     m.a1 = m.a0;
@@ -674,6 +734,7 @@ cudaError_t launch_linear_tc(const void *x, const void *w, void *y, int M, int K
   g.out = (__nv_bfloat16 *)y;
   g.out_ld = M;
   g.status = status;
+  g.vec_out = aligned16(y) && M % 8 == 0;
   return dispatch<false>(N, g, (M + 127) / 128, 1, s, [&](int G, int bn, Maps &m) {
     if (!map_a_kmajor(&m.a0, w, K, M, G)) return false;
     m.a1 = m.a0;
@@ -712,6 +773,7 @@ cudaError_t launch_append_tc(const mla_config &c, const void *h, int B, int T, c
   g.page_size = c.page_size;
   g.out_f32 = rows_out;
   g.status = status;
+  g.vec_out = aligned16(cache) && (c.d_c + c.d_r) % 8 == 0;
   const int mtiles = c.d_c / 128 + (c.d_r + 127) / 128;
   return dispatch<false>((int)N, g, mtiles, 1, s, [&](int G, int bn, Maps &m) {
     // W^DKV rows form the c^KV tiles, W^KR (d_r rows) the last tile
