@@ -254,6 +254,39 @@ def cpu_oracle_sample(wl, n_heads, budget_s=20.0):
     return gbs, desc, threads, el / reps
 
 
+def cpu_oracle_workload(wl, budget_s=15.0):
+    """The oracle's explicit-form decode step, every head, over the workload's
+    sequences in order (each sequence's rows the same seeded draw, cut to its
+    length) until all are done or budget_s has passed.  Returns a dict: GB/s
+    of latent cache scanned, how much of the workload ran, and the step time
+    that rate implies for the whole workload."""
+    from oracle import mla_oracle as O
+    from workloads import ctx_lengths, draw_weights, queries, random_cache
+    ctx = ctx_lengths(wl)
+    w = draw_weights(wl)
+    qn, qr = queries(wl)
+    rows = random_cache(wl.with_(B=1, ctx=(int(ctx.max()),)) if wl.ctx else wl.with_(B=1),
+                        int(ctx.max()))[0].astype(np.float64)
+    done_tok, done_seq, t0 = 0, 0, time.perf_counter()
+    for b in range(wl.B):
+        n = int(ctx[b])
+        if n > 0:
+            O.mla_decode_explicit(qn[b], qr[b], n - 1, rows[:n], w["w_uk"], w["w_uv"], n_h=wl.n_h, d_h=wl.d_h,
+                                  d_c=wl.d_c, d_r=wl.d_r, base=wl.rope_base)
+            done_tok += n
+        done_seq += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    total = int(ctx.sum())
+    return {"workload": wl.name, "sequences": f"{done_seq}/{wl.B}", "full": done_seq == wl.B,
+            "tokens": done_tok, "seconds": el,
+            "value": done_tok * wl.D * (2 if wl.dtype == "bf16" else 4) / el / 1e9 if el > 0 else None,
+            "unit": "GB/s", "us_per_step": el / max(done_tok, 1) * total * 1e6,
+            "kind": "oracle (explicit fp64, every head)",
+            "note": "whole workload" if done_seq == wl.B else "sequences in order until the time budget; us_per_step extrapolated by tokens"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -825,6 +858,9 @@ def run_ours(args):
     if not args.no_cpu_baseline:
         gbs, desc, threads, _ = cpu_oracle_sample(wl, 16, budget_s=15.0)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc}
+        if not args.batch:
+            cpu["configs"] = {name: cpu_oracle_workload(WORKLOADS[name], budget_s=15.0)
+                              for name in ("tiny_fp32", "v2lite_b32_ctx4k", "v2lite_paged_ragged_b128")}
     line = {
         "metric": "MLA decode: HBM GB/s (% of peak) and us/step at B=64, n_h=128, ctx 8K",
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
