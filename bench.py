@@ -512,7 +512,7 @@ def measure_workload(M, wl, dev, steps, seed, hbm_peak, n_samples=100):
             "step_gbs": (cache_bytes + w_bytes) / (step_us * 1e-6) / 1e9,
             "attn_median_us": med, "attn_p10_us": float(np.percentile(t, 10)),
             "attn_p90_us": float(np.percentile(t, 90)), "attn_gbs": gbs, "attn_frac": gbs / hbm_peak,
-            "tokens_scanned_per_s": tokens / (med * 1e-6), "attn_us_at_70pct_of_8TBps": cache_bytes / 5.6e3,
+            "tokens_scanned_per_s": tokens / (med * 1e-6), "attn_us_at_70pct_of_8TBps": cache_bytes / 5.6e6,
             "bound": "hbm"}
 
 
