@@ -35,7 +35,7 @@ EXPORTED = (
     "mla_fp8_scale_groups", "mla_cache_append_fp8_workspace_size", "mla_cache_append_fp8",
     "mla_quantize_rows_fp8", "mla_decode_attn_fp8", "mla_selftest_wait_timeout",
     "mla_set_strict", "mla_decode_attn_range", "mla_combine_splits_f32", "mla_merge_ranges",
-    "mla_combine_out_proj",
+    "mla_combine_out_proj", "mla_plan_pieces_tiled", "mla_plan_tile",
 )
 
 
@@ -94,6 +94,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "mla_combine_splits_f32": (i, [vp, vp, sz, i, i, vp, vp, vp]),
         "mla_merge_ranges": (i, [vp, vp, vp, i, i, vp, vp, vp]),
         "mla_combine_out_proj": (i, [vp, vp, sz, i, i, vp, vp, vp, vp, vp, vp, vp]),
+        "mla_plan_pieces_tiled": (ll, [vp, i, i, i, vp]),
+        "mla_plan_tile": (i, [vp, i]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -285,6 +287,20 @@ def mla_decode_attn_combine_noalloc(handle, q_abs, cache, cache_len, block_table
 
 def mla_noalloc_scratch_bytes() -> int:
     return load().mla_noalloc_scratch_bytes()
+
+
+def mla_plan_pieces_tiled(ctx_len, num_parts, tile_tokens):
+    """Host mirror of the split plan with tiles of tile_tokens tokens."""
+    B = len(ctx_len)
+    arr = (ctypes.c_int * max(B, 1))(*[int(c) for c in ctx_len])
+    base = (ctypes.c_longlong * (B + 1))()
+    n = load().mla_plan_pieces_tiled(ctypes.cast(arr, ctypes.c_void_p), B, num_parts, tile_tokens,
+                                     ctypes.cast(base, ctypes.c_void_p))
+    return n, list(base)
+
+
+def mla_plan_tile(handle, fp8=False):
+    return load().mla_plan_tile(handle, 1 if fp8 else 0)
 
 
 def mla_plan_pieces(ctx_len, num_parts):

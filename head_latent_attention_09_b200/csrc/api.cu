@@ -57,6 +57,14 @@ int default_parts(const mla_handle *h) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Tokens per tile of the split plan: the MMA tile of the attention kernel the
+// handle runs (a share then never pays for a partial tile inside a sequence).
+int plan_tile_of(const mla_handle *h, bool fp8) {
+  if (h->attn_kind == kAttnTcPair && !fp8) return 256;
+  if (h->attn_kind == kAttnTcSmallH) return 128;
+  return kTile;
+}
+
 // Appends to theta[0 .. nth) (double) the float pairs (hi, lo) with
 // hi + lo = theta[k] to about 2^-48 (the second half of the table).
 void split_theta(double *theta, int nth) {
@@ -256,7 +264,8 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
   // pages of its block-table row.
   const long long cap = c.page_size > 0 ? (long long)max_blocks_per_seq * c.page_size : cache_len;
   const long long cap_i = cap < 0x7fffffffLL ? cap : 0x7fffffffLL;
-  cudaError_t e = launch_plan(ctx_begin, ctx_len, B, P, cap_i, (char *)workspace, L, h->d_status, s);
+  const int tile = plan_tile_of(h, kv_scale != nullptr);
+  cudaError_t e = launch_plan(ctx_begin, ctx_len, B, P, cap_i, tile, (char *)workspace, L, h->d_status, s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   AttnArgs a;
   a.q_abs = q_abs;
@@ -274,6 +283,7 @@ int decode_attn(mla_handle *h, const void *q_abs, const void *cache, const float
   a.n_groups = fp8_num_groups(c.d_c, c.d_r);
   a.ws = (char *)workspace;
   a.L = L;
+  a.plan_tile = tile;
   a.status = h->d_status;
   e = cudaErrorNotSupported;
   if (h->attn_kind == kAttnTcPair && !kv_scale && aligned16(q_abs) && aligned16(cache))
@@ -505,23 +515,31 @@ int mla_get_device_status(mla_handle *h, mla_stream_t stream) {
   return MLA_OK;
 }
 
-long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *piece_base) {
-  if (!ctx_len || !piece_base || B < 0 || num_parts <= 0) return -1;
+long long mla_plan_pieces_tiled(const int *ctx_len, int B, int num_parts, int tile_tokens, long long *piece_base) {
+  if (!ctx_len || !piece_base || B < 0 || num_parts <= 0 || tile_tokens < kTile || tile_tokens % kTile != 0)
+    return -1;
+  const int tile = tile_tokens;
   long long Ttot = 0;
   for (int b = 0; b < B; ++b) {
     if (ctx_len[b] < 0) return -1;
-    Ttot += ceil_div_ll(ctx_len[b], kTile);
+    Ttot += ceil_div_ll(ctx_len[b], tile);
   }
   const long long P = Ttot < num_parts ? Ttot : num_parts;
   long long s = 0, n = 0;
   for (int b = 0; b < B; ++b) {
     piece_base[b] = n;
-    const long long t = ceil_div_ll(ctx_len[b], kTile);
+    const long long t = ceil_div_ll(ctx_len[b], tile);
     if (t > 0) n += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
     s += t;
   }
   piece_base[B] = n;
   return n;
 }
+
+long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *piece_base) {
+  return mla_plan_pieces_tiled(ctx_len, B, num_parts, kTile, piece_base);
+}
+
+int mla_plan_tile(const mla_handle *h, int fp8) { return h ? plan_tile_of(h, fp8 != 0) : -1; }
 
 }  // extern "C"

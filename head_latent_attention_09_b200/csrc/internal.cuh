@@ -16,8 +16,9 @@ namespace mla {
 // Devices a process may drive (per-device launch set-up is kept per index).
 constexpr int kMaxDevices = 64;
 
-// KV tokens per tile; the split plan and every attention kernel work in whole
-// tiles, and the paged fast paths require page_size == kTile.
+// KV tokens per page of the paged fast paths (page_size == kTile), the
+// granularity of a token range's first token, and the smallest tile of the
+// split plan.
 constexpr int kTile = 64;
 
 // FP8 latent cache: channels per scale group (over c^KV, then over k^R).
@@ -122,7 +123,10 @@ struct mla_handle {
 namespace mla {
 
 // ---------------------------------------------------------------------------
-// Split plan.  Sequence b contributes T_b = ceil(ctx_b / kTile) tiles; the
+// Split plan.  Sequence b contributes T_b = ceil((end_b - begin_b) / tile)
+// tiles of `tile` tokens (the MMA tile of the attention kernel that runs:
+// 256 for 128 heads, 128 for 16/32 heads, 64 on the CUDA cores, so that a
+// share never pays for a partial tile in the middle of a sequence); the
 // batch's Ttot tiles, in sequence order, are cut into P equal shares
 // [begin(w), begin(w+1)).  A (share, sequence) intersection is a piece: it
 // yields one partial ctx_lat and log-sum-exp.  P is clamped to Ttot so that no
@@ -199,6 +203,7 @@ struct AttnArgs {
   int n_groups;
   char *ws;
   WsLayout L;
+  int plan_tile;     // tokens per tile of the split plan
   unsigned *status;
 };
 
@@ -211,8 +216,9 @@ struct AttnArgs {
 // a multiple of kTile and clamped to [0, end_b].  Any value it has to change
 // is flagged in the status word.  It stores both in the workspace; every
 // attention kernel reads those instead of the caller's arrays, so that the
-// plan's tiles and the kernels' token ranges agree.
-cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, char *ws,
+// plan's tiles and the kernels' token ranges agree.  `tile` (a multiple of
+// kTile) is the plan's tile in tokens.
+cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, int tile, char *ws,
                         const WsLayout &L, unsigned *status, cudaStream_t s);
 
 // The clamped end (context length) of sequence b, as the plan stored it.

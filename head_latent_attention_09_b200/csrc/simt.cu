@@ -74,7 +74,8 @@ __device__ long long block_exclusive_scan(long long v, long long *smem, long lon
 }
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const int *ctx_len, int B, int P_req,
-                                                    long long cap, char *ws, WsLayout L, unsigned *status) {
+                                                    long long cap, int tile, char *ws, WsLayout L,
+                                                    unsigned *status) {
   pdl_trigger();
   pdl_wait();   // the workspace may still be read by the previous step's combine
   __shared__ long long scan[32];
@@ -103,13 +104,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const 
     }
     ctx_eff[b] = (int)c;
     beg_eff[b] = (int)g;
-    local += ceil_div_ll(c - g, kTile);
+    local += ceil_div_ll(c - g, tile);
   }
   long long Ttot;
   long long run = block_exclusive_scan(local, scan, &Ttot);
   for (int b = b0; b < b1; ++b) {
     tile_prefix[b] = run;
-    run += ceil_div_ll(ctx_eff[b] - beg_eff[b], kTile);
+    run += ceil_div_ll(ctx_eff[b] - beg_eff[b], tile);
   }
   if (tid == 0) tile_prefix[B] = Ttot;
   const long long P = Ttot < (long long)P_req ? Ttot : (long long)P_req;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const 
   long long local_pieces = 0;
   for (int b = b0; b < b1; ++b) {
     long long s = tile_prefix[b];
-    long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], kTile);
+    long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], tile);
     if (t > 0) local_pieces += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
   long long n_pieces;
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const 
   for (int b = b0; b < b1; ++b) {
     piece_base[b] = prun;
     long long s = tile_prefix[b];
-    long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], kTile);
+    long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], tile);
     if (t > 0) prun += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
   if (tid == 0) {
@@ -190,8 +191,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
     const long long piece = pb[b] + (w - plan_share_of_tile(tp[b], P, Ttot));
     const int ctx = plan_ctx(a.ws, a.L, b);
     const long long beg = plan_begin_tok(a.ws, a.L, b, a.B);
-    const long long p_begin = beg + (s0 - tp[b]) * kTile;
-    const long long p_end = min((long long)ctx, beg + (s1 - tp[b]) * kTile);
+    const long long p_begin = beg + (s0 - tp[b]) * a.plan_tile;
+    const long long p_end = min((long long)ctx, beg + (s1 - tp[b]) * a.plan_tile);
 
     float q[kQPerLane];
 #pragma unroll
@@ -512,11 +513,13 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const T *o, const T *w
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, char *ws,
+cudaError_t launch_plan(const int *ctx_begin, const int *ctx_len, int B, int P, long long cap, int tile, char *ws,
                         const WsLayout &L, unsigned *status, cudaStream_t s) {
+  if (tile < kTile || tile % kTile != 0) return cudaErrorInvalidValue;
   // one thread per sequence up to 1024 (each thread takes a run of sequences beyond)
   const int threads = B >= 1024 ? 1024 : (B <= 32 ? 32 : (B + 31) / 32 * 32);
-  return launch_pdl(plan_kernel, dim3(1), dim3(threads), 0, s, 1, ctx_begin, ctx_len, B, P, cap, ws, L, status);
+  return launch_pdl(plan_kernel, dim3(1), dim3(threads), 0, s, 1, ctx_begin, ctx_len, B, P, cap, tile, ws, L,
+                    status);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &a, int P, bool fp32, cudaStream_t s) {

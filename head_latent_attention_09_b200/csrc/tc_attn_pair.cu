@@ -150,8 +150,8 @@ __device__ __forceinline__ bool walk_next(Walk &w, const AttnArgs &a, int share,
     const int beg = plan_begin_tok(a.ws, a.L, b, a.B);
     pc.b = b;
     pc.piece = w.pb[b] + (share - plan_share_of_tile(w.tp[b], w.P, w.Ttot));
-    pc.tok_begin = beg + (int)((s0 - w.tp[b]) * kTile);
-    const long long e = beg + (s1 - w.tp[b]) * kTile;
+    pc.tok_begin = beg + (int)((s0 - w.tp[b]) * a.plan_tile);
+    const long long e = beg + (s1 - w.tp[b]) * a.plan_tile;
     pc.tok_end = (int)(e < ctx ? e : ctx);
     pc.ctx = ctx;
     pc.ntiles = (pc.tok_end - pc.tok_begin + kTileTok - 1) / kTileTok;

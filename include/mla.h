@@ -39,7 +39,10 @@
  *       block_table[b*max_blocks_per_seq + p/page_size], row p%page_size.
  *   - RoPE rotates consecutive pairs (x_2k, x_2k+1) of the d_r-wide rotary part
  *     by angle pos*theta_k, theta_k = rope_base^(-2k/d_r) (RoFormer form; the
- *     angle is formed in double precision).
+ *     angle keeps double-precision accuracy: formed in double on the CUDA
+ *     cores; in the tensor-core GEMMs as the exact product pos*theta_hi plus
+ *     pos*theta_lo for a float pair theta_hi + theta_lo = theta_k, reduced by
+ *     2 pi in three parts before the sine and cosine).
  *   - Host-side argument checks return an error before anything is launched.
  *     Checks that need device data (positions, lengths, block ids beyond the
  *     table or pool) are made in the kernels: an offending access is skipped
@@ -302,6 +305,19 @@ int mla_get_device_status(mla_handle *handle, mla_stream_t stream);
  *   piece_base[b] .. piece_base[b+1]-1.  Returns the total number of pieces,
  *   or -1 on invalid arguments. */
 long long mla_plan_pieces(const int *ctx_len, int B, int num_parts, long long *piece_base);
+
+/* The same plan with tiles of tile_tokens tokens (a multiple of 64):
+ * sequence b contributes ceil(ctx_len[b] / tile_tokens) tiles, and the batch's
+ * tiles are cut into num_parts equal shares.  mla_plan_pieces is this with 64.
+ * Returns -1 on invalid arguments. */
+long long mla_plan_pieces_tiled(const int *ctx_len, int B, int num_parts, int tile_tokens, long long *piece_base);
+
+/* Tokens per tile of the split plan mla_decode_attn (fp8 = 0) or
+ * mla_decode_attn_fp8 (fp8 = 1) uses with this handle: the MMA tile of the
+ * attention kernel it runs (256 for 128 heads in bf16, 128 for 16 or 32
+ * heads, 64 on the CUDA cores), so that a share pays for no partial tile
+ * inside a sequence.  -1 for a NULL handle. */
+int mla_plan_tile(const mla_handle *handle, int fp8);
 
 /* Allocation-free variant of mla_decode_attn followed by mla_combine_splits.
  * The pages have no counterpart: this entry point exists for callers that

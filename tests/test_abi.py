@@ -88,9 +88,9 @@ def test_create_without_device_fails_cleanly(lib):
                                    None) == M.MLA_ERR_INVALID_ARG
 
 
-def python_plan(ctx, P):
+def python_plan(ctx, P, tile=64):
     """Independent restatement of the split plan for checking the library's."""
-    tiles = [(c + 63) // 64 for c in ctx]
+    tiles = [(c + tile - 1) // tile for c in ctx]
     starts = np.concatenate([[0], np.cumsum(tiles)]).astype(int)
     total = int(starts[-1])
     P = min(P, total)
@@ -127,6 +127,21 @@ def test_plan_matches_independent_restatement(lib, seed):
         if share:
             sizes = [b - a for a, b in share]
             assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+@pytest.mark.parametrize("tile", [64, 128, 256])
+@pytest.mark.parametrize("seed", range(3))
+def test_tiled_plan_matches_independent_restatement(lib, seed, tile):
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.integers(1, 40))
+    ctx = rng.integers(0, 5000, size=B)
+    ctx[rng.random(B) < 0.2] = 0
+    for P in (1, 3, 74, 148, 1000):
+        n, base = M.mla_plan_pieces_tiled(ctx.tolist(), P, tile)
+        n2, base2, _ = python_plan(ctx.tolist(), P, tile)
+        assert n == n2 and base == base2 and n <= P + B
+    assert M.mla_plan_pieces_tiled(ctx.tolist(), 4, 96)[0] == -1     # not a multiple of 64
+    assert M.mla_plan_pieces_tiled(ctx.tolist(), 4, 64) == M.mla_plan_pieces(ctx.tolist(), 4)
 
 
 def test_plan_v2_workload(lib):

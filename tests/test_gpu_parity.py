@@ -313,3 +313,14 @@ def test_strict_mode_refuses_instead_of_substituting():
         assert M.mla_get_device_status(handle) == M.MLA_OK
     finally:
         M.mla_destroy(handle)
+
+
+def test_plan_tile_follows_the_attention_kernel():
+    # the split plan counts tiles of the attention kernel's own MMA tile
+    for n_h, tile, tile_fp8 in ((128, 256, 64), (16, 128, 128), (32, 128, 128), (8, 64, 64)):
+        wl = WORKLOADS["v2lite_b32_ctx4k"].with_(n_h=n_h)
+        h = M.mla_create(config_of(wl))
+        try:
+            assert M.mla_plan_tile(h) == tile and M.mla_plan_tile(h, fp8=True) == tile_fp8
+        finally:
+            M.mla_destroy(h)
