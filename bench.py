@@ -51,6 +51,9 @@ def parse():
                     help="skip the separate timings of the other workloads (V2-Lite, ragged paged, 128K)")
     ap.add_argument("--attn-samples", type=int, default=200,
                     help="attention calls timed one by one for the median and p10/p90")
+    ap.add_argument("--only-config", default=None,
+                    help="run only the step and attention timing of this workload (any in workloads.WORKLOADS, "
+                         "paged and ragged ones included) and print its object; for profiling")
     ap.add_argument("--fused", action="store_true",
                     help="finish the step with mla_combine_out_proj instead of mla_combine_splits + mla_out_proj")
     ap.add_argument("--launch-check", action="store_true",
@@ -85,6 +88,25 @@ def measured_traffic(workload_name):
     if workload_name != WORKLOAD or rec.get("kernel_source_sha256") != sha:
         return None
     return float(rec["traffic_per_bench_launch"])
+
+
+def smallh_traffic(workload_name):
+    """DRAM bytes of one 16/32-head attention launch on this workload, from the
+    committed ncu record (profiles/attn_smallh_traffic.json); None when the
+    kernel source has changed since the capture or the workload is not in it."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_smallh_traffic.json")) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "head_latent_attention_09_b200", "csrc", "tc_attn_smallh.cu")
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except Exception:
+        return None
+    w = rec.get("workloads", {}).get(workload_name)
+    if w is None or rec.get("kernel_source_sha256") != sha:
+        return None
+    return float(w["traffic_per_launch"])
 
 
 def algorithmic_bytes(wl, ctx_sum, with_wo=False):
@@ -506,6 +528,7 @@ def measure_workload(M, wl, dev, steps, seed, hbm_peak, n_samples=100):
         M.mla_destroy(handle)
     med = float(np.median(t))
     gbs = cache_bytes / (med * 1e-6) / 1e9
+    traffic = smallh_traffic(wl.name) if H in (16, 32) else None
     w_bytes = ((wl.d_c + wl.d_r) * d + 2 * H * wl.d_h * wl.d_c) * 2
     return {"B": B, "n_h": H, "tokens": tokens, "page_size": wl.page_size, "cache_bytes": cache_bytes,
             "cache_copies": copies, "num_parts": P, "us_per_step": step_us,
@@ -513,7 +536,26 @@ def measure_workload(M, wl, dev, steps, seed, hbm_peak, n_samples=100):
             "attn_median_us": med, "attn_p10_us": float(np.percentile(t, 10)),
             "attn_p90_us": float(np.percentile(t, 90)), "attn_gbs": gbs, "attn_frac": gbs / hbm_peak,
             "tokens_scanned_per_s": tokens / (med * 1e-6), "attn_us_at_70pct_of_8TBps": cache_bytes / 5.6e6,
-            "bound": "hbm"}
+            "bound": "hbm",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": traffic, "kernel": "mla_decode_attn (plan + attention)"}}
+
+
+def run_only_config(args):
+    """One workload's decode step and attention calls (measure_workload), on
+    one GPU; prints its object.  Lets a profiler capture the attention kernel
+    of any workload, paged and ragged ones included."""
+    import torch
+
+    import head_latent_attention_09_b200 as M
+    from head_latent_attention_09_b200 import build as _build
+    from workloads import WORKLOADS
+    torch.cuda.set_device(0)
+    _build.build()
+    M.load()
+    r = measure_workload(M, WORKLOADS[args.only_config], torch.device("cuda", 0), args.steps, rank_seed(0) + 29,
+                         peaks()[0], n_samples=max(1, min(args.attn_samples, 100)))
+    print(json.dumps({"workload": args.only_config, **r}), flush=True)
 
 
 def run_ours(args):
@@ -972,6 +1014,8 @@ def main():
         sys.exit(subprocess.call(cmd))
     if args.launch_check:
         launch_check(args)
+    elif args.only_config:
+        run_only_config(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
