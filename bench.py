@@ -957,6 +957,23 @@ def run_ours(args):
             "note": "mla_decode_attn_fp8 vs mla_decode_attn on the same cache; not part of the step"}
     if configs is not None:
         line["configs"] = configs
+    # the step's GEMMs against both of their rooflines: tensor pipe (bf16,
+    # sustained peak) and HBM (their weights and activations once)
+    esz = 2
+    gemm_work = {
+        "cache_append": (2.0 * B * D * d, (D * d + B * d + B * D) * esz),
+        "absorb_q": (2.0 * B * H * wl.d_h * wl.d_c, (H * wl.d_h * wl.d_c + B * H * wl.d_h + B * H * D) * esz),
+        "out_proj": (2.0 * B * H * wl.d_h * wl.d_c, (H * wl.d_h * wl.d_c + B * H * wl.d_c + B * H * wl.d_h) * esz),
+    }
+    line["gemms"] = {}
+    for name, (fl, by) in gemm_work.items():
+        us = per_call[name]
+        line["gemms"][name] = {
+            "us_per_call": us, "gflop": fl / 1e9, "tflops": fl / (us * 1e-6) / 1e12,
+            "tensor_frac": fl / (us * 1e-6) / 1e12 / tf_peak, "algorithmic_bytes": by,
+            "gbs": by / (us * 1e-6) / 1e9, "hbm_frac": by / (us * 1e-6) / 1e9 / hbm_peak}
+    line["gemms"]["note"] = ("per call, events between calls; tensor_frac against the bf16 sustained peak "
+                             "(TFLOP/s), hbm_frac against the HBM peak")
     if qproj is not None:
         gbs = qproj["bytes"] / (qproj["us"] * 1e-6) / 1e9
         line["query_proj"] = {

@@ -170,6 +170,36 @@ def test_attention_split_counts(name, parts):
 
 
 @pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k"])
+def test_attention_long_ragged_contexts(name):
+    """Long contexts of unequal length at the default split count: shares cut
+    in the kernel's own tile (256 or 128 tokens) cross sequence ends that are
+    not on a tile boundary."""
+    wl = WORKLOADS[name]
+    ctx = [40000, 1, 70001, 257, 0, 12345]
+    gc, gl, wc, wlse = _attention_only(wl, ctx, 0)
+    seqs = [b for b in range(len(ctx)) if ctx[b] > 0]
+    compare(gc, wc, wl, "ctx_lat long ragged", seqs)
+    compare(gl, wlse, wl, "lse long ragged", seqs)
+
+
+@pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k"])
+def test_attention_many_short_sequences(name):
+    """300 short ragged sequences at the default split count: many pieces per
+    share, sequences of one token and empty ones."""
+    wl = WORKLOADS[name]
+    rng = np.random.default_rng(77)
+    ctx = rng.integers(0, 700, size=300)
+    ctx[::37] = 0
+    ctx[5::41] = 1
+    gc, gl, wc, wlse = _attention_only(wl, ctx.tolist(), 0)
+    seqs = [b for b in range(len(ctx)) if ctx[b] > 0][::7]
+    compare(gc, wc, wl, "ctx_lat many short", seqs)
+    compare(gl, wlse, wl, "lse many short", seqs)
+    for b in np.nonzero(ctx == 0)[0]:
+        assert np.all(gc[b] == 0) and np.all(np.isneginf(gl[b]))
+
+
+@pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k"])
 def test_attention_late_dominant_key(name):
     """A key far above the others late in the sequence forces the running
     maximum to jump (the rescale path)."""
