@@ -154,6 +154,7 @@ struct WsLayout {
   size_t tile_prefix_off;  // int64 [B+1]
   size_t piece_base_off;   // int64 [B+1]
   size_t ctx_off;          // int32 [2][B]: each sequence's end and first token as attended (clamped by the plan)
+  size_t share_first_off;  // int32 [P]: the first sequence whose tiles reach into each share
   size_t opart_off;        // float [n_h, max_pieces, d_c]: a head's pieces are consecutive rows
   size_t lse_off;          // float [n_h, max_pieces]
   size_t total;
@@ -178,6 +179,8 @@ inline WsLayout ws_layout(const mla_config &cfg, int B, int P) {
   off = align_up(off + sizeof(long long) * (size_t)(B + 1), 256);
   L.ctx_off = off;
   off = align_up(off + 2 * sizeof(int) * (size_t)(B > 0 ? B : 1), 256);
+  L.share_first_off = off;
+  off = align_up(off + sizeof(int) * (size_t)(P > 0 ? P : 1), 256);
   L.opart_off = off;
   off = align_up(off + sizeof(float) * (size_t)L.max_pieces * cfg.n_h * cfg.d_c, 256);
   L.lse_off = off;

@@ -129,6 +129,19 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int *ctx_begin, const 
     long long t = ceil_div_ll(ctx_eff[b] - beg_eff[b], tile);
     if (t > 0) prun += plan_share_of_tile(s + t - 1, P, Ttot) - plan_share_of_tile(s, P, Ttot) + 1;
   }
+  // Each share's first sequence (the first whose tiles reach past the share's
+  // first tile), so that the attention kernels need no search; tile_prefix is
+  // complete here (the scan above synchronised the block).
+  int *share_first = reinterpret_cast<int *>(ws + L.share_first_off);
+  for (long long w = tid; w < P; w += nt) {
+    const long long t0 = plan_begin(w, P, Ttot);
+    int lo = 0, hi = B;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_prefix[mid + 1] <= t0) lo = mid + 1; else hi = mid;
+    }
+    share_first[w] = lo;
+  }
   if (tid == 0) {
     piece_base[B] = n_pieces;
     WsHeader *hd = reinterpret_cast<WsHeader *>(ws);
@@ -178,12 +191,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
   const T *qg = reinterpret_cast<const T *>(a.q_abs);
 
   const long long t0 = plan_begin(w, P, Ttot), t1 = plan_begin(w + 1, P, Ttot);
-  // first sequence whose tiles reach past t0
-  int lo = 0, hi = a.B;
-  while (lo < hi) {
-    int mid = (lo + hi) >> 1;
-    if (tp[mid + 1] <= t0) lo = mid + 1; else hi = mid;
-  }
+  // first sequence whose tiles reach past t0 (found by the plan)
+  const int lo = reinterpret_cast<const int *>(a.ws + a.L.share_first_off)[w];
   for (int b = lo; b < a.B && tp[b] < t1; ++b) {
     const long long s0 = t0 > tp[b] ? t0 : tp[b];
     const long long s1 = t1 < tp[b + 1] ? t1 : tp[b + 1];

@@ -127,12 +127,7 @@ __device__ __forceinline__ void walk_init(Walk &w, const AttnArgs &a, int share)
   }
   w.t0 = plan_begin(share, w.P, w.Ttot);
   w.t1 = plan_begin(share + 1, w.P, w.Ttot);
-  int lo = 0, hi = a.B;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (w.tp[mid + 1] <= w.t0) lo = mid + 1; else hi = mid;
-  }
-  w.b = lo;
+  w.b = reinterpret_cast<const int *>(a.ws + a.L.share_first_off)[share];   // found by the plan
 }
 
 __device__ __forceinline__ bool walk_next(Walk &w, const AttnArgs &a, int share, Piece &pc) {
