@@ -197,7 +197,9 @@ int mla_default_num_parts(const mla_handle *handle);
 
 /* Split-KV decode attention over the latent cache (V3 note: o_{t,i} with the
  * softmax over j = 1..t, scale 1/sqrt(d_h + d_r); absorbed form of V2 App. C).
- * The batch's KV tokens, in 64-token tiles, are cut into num_parts equal shares;
+ * The batch's KV tokens, in tiles of mla_plan_tile(handle, 0) tokens (the
+ * attention kernel's own tile: 256, 128 or 64), are cut into num_parts equal
+ * shares;
  * each share is processed by one worker (one CTA, or one CTA pair for 128
  * heads) and yields, per (sequence, share) piece, the normalised partial
  * ctx_lat and its log-sum-exp, written into the workspace.
@@ -299,7 +301,9 @@ int mla_selftest_wait_timeout(mla_handle *handle, long long limit_ns, mla_stream
  * Returns MLA_OK, MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_BOUNDS or MLA_ERR_CUDA. */
 int mla_get_device_status(mla_handle *handle, mla_stream_t stream);
 
-/* Host mirror of the split plan mla_decode_attn uses (no CUDA calls).
+/* Host mirror of the split plan with 64-token tiles, the plan of the CUDA-core
+ * kernels (no CUDA calls); mla_plan_pieces_tiled with mla_plan_tile(handle, fp8)
+ * mirrors the plan any handle uses.
  *   ctx_len host int32 [B]; num_parts as for mla_decode_attn (must be > 0 here).
  *   piece_base host int64 [B+1] (out): pieces of sequence b are
  *   piece_base[b] .. piece_base[b+1]-1.  Returns the total number of pieces,
