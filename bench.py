@@ -901,7 +901,7 @@ def run_ours(args):
         gbs, desc, threads, _ = cpu_oracle_sample(wl, 16, budget_s=15.0)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc}
         if not args.batch:
-            cpu["configs"] = {name: cpu_oracle_workload(WORKLOADS[name], budget_s=15.0)
+            cpu["configs"] = {name: cpu_oracle_workload(WORKLOADS[name], budget_s=45.0)
                               for name in ("tiny_fp32", "v2lite_b32_ctx4k", "v2lite_paged_ragged_b128")}
     line = {
         "metric": "MLA decode: HBM GB/s (% of peak) and us/step at B=64, n_h=128, ctx 8K",
