@@ -108,6 +108,14 @@ def test_small_ragged_steps(name, ctx):
             assert np.all(got["ctx_lat"][b] == 0) and np.all(np.isneginf(got["lse"][b]))
 
 
+def test_paged_128_heads():
+    """The 128-head pair kernel over a paged pool (64-token pages, each 128-token
+    half of a tile staged as two page boxes), ragged contexts, W^O."""
+    wl = WORKLOADS["v2_b64_ctx8k"].with_(B=5, ctx=(1, 64, 65, 300, 1000), page_size=64)
+    got = run_decode_step(wl, with_wo=True)
+    _check_step(wl, got, list(range(5)), with_wo=True, explicit_heads=[0, 127])
+
+
 def test_paged_small():
     wl = WORKLOADS["v2lite_paged_ragged_b128"].with_(B=6, ctx=(1, 64, 65, 300, 1, 130))
     got = run_decode_step(wl)
