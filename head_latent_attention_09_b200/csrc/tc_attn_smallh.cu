@@ -26,15 +26,21 @@
 // Per-head softmax statistics are reductions across tokens, i.e. across
 // threads: warp shuffles over 32 lanes, then shared memory across the warps.
 //
-// Warp roles: warp 0 TMA producer, warp 1 tensor-memory allocation and MMA
-// issue, warps 2-5 softmax / rescale / epilogue.
+// Warp roles: warps 0 and 6 TMA producers (bf16; FP8 has warp 0 only), warp 1
+// tensor-memory allocation and MMA issue, warps 2-5 softmax / rescale /
+// epilogue.
 //
 // FP8 cache (E4M3 codes, a float32 scale per token and 128-channel group):
-// the producer stages each 128 x 64 chunk of codes (8 KB) by TMA, and four
-// more warps (6-9) widen it into the bf16 chunk the MMAs read, applying the
-// group scale on the way (code * sigma rounded to bf16).  HBM then carries
-// 576 B + 20 B of scales per token instead of 1152 B; the products, the
-// softmax and the epilogue are those of the bf16 cache.
+// the producer stages the codes by TMA (16 heads: per 64-row half of a tile,
+// one box of three 64-code chunks), and six more warps (6-11) widen each
+// 128 x 64 chunk into the bf16 chunk the MMAs read, applying the group scale
+// on the way (code * sigma rounded to bf16).  HBM then carries 576 B + 20 B
+// of scales per token instead of 1152 B; the products, the softmax and the
+// epilogue are those of the bf16 cache, with the rotary chunk taken last.
+// The widening sets the pace: a tile's chunks are widened one after another
+// into the pair slots as P.V of the previous tile frees them, at about 0.6 us
+// a chunk inside the kernel (a clock trace of one CTA), so the FP8 tile takes
+// longer than the bf16 one although it reads half the bytes.
 //
 // Every wait is bounded; a wait that runs out flags MLA_ERR_TIMEOUT and the
 // kernel winds down without further waits.
@@ -55,7 +61,10 @@ constexpr int kGroups8 = 5;                // scale groups of a 576-wide row
 
 template <int H, bool F8>
 struct Cfg {
-  static constexpr int kConvWarps = F8 ? 4 : 0;                 // FP8 converter warps
+  // FP8 converter warps: six make 12 warps, three per sub-partition, which
+  // leaves the 168-register cap of ten warps unchanged (measured 2 % faster
+  // than four).
+  static constexpr int kConvWarps = F8 ? 6 : 0;
   // bf16: a second TMA producer, warp 6 (the rotary chunk and latent pairs
   // 2-3 of every tile; warp 0 the query and pairs 0-1).  A thread issuing
   // cp.async.bulk.tensor copies sustains about two per microsecond, and a
@@ -63,18 +72,32 @@ struct Cfg {
   static constexpr int kProducers = F8 ? 1 : 2;
   static constexpr int kProd1Warp = 6;
   static constexpr int kThreads = 192 + 32 * kConvWarps + 32 * (kProducers - 1);
-  static constexpr int kNL = (!F8 && H <= 16) ? 5 : 4;          // latent pair slots (a tile takes 4)
-  static constexpr int kNR = (F8 && H > 16) ? 1 : 2;            // rotary chunk slots
-  static constexpr int kNSt = F8 ? (H <= 16 ? 4 : 3) : 0;       // FP8 staging chunks
+  // Latent pair slots: a tile takes 4; with a fifth (bf16, 16 heads) the
+  // next tile's first pair is staged, and its S^T chunks issued, before P.V
+  // of this tile frees a slot.  (FP8 has no room for one beside a staging
+  // ring deep enough to cover the TMA latency.)
+  static constexpr int kNL = (!F8 && H <= 16) ? 5 : 4;
+  static constexpr int kNR = F8 ? 1 : 2;                        // rotary chunk slots
+  // FP8 staging: slots of kStCh chunks of codes, laid out [64-row half]
+  // [chunk][64 rows][64 B] so that one 3D box brings a half's kStCh chunks
+  // (kStCh = 1: a 2D box per half).  16 heads: two slots of three chunks,
+  // six copies per tile in place of eighteen.
+  static constexpr int kStCh = (F8 && H <= 16) ? 3 : 1;
+  static constexpr int kNSt = F8 ? (H <= 16 ? 2 : 3) : 0;       // FP8 staging slots
+  static constexpr int kStBytes = kStCh * kChunk8;
   static constexpr int kEarlyPairs = kNL - 4;                   // next tile's pairs issued before P.V
   static constexpr bool kEarlyRope = kNR >= 2;                  // next tile's rotary chunk likewise
+  // FP8: S^T takes the latent chunks first and the rotary chunk last, the
+  // order in which the converters fill them (chunk indices consecutive, as
+  // a multi-chunk staging box needs).
+  static constexpr bool kRopeLast = F8;
   static constexpr int kQ = 9 * H * 128;                        // H rows x 576, nine 64-column chunks
   static constexpr int kPT = 2 * H * 128;                       // P^T: H rows x 128 tokens, two 64-token chunks
   static constexpr int kOffQ = 0;
   static constexpr int kOffLat = (kQ + 1023) / 1024 * 1024;
   static constexpr int kOffRope = kOffLat + kNL * kPair;
   static constexpr int kOffStage = kOffRope + kNR * kChunk;
-  static constexpr int kOffP = kOffStage + kNSt * kChunk8;
+  static constexpr int kOffP = kOffStage + kNSt * kStBytes;
   static constexpr int kPStride = (kPT + 1023) / 1024 * 1024;
   static constexpr int kOffRed = kOffP + 2 * kPStride;          // float [2][4][H] max, [4][H] sum
   static constexpr int kOffBar = kOffRed + 12 * H * 4;
@@ -90,6 +113,8 @@ struct Cfg {
   static constexpr uint32_t kColO = 2 * H;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static_assert(kNL >= 4, "a tile takes four pair slots");
+  static_assert(9 % kStCh == 0, "staging slots hold whole thirds or ninths of a row");
+  static_assert(!kRopeLast || !kEarlyRope, "the rotary chunk is either first (and may be early) or last");
 };
 
 // Two E4M3 codes (low byte first) times sigma, as a bf16 pair.
@@ -295,7 +320,7 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
     // ------------------------------------------------------------- producers
     // Per tile, in the order the MMAs consume them: the rotary chunk, then
     // the four latent pairs (bf16), or the nine chunks of codes into the
-    // staging ring (FP8: rotary chunk first, then latent chunks 0-7).  With
+    // staging ring (FP8: latent chunks 0-7, then the rotary chunk).  With
     // two producers each walks every tile and ring position but fills only
     // its own slots: producer 0 the query and pairs 0-1, producer 1 the
     // rotary chunk and pairs 2-3.
@@ -366,16 +391,35 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
           if (lane == 0) ptx::mbar_arrive_expect_tx(full, tx);
         };
         if (F8) {
-          // nine chunks of codes, rotary first
-          for (int j = 0; j < 9 && ok; ++j) {
-            const int c = j == 0 ? 8 : j - 1;
+          // The nine chunks of codes in index order (the rotary chunk last),
+          // kStCh to a staging slot: per 64-row half one box of kStCh chunks
+          // (3D map) or of one chunk (2D map), or the hand copy of the half
+          // that holds the sequence's end.
+          constexpr int SC = C::kStCh, kHalfSt = SC * kChunk8 / 2;
+          for (int g = 0; g < 9 / SC && ok; ++g) {
             uint64_t *full = bar + C::bStFull + stg.slot;
             if (!slot_free(bar + C::bStEmpty + stg.slot, stg)) { ok = false; break; }
-            uint8_t *dst = sStage + stg.slot * kChunk8;
+            uint8_t *dst = sStage + stg.slot * C::kStBytes;
             uint32_t tx = 0;
-            stage_chunk(dst, c, kChunk8 / 2, tx);
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+              if (kind[h2] == 2) {
+#pragma unroll 1
+                for (int cc = 0; cc < SC; ++cc)
+                  hand_copy_half<true>(a, pc, tok0 + 64 * h2, SC * g + cc, dst + h2 * kHalfSt + cc * (kChunk8 / 2));
+              } else {
+                tx += kHalfSt;
+              }
+            }
             arm(full, tx);
-            if (lane == 0) issue_chunk(dst, c, kChunk8 / 2, &mapKV64, full);
+            if (lane == 0) {
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                if (kind[h2] == 2) continue;
+                if (SC == 1) ptx::tma_load_2d(dst + h2 * kHalfSt, &mapKV64, full, 64 * g, yy[h2]);
+                else ptx::tma_load_3d(dst + h2 * kHalfSt, &mapKV, full, 0, yy[h2], SC * g);
+              }
+            }
             stg.advance(NSt);
           }
           continue;
@@ -489,20 +533,25 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
         for (int k = 0; k < pc.ntiles && ok; ++k) {
           const uint32_t dS = tmem + (i & 1) * H;
           // the rest of S^T(i): the rotary chunk and pairs not issued early
-          if (!early_rope) {
+          if (!early_rope && !C::kRopeLast) {
             if (!wait_full(bar + C::bRopeFull + rope.slot, rope.phase)) { ok = false; break; }
             s_chunk(r0 + rope.slot * kChunk, 8, dS, true);
           }
           const int rope_slot = rope.slot;
+          const uint32_t rope_phase = rope.phase;
           rope.advance(NR);
           for (int pb = early_pairs; pb < 4; ++pb) {
             if (!wait_full(bar + C::bLatFull + lat.slot, lat.phase)) { ok = false; break; }
             const uint32_t src = l0 + lat.slot * kPair;
-            s_chunk(src, 2 * pb, dS, false);
+            s_chunk(src, 2 * pb, dS, C::kRopeLast && pb == 0);
             s_chunk(src + kChunk, 2 * pb + 1, dS, false);
             lat.advance(NL);
           }
           if (!ok) break;
+          if (C::kRopeLast) {
+            if (!wait_full(bar + C::bRopeFull + rope_slot, rope_phase)) { ok = false; break; }
+            s_chunk(r0 + rope_slot * kChunk, 8, dS, false);
+          }
           ptx::mma_commit(bar + C::bRopeEmpty + rope_slot);   // the rotary chunk only feeds S
           ptx::mma_commit(bar + C::bSFull + (i & 1));
           if (k == pc.ntiles - 1) ptx::mma_commit(bar + C::bQEmpty);
@@ -686,13 +735,21 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
     }
   } else if (F8) {
     // ------------------------------------------ FP8 converters (warps 6 ..)
-    // A staged chunk is 128 rows x 4 units of 16 codes.  Thread ct handles
-    // unit ct % 4 of rows ct / 4 + 32 rr (rr = 0..3): 16 codes become 32 bytes
-    // of bf16, two 16-byte units of the 128-byte-swizzled chunk.  Chunks come
-    // in the producer's order: the rotary chunk, then latent chunks 0-7.
-    constexpr int RS = 32, NRR = kTileTok / RS;
+    // A staged chunk is 128 rows x 4 units of 16 codes (each 64-row half of a
+    // staging slot holds its kStCh chunks one after another).  Converter
+    // thread ct handles units ct + kCT rr of the chunk (unit n: row n / 4,
+    // 16 codes n % 4): 16 codes become 32 bytes of bf16, two 16-byte units of
+    // the 128-byte-swizzled chunk.  Chunks come in index order: latent
+    // chunks 0-7, then the rotary chunk.
+    constexpr int kCT = 32 * (C::kConvWarps > 0 ? C::kConvWarps : 1), kUnitsCh = kTileTok * 4;   // (bf16: never runs)
+    constexpr int RS = kCT / 4, NRR = (kUnitsCh + kCT - 1) / kCT;
+    static_assert(kCT % 4 == 0 && kCT % 32 == 0, "converter rows");
+    constexpr int SC = C::kStCh, kHalfSt = SC * kChunk8 / 2;
     const int ct = (warp - 6) * 32 + lane;
     const int r0 = ct >> 2, u = ct & 3;
+    // unit rr of this thread lies in the chunk (warp-uniform: kCT and the
+    // chunk's unit count are multiples of 32)
+    auto has = [&](int rr) { return ct + kCT * rr < kUnitsCh; };
     Walk w;
     walk_init(w, a, share);
     Piece pc;
@@ -709,55 +766,60 @@ __global__ void __launch_bounds__(Cfg<H, F8>::kThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < NRR; ++rr) {
           const int t = tok0 + r0 + RS * rr;
-          const long long r = t < pc.ctx ? kv_row(a, pc.b, t) : -1;
+          const long long r = has(rr) && t < pc.ctx ? kv_row(a, pc.b, t) : -1;
 #pragma unroll
           for (int g = 0; g < kGroups8; ++g) sig[rr][g] = r >= 0 ? a.kv_scale[r * kGroups8 + g] : 0.f;
         }
-        for (int j = 0; j < 9; ++j) {
-          const int c = j == 0 ? 8 : j - 1;
+        for (int g = 0; g < 9 / SC && ok; ++g) {
           if (!warp_wait(bar + C::bStFull + stg.slot, stg.phase, a.status, abort_flag)) { ok = false; break; }
-          uint8_t *dst;
-          uint64_t *full;
-          if (c == 8) {
-            if (!slot_free(bar + C::bRopeEmpty + rope.slot, rope)) { ok = false; break; }
-            dst = sRope + rope.slot * kChunk;
-            full = bar + C::bRopeFull + rope.slot;
-          } else {
-            if ((c & 1) == 0 && !slot_free(bar + C::bLatEmpty + lat.slot, lat)) { ok = false; break; }
-            dst = sLat + lat.slot * kPair + (c & 1) * kChunk;
-            full = bar + C::bLatFull + lat.slot;
-          }
-          const int g = c >> 1;   // chunks 0-7: c^KV groups 0-3; chunk 8: the k^R group
+          const uint8_t *src = sStage + stg.slot * C::kStBytes;
+          for (int cc = 0; cc < SC; ++cc) {
+            const int c = SC * g + cc;
+            uint8_t *dst;
+            uint64_t *full;
+            if (c == 8) {
+              if (!slot_free(bar + C::bRopeEmpty + rope.slot, rope)) { ok = false; break; }
+              dst = sRope + rope.slot * kChunk;
+              full = bar + C::bRopeFull + rope.slot;
+            } else {
+              if ((c & 1) == 0 && !slot_free(bar + C::bLatEmpty + lat.slot, lat)) { ok = false; break; }
+              dst = sLat + lat.slot * kPair + (c & 1) * kChunk;
+              full = bar + C::bLatFull + lat.slot;
+            }
+            const int gi = c >> 1;   // chunks 0-7: c^KV groups 0-3; chunk 8: the k^R group
 #pragma unroll
-          for (int rr = 0; rr < NRR; ++rr) {
-            const int rw = r0 + RS * rr;
-            // select the group's scale without indexing the array at run time
-            float sg = sig[rr][0];
+            for (int rr = 0; rr < NRR; ++rr) {
+              if (!has(rr)) continue;
+              const int rw = r0 + RS * rr;
+              // select the group's scale without indexing the array at run time
+              float sg = sig[rr][0];
 #pragma unroll
-            for (int gg = 1; gg < kGroups8; ++gg) sg = g == gg ? sig[rr][gg] : sg;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(sStage + stg.slot * kChunk8 + rw * 64 + 16 * u);
-            uint4 lo, hi;
-            lo.x = e4m3x2_to_bf16x2(raw.x, sg);
-            lo.y = e4m3x2_to_bf16x2(raw.x >> 16, sg);
-            lo.z = e4m3x2_to_bf16x2(raw.y, sg);
-            lo.w = e4m3x2_to_bf16x2(raw.y >> 16, sg);
-            hi.x = e4m3x2_to_bf16x2(raw.z, sg);
-            hi.y = e4m3x2_to_bf16x2(raw.z >> 16, sg);
-            hi.z = e4m3x2_to_bf16x2(raw.w, sg);
-            hi.w = e4m3x2_to_bf16x2(raw.w >> 16, sg);
-            uint8_t *d = dst + rw * 128;
-            *reinterpret_cast<uint4 *>(d + (((2 * u) ^ (rw & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4 *>(d + (((2 * u + 1) ^ (rw & 7)) << 4)) = hi;
+              for (int gg = 1; gg < kGroups8; ++gg) sg = gi == gg ? sig[rr][gg] : sg;
+              const uint4 raw = *reinterpret_cast<const uint4 *>(src + (rw >> 6) * kHalfSt + cc * (kChunk8 / 2) +
+                                                                 (rw & 63) * 64 + 16 * u);
+              uint4 lo, hi;
+              lo.x = e4m3x2_to_bf16x2(raw.x, sg);
+              lo.y = e4m3x2_to_bf16x2(raw.x >> 16, sg);
+              lo.z = e4m3x2_to_bf16x2(raw.y, sg);
+              lo.w = e4m3x2_to_bf16x2(raw.y >> 16, sg);
+              hi.x = e4m3x2_to_bf16x2(raw.z, sg);
+              hi.y = e4m3x2_to_bf16x2(raw.z >> 16, sg);
+              hi.z = e4m3x2_to_bf16x2(raw.w, sg);
+              hi.w = e4m3x2_to_bf16x2(raw.w >> 16, sg);
+              uint8_t *d = dst + rw * 128;
+              *reinterpret_cast<uint4 *>(d + (((2 * u) ^ (rw & 7)) << 4)) = lo;
+              *reinterpret_cast<uint4 *>(d + (((2 * u + 1) ^ (rw & 7)) << 4)) = hi;
+            }
+            ptx::fence_proxy_async_smem();   // the MMAs read the slot through the async proxy
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(full);
+            if (c == 8) rope.advance(NR);
+            else if (c & 1) lat.advance(NL);
           }
-          ptx::fence_proxy_async_smem();   // the MMAs read the slot through the async proxy
+          if (!ok) break;
           __syncwarp();
-          if (lane == 0) {
-            ptx::mbar_arrive(full);
-            ptx::mbar_arrive(bar + C::bStEmpty + stg.slot);
-          }
+          if (lane == 0) ptx::mbar_arrive(bar + C::bStEmpty + stg.slot);
           stg.advance(NSt);
-          if (c == 8) rope.advance(NR);
-          else if (c & 1) lat.advance(NL);
         }
       }
     }
@@ -789,6 +851,14 @@ cudaError_t launch_h(const AttnArgs &a, int P, cudaStream_t s) {
     if (!encode_map_u8(&mkv64, a.cache, 2, dkv, st8, bkv64, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorNotSupported;
     mkv = mkv64;
     mpair = mkv64;
+    if (C::kStCh > 1) {
+      // The codes viewed as [9 chunks][rows][64 codes]: one box of 64 rows x
+      // kStCh chunks is one half of a staging slot.
+      const uint64_t d3[3] = {64, (uint64_t)rows, 9};
+      const uint64_t s3[2] = {576, 64};
+      const uint32_t b3[3] = {64, 64, (uint32_t)C::kStCh};
+      if (!encode_map_u8(&mkv, a.cache, 3, d3, s3, b3, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorNotSupported;
+    }
   } else {
     // The cache viewed as [9 chunks][rows][64 columns]: one box of 128 rows x 2
     // chunks lands as two 16 KB row-major chunks, a latent pair slot.

@@ -278,3 +278,61 @@ def test_fp8_attention_rejects_missing_scales():
                                    torch.empty(5, device="cuda"), 64, None, 0, small, 64)
     finally:
         M.mla_destroy(handle)
+
+
+@pytest.mark.parametrize("n_h", [16, 32])
+def test_fp8_attention_every_code(n_h):
+    """Attention over codes drawn directly (not by the quantiser): each row and
+    scale group holds either all 254 non-NaN E4M3 codes at random, or only the
+    subnormal codes (exponent field 0, both signs), with the group's scale
+    chosen so that both kinds carry values of the same size.  Against the
+    oracle's softmax over the dequantised rows (value = code * sigma), this
+    pins the kernel's widening of every code, subnormals included, which the
+    quantiser's output reaches only by chance."""
+    wl = WORKLOADS["v2lite_b32_ctx4k"].with_(B=3, ctx=(700, 129, 1), n_h=n_h)
+    D, G, cache_len = wl.D, 5, 704
+    rng = np.random.default_rng(8675309 + n_h)
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    subnormal = np.array([c for c in range(256) if (c & 0x78) == 0], dtype=np.uint8)
+    codes = rng.choice(finite, size=(wl.B, cache_len, D)).astype(np.uint8)
+    sub_group = rng.random((wl.B, cache_len, G)) < 0.4
+    groups = O.fp8_groups(wl.d_c, wl.d_r)
+    scales = np.empty((wl.B, cache_len, G), np.float32)
+    for g, (a, b) in enumerate(groups):
+        sub_codes = rng.choice(subnormal, size=(wl.B, cache_len, b - a)).astype(np.uint8)
+        codes[:, :, a:b] = np.where(sub_group[:, :, g:g + 1], sub_codes, codes[:, :, a:b])
+        # largest magnitude of the group: 448 for all codes, 7 * 2^-9 for subnormals
+        top = np.where(sub_group[:, :, g], 7.0 * 2.0 ** -9, 448.0)
+        scales[:, :, g] = (0.5 * np.exp2(rng.uniform(-2.0, 2.0, (wl.B, cache_len))) / top).astype(np.float32)
+    q_abs = bf16_round(rng.standard_normal((wl.B, n_h, D)).astype(np.float32))
+    ctx = np.asarray(wl.ctx, np.int32)
+
+    handle = create_handle(wl)
+    try:
+        P = M.mla_default_num_parts(handle)
+        ws_bytes = M.mla_decode_workspace_size(handle, wl.B, P)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        ctx_lat = torch.empty((wl.B, n_h, wl.d_c), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((wl.B, n_h), dtype=torch.float32, device="cuda")
+        M.mla_decode_attn_fp8(handle, torch.from_numpy(q_abs).to(torch.bfloat16).cuda(),
+                              torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(),
+                              cache_len, None, 0, torch.from_numpy(ctx).cuda(), wl.B, P, ws, ws_bytes)
+        M.mla_combine_splits(handle, ws, ws_bytes, wl.B, P, ctx_lat, lse)
+        assert M.mla_get_device_status(handle) == M.MLA_OK
+        got = {"ctx_lat": to_host(ctx_lat), "lse": to_host(lse)}
+    finally:
+        M.mla_destroy(handle)
+    scale = O.attention_scale(wl.d_h, wl.d_r, rope_arg(wl))
+    want = {"ctx_lat": {}, "lse": {}}
+    for b in range(wl.B):
+        rows = O.dequantize_rows_fp8(codes[b, :ctx[b]], scales[b, :ctx[b]], wl.d_c, wl.d_r)
+        want["ctx_lat"][b], want["lse"][b] = O.latent_attention(q_abs[b], rows, d_c=wl.d_c, scale=scale)
+    for k in want:
+        compare(got[k], want[k], wl, f"fp8 every code {k}")
+    # each 128-column group on its own, so that an error confined to one
+    # group's widening is not diluted by the other groups' norm
+    for b in range(wl.B):
+        for g, (a, e) in enumerate(groups[:4]):
+            err = got["ctx_lat"][b][:, a:e] - want["ctx_lat"][b][:, a:e]
+            ref = np.linalg.norm(want["ctx_lat"][b][:, a:e])
+            assert np.linalg.norm(err) <= 5e-3 * max(ref, 1e-30), (b, g, np.linalg.norm(err) / ref)
