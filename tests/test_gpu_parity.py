@@ -208,6 +208,24 @@ def test_attention_many_short_sequences(name):
 
 
 @pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k"])
+def test_attention_more_sequences_than_plan_threads(name):
+    """1500 short sequences, more than the split plan's 1024 threads: each
+    thread scans two sequences (and the last threads none) in both prefix
+    scans; default split count, so every share spans many sequences."""
+    wl = WORKLOADS[name]
+    rng = np.random.default_rng(1500)
+    ctx = rng.integers(0, 48, size=1500)
+    ctx[::97] = 0
+    ctx[3::89] = 1
+    gc, gl, wc, wlse = _attention_only(wl, ctx.tolist(), 0)
+    seqs = [b for b in range(len(ctx)) if ctx[b] > 0]
+    compare(gc, wc, wl, "ctx_lat 1500 sequences", seqs)
+    compare(gl, wlse, wl, "lse 1500 sequences", seqs)
+    for b in np.nonzero(ctx == 0)[0]:
+        assert np.all(gc[b] == 0) and np.all(np.isneginf(gl[b]))
+
+
+@pytest.mark.parametrize("name", ["v2_b64_ctx8k", "v2lite_b32_ctx4k"])
 def test_attention_late_dominant_key(name):
     """A key far above the others late in the sequence forces the running
     maximum to jump (the rescale path)."""
