@@ -192,7 +192,8 @@ int mla_absorb_q(mla_handle *handle, const void *q_nope, const void *q_rope, con
 size_t mla_decode_workspace_size(const mla_handle *handle, int B, int num_parts);
 
 /* Default number of work partitions for this handle (depends on the kernel
- * selected for the configuration and on the device's SM count). */
+ * selected for the configuration and on the device's SM count); 0 for a NULL
+ * handle. */
 int mla_default_num_parts(const mla_handle *handle);
 
 /* Split-KV decode attention over the latent cache (V3 note: o_{t,i} with the

@@ -88,6 +88,50 @@ def test_create_without_device_fails_cleanly(lib):
                                    None) == M.MLA_ERR_INVALID_ARG
 
 
+# Entry points that take the handle first and answer a query instead of a
+# status: their documented value for a NULL handle.
+NULL_HANDLE_QUERIES = {
+    "mla_decode_workspace_size": 0,
+    "mla_cache_append_fp8_workspace_size": 0,
+    "mla_default_num_parts": 0,
+    "mla_fp8_scale_groups": 0,
+    "mla_plan_tile": -1,
+}
+NOT_HANDLE_FIRST = {"mla_status_string", "mla_config_validate", "mla_create", "mla_destroy",
+                    "mla_plan_pieces", "mla_plan_pieces_tiled", "mla_noalloc_scratch_bytes"}
+
+
+def null_handle_args(fn):
+    """Arguments for a call with a NULL handle: NULL pointers, batch and
+    counts of 1, sizes of 0, the scalars 1."""
+    out = []
+    for t in fn.argtypes:
+        if t is ctypes.c_void_p or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+            out.append(None)
+        elif t is ctypes.c_size_t:
+            out.append(0)
+        elif t is ctypes.c_double:
+            out.append(1.0)
+        else:
+            out.append(1)
+    return out
+
+
+def test_every_entry_point_rejects_a_null_handle(lib):
+    """The header's convention: a NULL handle is rejected on the host before
+    any CUDA call (here, with no device, a CUDA call would fail differently):
+    MLA_ERR_INVALID_ARG from every status-returning entry point, the
+    documented value from the queries."""
+    names = [n for n in declared_functions() if n not in NOT_HANDLE_FIRST]
+    assert len(names) >= 20
+    for name in names:
+        fn = getattr(lib, name)
+        assert fn.argtypes and fn.argtypes[0] is ctypes.c_void_p, name
+        got = fn(*null_handle_args(fn))
+        want = NULL_HANDLE_QUERIES.get(name, M.MLA_ERR_INVALID_ARG)
+        assert got == want, (name, got, want)
+
+
 def python_plan(ctx, P, tile=64):
     """Independent restatement of the split plan for checking the library's."""
     tiles = [(c + tile - 1) // tile for c in ctx]
