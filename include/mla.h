@@ -405,7 +405,8 @@ int mla_quantize_rows_fp8(mla_handle *handle, const void *rows, long long n_rows
  * mla_decode_attn.  16 or 32 heads at d_c = 512, d_r = 64 run on the tensor
  * cores (the codes are widened to bf16 in shared memory, code * sigma rounded
  * to bf16); every other shape, 128 heads included, on the CUDA-core kernel,
- * which is functional but not fast.  kv_scale NULL is MLA_ERR_INVALID_ARG. */
+ * which is functional but hundreds of times slower than the bf16 tensor-core
+ * path at DeepSeek-V2 shapes.  kv_scale NULL is MLA_ERR_INVALID_ARG. */
 int mla_decode_attn_fp8(mla_handle *handle, const void *q_abs, const void *cache, const float *kv_scale,
                         long long cache_len, const int *block_table, int max_blocks_per_seq,
                         const int *ctx_len, int B, int num_parts, void *workspace, size_t ws_bytes,
