@@ -13,6 +13,8 @@ import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from head_latent_attention_09_b200.splitkv import TILE, token_ranges
 
@@ -29,6 +31,22 @@ def test_token_ranges_partition_each_sequence(world):
         assert np.array_equal(toks, np.arange(c)), (world, c)
         tiles = np.ceil((end[:, b] - begin[:, b]) / TILE)
         assert tiles.max() - tiles.min() <= 1
+
+
+@settings(max_examples=60, deadline=None, derandomize=True)
+@given(ctx=st.lists(st.integers(0, 300_000), min_size=1, max_size=12), world=st.integers(1, 16),
+       tile=st.sampled_from([64, 128, 256]))
+def test_token_ranges_partition_any_lengths(ctx, world, tile):
+    """The same properties for drawn lengths, world sizes and tiles: the
+    ranges cover each sequence exactly, in rank order, every begin on a tile,
+    and the tile counts of the ranks differ by at most one."""
+    ctx = np.array(ctx)
+    begin, end = token_ranges(ctx, world, tile)
+    assert np.all(begin % tile == 0) and np.all(begin <= end)
+    assert np.all(begin[0] == 0) and np.array_equal(end[-1], ctx)
+    assert np.array_equal(begin[1:], end[:-1])
+    tiles = (end - begin + tile - 1) // tile
+    assert np.all(tiles.max(axis=0) - tiles.min(axis=0) <= 1)
 
 
 def _free_port() -> int:
