@@ -8,6 +8,8 @@ import re
 
 import numpy as np
 import pytest
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
 
 import head_latent_attention_09_b200 as M
 from head_latent_attention_09_b200 import build as B
@@ -195,3 +197,16 @@ def test_plan_v2_workload(lib):
     assert all(base[b + 1] - base[b] >= 1 for b in range(64))
     assert M.mla_plan_pieces([], 5)[0] == 0
     assert lib.mla_plan_pieces(None, 0, 1, None) == -1
+
+
+@settings(max_examples=50, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(ctx=st.lists(st.integers(0, 20_000), min_size=1, max_size=120), P=st.integers(1, 600),
+       tile=st.sampled_from([64, 128, 256]))
+def test_tiled_plan_matches_restatement_for_any_batch(lib, ctx, P, tile):
+    """The library's split plan against the restatement over drawn batches,
+    split counts (more or fewer than the tiles) and tiles."""
+    n, base = M.mla_plan_pieces_tiled(ctx, P, tile)
+    n2, base2, _ = python_plan(ctx, P, tile)
+    assert n == n2 and base == base2
+    assert n <= P + len(ctx)
